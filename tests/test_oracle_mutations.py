@@ -1,0 +1,96 @@
+"""Planted mistakes in copies of the oracle must fail the pins.
+
+Each case compiles a mutated copy of oracle/fp8bl_oracle.c into a temporary
+library, swaps it in for the real one, and checks that at least one pin of
+the relevant kind fails.  This shows the pins are sensitive to the plausible
+errors they are meant to catch (a dropped term, a transposed index, the
+reciprocal instead of the division, a wrong rounding).
+"""
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads as wl
+from tests import test_oracle_gemm as tg
+from tests import test_oracle_quant as tq
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "oracle", "fp8bl_oracle.c")
+
+
+def _build_mutant(tmp_path, old, new):
+    src = open(SRC).read()
+    assert old in src, old
+    p = tmp_path / "mutant.c"
+    p.write_text(src.replace(old, new, 1))
+    so = str(tmp_path / "libmutant.so")
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off",
+                    "-fPIC", "-shared", "-pthread", str(p), "-o", so, "-lm"], check=True)
+    return oracle.bind(so)
+
+
+def _fails(fn):
+    try:
+        fn()
+    except AssertionError:
+        return True
+    return False
+
+
+QUANT_MUTANTS = [
+    # multiply by the reciprocal instead of dividing
+    ("oracle_e4m3_encode(bf16_to_f32(xg[i]) / sc)", "oracle_e4m3_encode(bf16_to_f32(xg[i]) * (1.0f / sc))"),
+    # amax taken without the absolute value
+    ("float a = fabsf(bf16_to_f32(xg[i]));", "float a = bf16_to_f32(xg[i]);"),
+    # scale off by the e4m3 max (uses 240, the e4m3fnuz max)
+    ("#define OR_E4M3_MAX 448.0f", "#define OR_E4M3_MAX 240.0f"),
+    # amax window misplaced (stride 64 instead of 128, stays in bounds)
+    ("const uint16_t *xg = x + m * K + g * OR_BLOCK;", "const uint16_t *xg = x + m * K + g * 64;"),
+]
+
+
+@pytest.mark.parametrize("old,new", QUANT_MUTANTS)
+def test_quant_pins_catch(tmp_path, monkeypatch, old, new):
+    lib = _build_mutant(tmp_path, old, new)
+    monkeypatch.setattr(oracle, "_lib", lib)
+    checks = [
+        lambda: tq.test_quant_act_vs_library_composition((32, 512), 0),
+        lambda: tq.test_quant_act_heavy_tails_and_zero_groups(),
+        lambda: tq.test_amax_element_maps_to_448(),
+    ]
+    assert any(_fails(c) for c in checks)
+
+
+GEMM_MUTANTS = [
+    # transposed weight-scale index
+    ("(double)jb->sw[(n / OR_BLOCK) * KB + j]", "(double)jb->sw[j * (N / OR_BLOCK) + (n / OR_BLOCK) % KB]"),
+    # activation scale of the wrong K block
+    ("(double)jb->sa[m * KB + j]", "(double)jb->sa[m * KB]"),
+    # dropped last K block
+    ("for (int64_t j = 0; j < KB; ++j) {", "for (int64_t j = 0; j + 1 < KB; ++j) {"),
+    # off-by-one K range inside a block
+    ("k < (j + 1) * OR_BLOCK; ++k)", "k < (j + 1) * OR_BLOCK - 1; ++k)"),
+]
+
+
+@pytest.mark.parametrize("old,new", GEMM_MUTANTS)
+def test_gemm_pins_catch(tmp_path, monkeypatch, old, new):
+    lib = _build_mutant(tmp_path, old, new)
+    monkeypatch.setattr(oracle, "_lib", lib)
+    checks = [
+        lambda: tg.test_gemm_vs_exact_rationals(256),
+        lambda: tg.test_unit_scales_reduce_to_integer_matmul(),
+        lambda: tg.test_block_sums_exact_per_block(),
+        lambda: tg.test_scale_linearity_and_block_index(),
+    ]
+    assert any(_fails(c) for c in checks)
+
+
+def test_real_oracle_passes_same_checks():
+    tq.test_quant_act_vs_library_composition((32, 512), 0)
+    tg.test_gemm_vs_exact_rationals(256)
+    assert np.all(np.isfinite(oracle.block_linear(*tg._random_case(2, 128, 128, 0))))
+    assert wl.tiny()[0].shape == (32, 512)
