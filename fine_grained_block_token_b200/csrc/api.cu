@@ -1,0 +1,215 @@
+// C-ABI entry points of libfp8bl (declared in include/fp8bl.h): argument
+// validation on the host, schedule choice, launch on the caller's stream,
+// and status reporting.  No call allocates device memory.
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+#include <mutex>
+
+#include "../../include/fp8bl.h"
+#include "fp8bl_internal.h"
+
+namespace fp8bl {
+namespace {
+
+// Error word written by kernels whose bounded waits ran out.  One int per
+// device image of this library; read and cleared by fp8bl_check().
+__device__ int g_kernel_error;
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_info[kMaxDevices];
+std::once_flag g_once[kMaxDevices];
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+bool dim_ok(int64_t v, bool allow_zero) {
+  return (allow_zero ? v >= 0 : v > 0) && v <= FP8BL_MAX_DIM;
+}
+
+cudaStream_t as_cuda(fp8bl_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+fp8bl_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FP8BL_OK : FP8BL_ERR_CUDA; }
+
+// Common checks: device architecture; returns the device facts.
+fp8bl_status current_device(const DeviceInfo** out) {
+  const DeviceInfo* d = device_info();
+  if (!d) return FP8BL_ERR_CUDA;
+  if (d->major != 10 || d->minor != 0) return FP8BL_ERR_ARCH;
+  *out = d;
+  return FP8BL_OK;
+}
+
+}  // namespace
+
+const DeviceInfo* device_info() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::call_once(g_once[dev], [dev] {
+    DeviceInfo& d = g_info[dev];
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return;
+    d.sm_count = v;
+    cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    d.max_smem_optin = static_cast<size_t>(v);
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kernel_error) != cudaSuccess) return;
+    d.error_flag = static_cast<int*>(p);
+    d.device = dev;
+  });
+  const DeviceInfo* d = &g_info[dev];
+  return d->device == dev ? d : nullptr;
+}
+
+}  // namespace fp8bl
+
+using namespace fp8bl;
+
+extern "C" {
+
+int fp8bl_version(void) { return 100; }
+
+const char* fp8bl_status_string(fp8bl_status s) {
+  switch (s) {
+    case FP8BL_OK: return "ok";
+    case FP8BL_ERR_NULL: return "a required pointer is NULL";
+    case FP8BL_ERR_SHAPE: return "invalid sizes (need K, N multiples of 128, within limits)";
+    case FP8BL_ERR_ALIGN: return "pointer not 16-byte aligned (4-byte for scales)";
+    case FP8BL_ERR_ARCH: return "current device is not compute capability 10.0 (sm_100)";
+    case FP8BL_ERR_CUDA: return "CUDA call failed";
+    case FP8BL_ERR_TIMEOUT: return "a kernel wait ran out of time";
+    case FP8BL_ERR_WORKSPACE: return "workspace smaller than required";
+    case FP8BL_ERR_OVERLAP: return "an output buffer overlaps an input buffer";
+  }
+  return "unknown status";
+}
+
+fp8bl_status fp8_quant_act(const void* x_bf16, int64_t M, int64_t K, void* q_e4m3, float* s,
+                           fp8bl_stream_t stream) {
+  if (!dim_ok(M, true) || !dim_ok(K, false) || K % FP8BL_BLOCK) return FP8BL_ERR_SHAPE;
+  if (M == 0) return FP8BL_OK;
+  if (!x_bf16 || !q_e4m3 || !s) return FP8BL_ERR_NULL;
+  if (!aligned(x_bf16, 16) || !aligned(q_e4m3, 16) || !aligned(s, 4)) return FP8BL_ERR_ALIGN;
+  const size_t nx = static_cast<size_t>(M * K) * 2, nq = static_cast<size_t>(M * K),
+               ns = static_cast<size_t>(M * (K / 128)) * 4;
+  if (overlap(x_bf16, nx, q_e4m3, nq) || overlap(x_bf16, nx, s, ns) || overlap(q_e4m3, nq, s, ns))
+    return FP8BL_ERR_OVERLAP;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  return from_cuda(launch_act_quant(x_bf16, M, K, q_e4m3, s, d->sm_count, as_cuda(stream)));
+}
+
+fp8bl_status fp8_quant_weight(const void* w_bf16, int64_t N, int64_t K, void* q_e4m3, float* s,
+                              fp8bl_stream_t stream) {
+  if (!dim_ok(N, false) || !dim_ok(K, false) || N % FP8BL_BLOCK || K % FP8BL_BLOCK)
+    return FP8BL_ERR_SHAPE;
+  if (!w_bf16 || !q_e4m3 || !s) return FP8BL_ERR_NULL;
+  if (!aligned(w_bf16, 16) || !aligned(q_e4m3, 16) || !aligned(s, 4)) return FP8BL_ERR_ALIGN;
+  const size_t nw = static_cast<size_t>(N * K) * 2, nq = static_cast<size_t>(N * K),
+               ns = static_cast<size_t>((N / 128) * (K / 128)) * 4;
+  if (overlap(w_bf16, nw, q_e4m3, nq) || overlap(w_bf16, nw, s, ns) || overlap(q_e4m3, nq, s, ns))
+    return FP8BL_ERR_OVERLAP;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  return from_cuda(launch_weight_quant(w_bf16, N, K, q_e4m3, s, as_cuda(stream)));
+}
+
+static bool linear_dims_ok(int64_t M, int64_t N, int64_t K) {
+  return dim_ok(M, true) && dim_ok(N, false) && dim_ok(K, false) && N % FP8BL_BLOCK == 0 &&
+         K % FP8BL_BLOCK == 0;
+}
+
+size_t fp8_block_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (!linear_dims_ok(M, N, K)) return 0;
+  const DeviceInfo* d = device_info();
+  return plan_block_linear(M, N, K, d ? d->sm_count : 148, false).workspace;
+}
+
+size_t fp8_block_linear_fused_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (!linear_dims_ok(M, N, K)) return 0;
+  const DeviceInfo* d = device_info();
+  return plan_block_linear(M, N, K, d ? d->sm_count : 148, true).workspace;
+}
+
+fp8bl_status fp8_block_linear(const void* q_a, const float* s_a, const void* q_w,
+                              const float* s_w, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                              void* workspace, size_t workspace_bytes, fp8bl_stream_t stream) {
+  if (!linear_dims_ok(M, N, K)) return FP8BL_ERR_SHAPE;
+  if (M == 0) return FP8BL_OK;
+  if (!q_a || !s_a || !q_w || !s_w || !y_bf16) return FP8BL_ERR_NULL;
+  if (!aligned(q_a, 16) || !aligned(q_w, 16) || !aligned(y_bf16, 16) || !aligned(s_a, 4) ||
+      !aligned(s_w, 4) || !aligned(workspace, 16))
+    return FP8BL_ERR_ALIGN;
+  const size_t ny = static_cast<size_t>(M * N) * 2;
+  if (overlap(y_bf16, ny, q_a, static_cast<size_t>(M * K)) ||
+      overlap(y_bf16, ny, q_w, static_cast<size_t>(N * K)) ||
+      overlap(y_bf16, ny, s_a, static_cast<size_t>(M * (K / 128)) * 4) ||
+      overlap(y_bf16, ny, s_w, static_cast<size_t>((N / 128) * (K / 128)) * 4))
+    return FP8BL_ERR_OVERLAP;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  const GemmPlan plan = plan_block_linear(M, N, K, d->sm_count, false);
+  if (plan.workspace > 0) {
+    if (!workspace) return FP8BL_ERR_NULL;
+    if (workspace_bytes < plan.workspace) return FP8BL_ERR_WORKSPACE;
+    if (overlap(workspace, plan.workspace, y_bf16, ny)) return FP8BL_ERR_OVERLAP;
+  }
+  return from_cuda(launch_block_linear(q_a, s_a, q_w, s_w, y_bf16, M, N, K, plan, workspace, *d,
+                                       as_cuda(stream)));
+}
+
+fp8bl_status fp8_block_linear_fused(const void* x_bf16, const void* q_w, const float* s_w,
+                                    void* y_bf16, int64_t M, int64_t N, int64_t K, void* workspace,
+                                    size_t workspace_bytes, fp8bl_stream_t stream) {
+  if (!linear_dims_ok(M, N, K)) return FP8BL_ERR_SHAPE;
+  if (M == 0) return FP8BL_OK;
+  if (!x_bf16 || !q_w || !s_w || !y_bf16) return FP8BL_ERR_NULL;
+  if (!aligned(x_bf16, 16) || !aligned(q_w, 16) || !aligned(y_bf16, 16) || !aligned(s_w, 4) ||
+      !aligned(workspace, 16))
+    return FP8BL_ERR_ALIGN;
+  const size_t ny = static_cast<size_t>(M * N) * 2;
+  if (overlap(y_bf16, ny, x_bf16, static_cast<size_t>(M * K) * 2) ||
+      overlap(y_bf16, ny, q_w, static_cast<size_t>(N * K)) ||
+      overlap(y_bf16, ny, s_w, static_cast<size_t>((N / 128) * (K / 128)) * 4))
+    return FP8BL_ERR_OVERLAP;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  const GemmPlan plan = plan_block_linear(M, N, K, d->sm_count, true);
+  if (plan.workspace > 0) {
+    if (!workspace) return FP8BL_ERR_NULL;
+    if (workspace_bytes < plan.workspace) return FP8BL_ERR_WORKSPACE;
+    if (overlap(workspace, plan.workspace, y_bf16, ny) ||
+        overlap(workspace, plan.workspace, x_bf16, static_cast<size_t>(M * K) * 2))
+      return FP8BL_ERR_OVERLAP;
+  }
+  return from_cuda(launch_block_linear_fused(x_bf16, q_w, s_w, y_bf16, M, N, K, plan, workspace,
+                                             *d, as_cuda(stream)));
+}
+
+fp8bl_status fp8bl_check(fp8bl_stream_t stream) {
+  if (cudaStreamSynchronize(as_cuda(stream)) != cudaSuccess) return FP8BL_ERR_CUDA;
+  const DeviceInfo* d = device_info();
+  if (!d) return FP8BL_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, d->error_flag, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return FP8BL_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpy(d->error_flag, &zero, sizeof zero, cudaMemcpyHostToDevice);
+    return FP8BL_ERR_TIMEOUT;
+  }
+  return FP8BL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the
+// kernel translation units.  Every launcher assumes the arguments were
+// validated by the C-ABI layer.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp8bl {
+
+struct DeviceInfo {
+  int device = -1;
+  int sm_count = 0;
+  int major = 0, minor = 0;
+  size_t max_smem_optin = 0;
+  int* error_flag = nullptr;   // device address of the kernel error word
+};
+
+// Per-device facts and the error-flag address (cached, thread-safe).
+// Returns nullptr if the current device cannot be queried.
+const DeviceInfo* device_info();
+
+// Activation quantization, bf16 [M,K] -> e4m3 [M,K] + fp32 [M,K/128].
+cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float* s,
+                             int sm_count, cudaStream_t st);
+
+// Weight quantization, bf16 [N,K] -> e4m3 [N,K] + fp32 [N/128,K/128].
+cudaError_t launch_weight_quant(const void* w, int64_t N, int64_t K, void* q, float* s,
+                                cudaStream_t st);
+
+// GEMM schedule, chosen on the host from the sizes.
+struct GemmPlan {
+  int kind = 0;          // 0 = prefill tile kernel, 1 = decode (swap-AB) kernel
+  int split_k = 1;       // number of K slices (decode / small grids)
+  size_t workspace = 0;  // bytes of fp32 partials needed
+};
+
+GemmPlan plan_block_linear(int64_t M, int64_t N, int64_t K, int sm_count, bool fused);
+
+cudaError_t launch_block_linear(const void* q_a, const float* s_a, const void* q_w,
+                                const float* s_w, void* y, int64_t M, int64_t N, int64_t K,
+                                const GemmPlan& plan, void* workspace, const DeviceInfo& dev,
+                                cudaStream_t st);
+
+cudaError_t launch_block_linear_fused(const void* x, const void* q_w, const float* s_w, void* y,
+                                      int64_t M, int64_t N, int64_t K, const GemmPlan& plan,
+                                      void* workspace, const DeviceInfo& dev, cudaStream_t st);
+
+// Error codes a kernel writes into the error word (first error wins).
+enum KernelError : int {
+  kErrNone = 0,
+  kErrTimeoutProducer = 1,
+  kErrTimeoutMma = 2,
+  kErrTimeoutEpilogue = 3,
+};
+
+}  // namespace fp8bl

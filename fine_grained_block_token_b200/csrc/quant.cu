@@ -1,0 +1,137 @@
+// Activation (1 x 128 per token) and weight (128 x 128) e4m3 quantization
+// kernels.  "Fine-grained FP8" page, opening bullet list: weights per
+// 128 x 128 block, activations per token in groups of 128 input channels.
+//
+// Activation kernel: with K % 128 == 0 the 1 x 128 groups of a row-major
+// [M, K] tensor are consecutive 256-byte chunks of the flat array, and the
+// scale of group g sits at s[g] of the row-major [M, K/128] scale tensor.
+// The kernel is therefore a flat stream over groups: a half-warp owns one
+// group (16 lanes x 16 bytes), reduces amax with four xor-shuffles, and
+// writes 8 bytes of codes per lane (the warp writes 256 contiguous bytes)
+// plus one scale.  Each warp keeps UNROLL pairs of groups in flight so the
+// SM has enough bytes outstanding to run at HBM bandwidth.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fp8bl_internal.h"
+#include "quant_math.cuh"
+
+namespace fp8bl {
+namespace {
+
+constexpr int kAqThreads = 256;
+constexpr int kAqUnroll = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// num_groups = M * K / 128.  x: 16 uint4 per group; q: 16 uint2 per group.
+__global__ void __launch_bounds__(kAqThreads)
+act_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, float* __restrict__ s,
+                 int64_t num_groups) {
+  const int lane = threadIdx.x & 31;
+  const int half = lane >> 4;
+  const int l16 = lane & 15;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kAqThreads + threadIdx.x) >> 5;
+  const int64_t num_warps = (static_cast<int64_t>(gridDim.x) * kAqThreads) >> 5;
+  const int64_t num_pairs = (num_groups + 1) >> 1;
+  // The loop bound depends on the warp only, so every shuffle below runs
+  // with all 32 lanes present.
+  for (int64_t p0 = warp; p0 < num_pairs; p0 += num_warps * kAqUnroll) {
+    uint4 v[kAqUnroll];
+#pragma unroll
+    for (int u = 0; u < kAqUnroll; ++u) {
+      const int64_t g = (p0 + u * num_warps) * 2 + half;
+      v[u] = g < num_groups ? ld_stream(x + g * 16 + l16) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kAqUnroll; ++u) {
+      const int64_t g = (p0 + u * num_warps) * 2 + half;
+      float a = amax8(v[u]);
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      const float sc = scale_from_amax(a);
+      const float r = __frcp_rn(sc);
+      const uint2 o = quant8(v[u], sc, r);
+      if (g < num_groups) {
+        q[g * 16 + l16] = o;
+        if (l16 == 0) s[g] = sc;
+      }
+    }
+  }
+}
+
+// One CTA per 128 x 128 block.  Thread t covers 16-byte chunk (t % 16) of
+// rows (t / 16) + 16 i, i = 0..7: every load instruction of a warp reads two
+// full 256-byte row segments.
+constexpr int kWqThreads = 256;
+
+__global__ void __launch_bounds__(kWqThreads)
+weight_quant_kernel(const uint4* __restrict__ w, uint2* __restrict__ q, float* __restrict__ s,
+                    int64_t K, int64_t KB) {
+  __shared__ float warp_amax[kWqThreads / 32];
+  const int64_t blk = blockIdx.x;
+  const int64_t bi = blk / KB, bj = blk % KB;
+  const int c = threadIdx.x & 15;
+  const int r0 = threadIdx.x >> 4;
+  const int64_t row_stride = K / 8;   // uint4 per row
+  const int64_t base = (bi * 128 + r0) * row_stride + bj * 16 + c;
+  uint4 v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = ld_stream(w + base + static_cast<int64_t>(16 * i) * row_stride);
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, amax8(v[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((threadIdx.x & 31) == 0) warp_amax[threadIdx.x >> 5] = a;
+  __syncthreads();
+  a = warp_amax[0];
+#pragma unroll
+  for (int i = 1; i < kWqThreads / 32; ++i) a = fmaxf(a, warp_amax[i]);
+  const float sc = scale_from_amax(a);
+  const float r = __frcp_rn(sc);
+  const int64_t qrow_stride = K / 8;  // uint2 per row
+  const int64_t qbase = (bi * 128 + r0) * qrow_stride + bj * 16 + c;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[qbase + static_cast<int64_t>(16 * i) * qrow_stride] = quant8(v[i], sc, r);
+  if (threadIdx.x == 0) s[bi * KB + bj] = sc;
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float* s,
+                             int sm_count, cudaStream_t st) {
+  const int64_t groups = M * (K / 128);
+  if (groups == 0) return cudaSuccess;
+  const int64_t pairs = (groups + 1) / 2;
+  const int64_t warps_needed = (pairs + kAqUnroll - 1) / kAqUnroll;
+  const int64_t blocks_needed = (warps_needed + (kAqThreads / 32) - 1) / (kAqThreads / 32);
+  // At most 4 resident CTAs per SM worth of work per pass; larger inputs
+  // loop inside the kernel.
+  const int64_t max_blocks = static_cast<int64_t>(sm_count) * 4;
+  const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
+  act_quant_kernel<<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
+                                                  static_cast<uint2*>(q), s, groups);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_weight_quant(const void* w, int64_t N, int64_t K, void* q, float* s,
+                                cudaStream_t st) {
+  const int64_t KB = K / 128;
+  const int64_t blocks = (N / 128) * KB;
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
+  weight_quant_kernel<<<static_cast<unsigned>(blocks), kWqThreads, 0, st>>>(
+      static_cast<const uint4*>(w), static_cast<uint2*>(q), s, K, KB);
+  return cudaGetLastError();
+}
+
+}  // namespace fp8bl

@@ -1,0 +1,163 @@
+/*
+ * fp8bl -- fine-grained (block-scaled) FP8 linear layers for NVIDIA B200
+ * (sm_100a).  C ABI.
+ *
+ * The method (transformers docs, "Fine-grained FP8" page, opening bullet
+ * list, and its "DeepGEMM fast path" section):
+ *   - weights are quantized to 8 bits per two-dimensional 128 x 128 block,
+ *     one scale per block;
+ *   - activations are quantized dynamically (at run time), per token, in
+ *     groups of 128 input channels aligned with the weight blocks, one scale
+ *     per (token, group);
+ *   - the linear layer multiplies the quantized operands and applies both
+ *     scale sets per 128-deep block of the input channel.
+ * The pages leave the numerics open; this library implements:
+ *   - e4m3 = OCP FP8 E4M3 (torch.float8_e4m3fn): max finite 448, NaN = S.1111.111;
+ *   - scale s = fp32(max(amax, FP8BL_AMAX_EPS) / 448), amax = max |x| over
+ *     the group or block; scales are fp32;
+ *   - q = e4m3(fp32(x / s)) with an IEEE-rounded fp32 quotient, then round to
+ *     nearest even and saturate to +-448;
+ *   - y[m,n] = bf16( sum_j s_a[m,j] * s_w[n/128,j] *
+ *                    sum_{k in block j} e4m3val(q_a[m,k]) * e4m3val(q_w[n,k]) )
+ *     accumulated in fp32 (fp32 partial per 128-deep block, promoted with
+ *     the product of the two scales), rounded once to bf16 (nearest even).
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers to caller-owned memory on the current
+ *     CUDA device; the library never allocates, frees or keeps them.
+ *   - All tensors are dense and row-major (last index fastest).
+ *   - Every pointer must be 16-byte aligned (fp32 scale arrays: 4-byte).
+ *   - Outputs must not overlap inputs.
+ *   - Work is enqueued asynchronously on `stream` (NULL = legacy default
+ *     stream); the call returns before the GPU finishes.
+ *   - Argument errors are detected on the host and returned BEFORE any work
+ *     is enqueued.  Launch failures return FP8BL_ERR_CUDA.  Kernels whose
+ *     internal waits exceed their time limit record an error that
+ *     fp8bl_check() reports as FP8BL_ERR_TIMEOUT.
+ *   - Results are bit-identical from run to run for the same arguments.
+ *   - The device must be compute capability 10.0 (B200 / sm_100a).
+ *   - No exceptions cross this interface; all calls are thread-safe as long
+ *     as concurrent calls do not share output buffers or workspaces.
+ */
+#ifndef FP8BL_H
+#define FP8BL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; declared here so that this header
+ * does not need the CUDA headers. */
+typedef struct CUstream_st *fp8bl_stream_t;
+
+typedef enum {
+    FP8BL_OK = 0,
+    FP8BL_ERR_NULL = 1,      /* a required pointer is NULL                  */
+    FP8BL_ERR_SHAPE = 2,     /* sizes out of range / not multiples of 128   */
+    FP8BL_ERR_ALIGN = 3,     /* a pointer is not suitably aligned           */
+    FP8BL_ERR_ARCH = 4,      /* current device is not sm_100                */
+    FP8BL_ERR_CUDA = 5,      /* a CUDA runtime/driver call failed           */
+    FP8BL_ERR_TIMEOUT = 6,   /* a kernel wait ran out (see fp8bl_check)     */
+    FP8BL_ERR_WORKSPACE = 7, /* workspace smaller than required             */
+    FP8BL_ERR_OVERLAP = 8    /* an output buffer overlaps an input buffer   */
+} fp8bl_status;
+
+#define FP8BL_BLOCK 128          /* group / block edge along K and N       */
+#define FP8BL_E4M3_MAX 448.0f    /* largest finite e4m3 value              */
+#define FP8BL_AMAX_EPS 1e-10f    /* amax floor for all-zero groups/blocks  */
+
+/* Largest sizes accepted (TMA coordinates are 32-bit signed). */
+#define FP8BL_MAX_DIM ((int64_t)1 << 30)
+
+/*
+ * fp8_quant_act -- dynamic per-token activation quantization.
+ * Passage: "Fine-grained FP8" page, second bullet of the opening list
+ * (per-token groups whose size matches the weight block along the input
+ * channel, 128), dynamic scheme per its "DeepGEMM fast path" section.
+ *
+ *   x_bf16  in : bf16 [M, K] row-major
+ *   q_e4m3  out: e4m3 codes [M, K] row-major (1 byte each)
+ *   s       out: fp32 [M, K/128] row-major; s[m,g] scales x[m, 128g .. 128g+127]
+ *   M >= 0 (M == 0 enqueues nothing), K > 0, K % 128 == 0, M, K <= FP8BL_MAX_DIM.
+ */
+fp8bl_status fp8_quant_act(const void *x_bf16, int64_t M, int64_t K,
+                           void *q_e4m3, float *s, fp8bl_stream_t stream);
+
+/*
+ * fp8_quant_weight -- 128 x 128 block weight quantization.
+ * Passage: "Fine-grained FP8" page, first bullet of the opening list
+ * (weight_block_size = (128, 128)).
+ *
+ *   w_bf16  in : bf16 [N, K] row-major (nn.Linear layout: out x in)
+ *   q_e4m3  out: e4m3 codes [N, K]
+ *   s       out: fp32 [N/128, K/128] row-major; s[i,j] scales the block of
+ *                rows 128i.. and columns 128j..
+ *   N, K > 0, multiples of 128, <= FP8BL_MAX_DIM.
+ */
+fp8bl_status fp8_quant_weight(const void *w_bf16, int64_t N, int64_t K,
+                              void *q_e4m3, float *s, fp8bl_stream_t stream);
+
+/*
+ * fp8_block_linear -- block-scaled FP8 linear, y = x W^T with both scale
+ * sets applied per 128-deep K block.
+ * Passage: "Fine-grained FP8" page, opening bullet list (the two
+ * quantization granularities the product must honour) and "DeepGEMM fast
+ * path" section (FP8 linear with weight_block_size (128,128) and dynamic
+ * activations).
+ *
+ *   q_a  in : e4m3 [M, K]          (from fp8_quant_act)
+ *   s_a  in : fp32 [M, K/128]
+ *   q_w  in : e4m3 [N, K]          (from fp8_quant_weight)
+ *   s_w  in : fp32 [N/128, K/128]
+ *   y_bf16 out: bf16 [M, N]
+ *   workspace: device scratch of at least
+ *              fp8_block_linear_workspace_bytes(M, N, K) bytes (16-byte
+ *              aligned), or NULL when that size is 0.  Contents on entry
+ *              are ignored; the library may overwrite all of it.
+ *   M >= 0, N, K > 0 and multiples of 128, all <= FP8BL_MAX_DIM.
+ */
+fp8bl_status fp8_block_linear(const void *q_a, const float *s_a,
+                              const void *q_w, const float *s_w,
+                              void *y_bf16, int64_t M, int64_t N, int64_t K,
+                              void *workspace, size_t workspace_bytes,
+                              fp8bl_stream_t stream);
+
+/*
+ * fp8_block_linear_fused -- the same linear with the activation
+ * quantization done inside the GEMM: x_bf16 [M, K] is quantized exactly as
+ * fp8_quant_act would (bit-identical codes and scales) and multiplied
+ * without writing q_a / s_a to memory.  y equals
+ * fp8_quant_act + fp8_block_linear bit for bit.
+ *   workspace: at least fp8_block_linear_fused_workspace_bytes(M, N, K).
+ */
+fp8bl_status fp8_block_linear_fused(const void *x_bf16,
+                                    const void *q_w, const float *s_w,
+                                    void *y_bf16, int64_t M, int64_t N, int64_t K,
+                                    void *workspace, size_t workspace_bytes,
+                                    fp8bl_stream_t stream);
+
+/* Workspace sizes (bytes) the two linear calls need for these sizes on the
+ * current device; 0 when no scratch is needed.  Never fails: invalid sizes
+ * return 0 (the linear call then reports the error). */
+size_t fp8_block_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+size_t fp8_block_linear_fused_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Waits for `stream`, then reports (and clears) a kernel wait that ran out
+ * on the current device since the last check: FP8BL_ERR_TIMEOUT, else
+ * FP8BL_OK (or FP8BL_ERR_CUDA if the synchronisation itself failed). */
+fp8bl_status fp8bl_check(fp8bl_stream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char *fp8bl_status_string(fp8bl_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int fp8bl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BL_H */

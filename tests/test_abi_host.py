@@ -1,0 +1,125 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The library must load, export every function declared in include/fp8bl.h,
+and reject invalid arguments with the documented status BEFORE touching the
+device.  Calls with valid arguments need a GPU and live in the gpu tests.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8bl.h")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w \*]*?\b(fp8\w*)\s*\(", txt, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fine_grained_block_token_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_expected_calls():
+    names = _declared()
+    for n in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
+              "fp8_block_linear_workspace_bytes", "fp8bl_check", "fp8bl_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from fine_grained_block_token_b200 import build
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if ln.strip()}
+    for n in _declared():
+        assert n in exported, n
+        assert getattr(lib, n) is not None
+
+
+def test_status_strings(lib):
+    lib.fp8bl_status_string.restype = ctypes.c_char_p
+    for s in range(9):
+        assert lib.fp8bl_status_string(s)
+    assert lib.fp8bl_status_string(99) == b"unknown status"
+
+
+V = ctypes.c_void_p
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_quant_act_argument_errors(lib):
+    f = lib.fp8_quant_act
+    f.argtypes = [V, ctypes.c_int64, ctypes.c_int64, V, V, V]
+    good = _p(0x10000)
+    assert f(good, 4, 100, good, good, None) == 2          # K not multiple of 128
+    assert f(good, -1, 128, good, good, None) == 2         # negative M
+    assert f(good, 4, 0, good, good, None) == 2            # K == 0
+    assert f(good, 1, (1 << 31) * 128, good, good, None) == 2  # beyond FP8BL_MAX_DIM
+    assert f(good, 0, 128, None, None, None) == 0          # M == 0 is a no-op
+    assert f(None, 4, 128, good, good, None) == 1          # null input
+    assert f(_p(0x10008), 4, 128, good, _p(0x20000), None) == 3  # misaligned x
+    assert f(good, 4, 128, _p(0x20001), _p(0x30000), None) == 3  # misaligned q
+    assert f(good, 4, 128, _p(0x10100), _p(0x40000), None) == 8  # q overlaps x
+
+
+def test_quant_weight_argument_errors(lib):
+    f = lib.fp8_quant_weight
+    f.argtypes = [V, ctypes.c_int64, ctypes.c_int64, V, V, V]
+    g = _p(0x100000)
+    assert f(g, 100, 128, _p(0x200000), _p(0x300000), None) == 2   # N not multiple of 128
+    assert f(g, 128, 0, _p(0x200000), _p(0x300000), None) == 2
+    assert f(g, 128, 128, None, _p(0x300000), None) == 1
+    assert f(g, 128, 128, _p(0x200000), _p(0x300002), None) == 3  # misaligned scales
+
+
+def test_block_linear_argument_errors(lib):
+    f = lib.fp8_block_linear
+    f.argtypes = [V, V, V, V, V, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, V,
+                  ctypes.c_size_t, V]
+    a, sa, w, sw, y = (_p(0x1000000 * (i + 1)) for i in range(5))
+    assert f(a, sa, w, sw, y, 4, 100, 128, None, 0, None) == 2    # N % 128
+    assert f(a, sa, w, sw, y, 4, 128, 130, None, 0, None) == 2    # K % 128
+    assert f(a, sa, w, sw, y, 0, 128, 128, None, 0, None) == 0    # empty M
+    assert f(None, sa, w, sw, y, 4, 128, 128, None, 0, None) == 1
+    assert f(a, sa, w, sw, _p(0x5000008), 4, 128, 128, None, 0, None) == 3
+    assert f(a, sa, w, sw, a, 4, 128, 128, None, 0, None) == 8    # y aliases q_a
+
+
+def test_fused_argument_errors(lib):
+    f = lib.fp8_block_linear_fused
+    f.argtypes = [V, V, V, V, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, V, ctypes.c_size_t, V]
+    x, w, sw, y = (_p(0x1000000 * (i + 1)) for i in range(4))
+    assert f(x, w, sw, y, 4, 128, 120, None, 0, None) == 2
+    assert f(x, None, sw, y, 4, 128, 128, None, 0, None) == 1
+    assert f(x, w, sw, x, 4, 128, 128, None, 0, None) == 8
+
+
+def test_valid_call_without_gpu_reports_cuda_error(lib):
+    """With no usable device the library answers FP8BL_ERR_CUDA (or ARCH on
+    a non-B200 device) instead of crashing or falling back to the CPU."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    f = lib.fp8_quant_act
+    f.argtypes = [V, ctypes.c_int64, ctypes.c_int64, V, V, V]
+    assert f(_p(0x10000), 4, 128, _p(0x20000), _p(0x30000), None) in (4, 5)
+
+
+def test_workspace_query_never_fails(lib):
+    f = lib.fp8_block_linear_workspace_bytes
+    f.argtypes = [ctypes.c_int64] * 3
+    f.restype = ctypes.c_size_t
+    assert f(4, 100, 128) == 0
+    assert f(-1, 128, 128) == 0

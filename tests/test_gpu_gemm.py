@@ -1,0 +1,122 @@
+"""GPU parity of the block-scaled FP8 GEMM against the oracle's fp64 result,
+through the C ABI.
+
+Definition ("Fine-grained FP8" page of the transformers docs): both scale
+sets applied per 128-deep K block.  Quantized operands come from the GPU
+quantizers, which the quant tests hold bit-exact to the oracle; the oracle
+then computes R from the same codes and scales, and the GPU output must meet
+the tolerance in tests/parity.py.  Small shapes compare every element; the
+full workload sizes compare sampled rows (all N columns) in the launch
+configuration the benchmark uses.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from tests.parity import check_gemm, f32, to_dev, u8
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    import fine_grained_block_token_b200 as m
+    return m
+
+
+def _run(fp8, xbits, wbits, rows=None):
+    x, w = to_dev(xbits), to_dev(wbits)
+    q_a, s_a = fp8.quant_act(x)
+    q_w, s_w = fp8.quant_weight(w)
+    y = fp8.block_linear(q_a, s_a, q_w, s_w)
+    fp8.check()
+    qa, sa, qw, sw = u8(q_a), f32(s_a), u8(q_w), f32(s_w)
+    R = oracle.block_linear(qa, sa, qw, sw, rows=rows, nthreads=8)
+    yv = f32(y) if rows is None else f32(y[torch.as_tensor(rows, device=y.device)])
+    return yv, R, (x, q_a, s_a, q_w, s_w, y)
+
+
+def test_tiny(fp8):
+    xb, wb = wl.tiny()
+    y, R, _ = _run(fp8, xb, wb)
+    check_gemm(y, R, "tiny")
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (1, 128, 128), (5, 384, 256), (127, 256, 384), (129, 640, 1024), (300, 512, 512),
+    (64, 1024, 4096), (257, 768, 2048),
+])
+def test_ragged_shapes(fp8, M, N, K):
+    xb = wl.normal((M, K), 1.0, 0, M + N + K)
+    wb = wl.normal((N, K), 0.02, 1, M + N + K)
+    y, R, _ = _run(fp8, xb, wb)
+    check_gemm(y, R, f"{M}x{N}x{K}")
+
+
+def test_scale_extremes(fp8):
+    """Per-token magnitudes spanning 1e-4..1e4 and zeroed weight blocks."""
+    M, N, K = 192, 512, 1024
+    g = np.random.default_rng(5)
+    x = g.standard_normal((M, K)).astype(np.float32) * np.exp(g.uniform(-9, 9, (M, 1))).astype(np.float32)
+    xb = wl.f32_to_bf16_bits(x)
+    xb[7, 256:384] = 0
+    wb = wl.zero_blocks(wl.normal((N, K), 0.02, 2), 0.2)
+    y, R, _ = _run(fp8, xb, wb)
+    check_gemm(y, R, "extremes")
+
+
+def test_deterministic(fp8):
+    xb = wl.normal((200, 1024), 1.0, 3)
+    wb = wl.normal((768, 1024), 0.02, 4)
+    _, _, (x, q_a, s_a, q_w, s_w, y) = _run(fp8, xb, wb)
+    y2 = fp8.block_linear(q_a, s_a, q_w, s_w)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+def _sample_rows(M, n=48, seed=0):
+    g = np.random.default_rng(seed)
+    r = set([0, 1, M - 1, M // 2]) | set(g.choice(M, n, replace=False).tolist())
+    return np.array(sorted(r), dtype=np.int64)
+
+
+@pytest.mark.parametrize("which", ["llama3_prefill_gate_up", "llama3_prefill_down"])
+def test_full_size_prefill(fp8, which):
+    xb, wb = wl.llama3_prefill(which.split("prefill_")[1])
+    rows = _sample_rows(xb.shape[0], 24)
+    y, R, _ = _run(fp8, xb, wb, rows=rows)
+    check_gemm(y, R, which)
+
+
+@pytest.mark.parametrize("name", ["qo", "kv", "gate_up", "down"])
+@pytest.mark.parametrize("M", [1, 8, 64])
+def test_full_size_decode(fp8, name, M):
+    xb, wb = wl.llama3_decode(M, name)
+    y, R, _ = _run(fp8, xb, wb)
+    check_gemm(y, R, f"decode {name} M={M}")
+
+
+def test_full_size_deepseek_up(fp8):
+    xb, wb = wl.deepseek_mlp("up")
+    rows = _sample_rows(xb.shape[0], 12)
+    y, R, _ = _run(fp8, xb, wb, rows=rows)
+    check_gemm(y, R, "deepseek up")
+
+
+def test_fused_bit_identical(fp8):
+    for (M, N, K) in [(32, 256, 512), (129, 640, 1024), (1, 1024, 4096)]:
+        xb = wl.sweep_x(M, K)
+        wb = wl.normal((N, K), 0.02, 1)
+        x, w = to_dev(xb), to_dev(wb)
+        q_w, s_w = fp8.quant_weight(w)
+        q_a, s_a = fp8.quant_act(x)
+        y1 = fp8.block_linear(q_a, s_a, q_w, s_w)
+        y2 = fp8.block_linear_fused(x, q_w, s_w)
+        torch.cuda.synchronize()
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), (M, N, K)
+
+
+def test_no_timeout_recorded(fp8):
+    fp8.check()

@@ -1,0 +1,95 @@
+"""GPU parity: activation and weight quantization must match the oracle bit
+for bit (codes and fp32 scales), through the C ABI.
+
+Shapes cover the workloads ("Fine-grained FP8" page: 1x128 activation
+groups, 128x128 weight blocks) plus ragged and degenerate cases: a single
+row, odd row counts, one group per row, all-zero and negative-zero groups,
+huge and tiny magnitudes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from tests.parity import to_dev, u8, f32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    import fine_grained_block_token_b200 as m
+    return m
+
+
+def _check_act(fp8, bits, nthreads=8):
+    x = to_dev(bits)
+    q, s = fp8.quant_act(x)
+    torch.cuda.synchronize()
+    qo, so = oracle.quant_act(bits, nthreads=nthreads)
+    gq, gs = u8(q), f32(s)
+    assert np.array_equal(gs.view(np.uint32), so.view(np.uint32)), "scales differ"
+    bad = np.count_nonzero(gq != qo)
+    assert bad == 0, f"{bad} codes differ"
+
+
+@pytest.mark.parametrize("M,K", [(32, 512), (1, 128), (3, 384), (127, 256), (129, 1024),
+                                 (1, 4096), (8, 14336), (33, 7168), (64, 18432)])
+def test_act_quant_shapes(fp8, M, K):
+    _check_act(fp8, wl.normal((M, K), 1.0, 0, M * 7 + K))
+
+
+def test_act_quant_edge_values(fp8):
+    bits = wl.student_t_outliers(40, 1024, 3.0, 0.01, 100.0)
+    bits[0, :128] = 0                       # all-zero group
+    bits[1, 128:256] = 0x8000               # all -0.0
+    bits[2, 256:384] = 0x0001               # bf16 denormals
+    bits[3, 384:512] = 0x7F7F               # bf16 max
+    bits[4, 512:640] = wl.f32_to_bf16_bits(np.full(128, 1e-38, np.float32))
+    bits[5, :] = wl.f32_to_bf16_bits(np.linspace(-3e30, 3e30, 1024).astype(np.float32))
+    bits[6, 0:128] = wl.f32_to_bf16_bits(np.float32(2.0) ** -np.arange(128, dtype=np.float32))
+    _check_act(fp8, bits)
+
+
+def test_act_quant_empty(fp8):
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    q, s = fp8.quant_act(x)
+    assert q.shape == (0, 256) and s.shape == (0, 2)
+
+
+@pytest.mark.parametrize("name", ["prefill_gate_up", "prefill_down", "sweep_16384"])
+def test_act_quant_full_size(fp8, name):
+    if name == "prefill_gate_up":
+        bits, _ = wl.llama3_prefill("gate_up")
+    elif name == "prefill_down":
+        bits, _ = wl.llama3_prefill("down")
+    else:
+        bits = wl.sweep_x(16384)
+    _check_act(fp8, bits)
+
+
+def test_act_quant_deepseek_full_size(fp8):
+    bits, _ = wl.deepseek_mlp("down")       # X [8192, 18432]
+    _check_act(fp8, bits)
+
+
+def _check_weight(fp8, bits):
+    w = to_dev(bits)
+    q, s = fp8.quant_weight(w)
+    torch.cuda.synchronize()
+    qo, so = oracle.quant_weight(bits)
+    assert np.array_equal(f32(s).view(np.uint32), so.view(np.uint32))
+    assert np.array_equal(u8(q), qo)
+
+
+@pytest.mark.parametrize("N,K", [(256, 512), (128, 128), (384, 640), (1024, 4096)])
+def test_weight_quant_shapes(fp8, N, K):
+    bits = wl.normal((N, K), 0.02, 1, N + K)
+    bits = wl.zero_blocks(bits, 0.1)
+    _check_weight(fp8, bits)
+
+
+def test_weight_quant_full_size(fp8):
+    _, wbits = wl.deepseek_mlp("up")        # W [18432, 7168], 1% zero blocks
+    _check_weight(fp8, wbits)
