@@ -1,0 +1,426 @@
+"""Benchmark of the fine-grained FP8 linear hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload llama3_prefill|deepseek_mlp|llama3_decode|sweep]
+
+One step (default workload, Llama-3-8B MLP prefill, M = 4096 tokens):
+    quant_act(X1 [4096, 4096])   -> block_linear vs W_gate_up [28672, 4096]
+    quant_act(X2 [4096, 14336])  -> block_linear vs W_down    [4096, 14336]
+X ~ Student-t(df=4) with 0.5% of channels x50, W ~ N(0, 0.02), weights
+quantized once before timing (load time).  Inputs of a step (~330 MB) are
+larger than the 126 MB L2, so no flush is needed between steps.
+
+Prints ONE JSON line (rank 0).  `value` is whole-job TFLOP/s (2 M N K per
+linear, all ranks) over the device-timed K steps (CUDA events, max over
+ranks).  `e2e` repeats the measurement through the public API with the
+inputs copied from pinned host memory and the outputs copied back inside
+every step.  `roofline` covers the dominant kernel (the block-scaled GEMM)
+against the measured peaks in MEASURED_PEAKS.json.  `cpu_baseline` and
+`--impl reference` time the plain CPU oracle on a bounded row sample.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "block-scaled FP8 linear TFLOP/s (% FP8 peak); act-quant GB/s (% HBM peak)"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP8_OVER_BF16 = 2.0          # nominal dense ratio, 4.5 / 2.25 PFLOP/s
+
+
+# ----------------------------------------------------------------- workloads
+
+def workload_linears(name: str):
+    """[(label, x_bits [M,K], w_bits [N,K])] for one step of the workload."""
+    if name == "llama3_prefill":
+        return [(f"{n}", *wl.llama3_prefill(n)) for n in ("gate_up", "down")]
+    if name == "deepseek_mlp":
+        return [(f"{n}", *wl.deepseek_mlp(n)) for n in ("up", "down")]
+    if name == "llama3_decode":
+        out = []
+        for M in wl.DECODE_M:
+            for n in ("qo", "kv", "gate_up", "down"):
+                out.append((f"{n}_M{M}", *wl.llama3_decode(M, n)))
+        return out
+    if name == "sweep":
+        w = wl.sweep_w()
+        return [(f"M{M}", wl.sweep_x(M), w) for M in wl.SWEEP_M]
+    raise ValueError(name)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def gemm_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "ptx_sm100.cuh", "quant_math.cuh"):
+        h.update(open(os.path.join(ROOT, "fine_grained_block_token_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """dram bytes per launch from profiles/traffic.txt if the entry was taken
+    on the current kernel source, else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = gemm_source_sha()
+    for line in open(p):
+        if line.startswith("#") or not line.strip():
+            continue
+        kv = dict(tok.split("=", 1) for tok in line.split() if "=" in tok)
+        if kv.get("kernel") == kernel and kv.get("workload") == workload and kv.get("source_sha") == sha:
+            return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+# ------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- CPU side
+
+def cpu_prepare(lins, rows_per_linear: int, seed: int = 0):
+    """Load-time work of the CPU oracle: quantize the weights (not timed) and
+    pick the row sample of every linear."""
+    import oracle
+    prepared = []
+    for i, (label, xb, wb) in enumerate(lins):
+        qw, sw = oracle.quant_weight(wb)
+        g = np.random.default_rng([seed, i])
+        M = xb.shape[0]
+        rows = np.sort(g.choice(M, min(rows_per_linear, M), replace=False))
+        prepared.append((label, rows, np.ascontiguousarray(xb[rows]), qw, sw))
+    return prepared
+
+
+def cpu_step(prepared):
+    """One timed CPU step: the oracle's activation quantization of the sampled
+    rows and its fp64 block-scaled GEMM for them (all N columns).
+    Returns (seconds, flops, threads, {label: (rows, R)})."""
+    import oracle
+    threads = os.cpu_count() or 1
+    out = {}
+    t0 = time.perf_counter()
+    flops = 0
+    for label, rows, xs, qw, sw in prepared:
+        qa, sa = oracle.quant_act(xs, nthreads=threads)
+        out[label] = (rows, oracle.block_linear(qa, sa, qw, sw, nthreads=threads))
+        flops += 2 * xs.shape[0] * qw.shape[0] * qw.shape[1]
+    return time.perf_counter() - t0, flops, threads, out
+
+
+def sample_desc(prepared):
+    n = len(prepared[0][1]) if prepared else 0
+    return (f"{n} random rows per linear ({', '.join(p[0] for p in prepared)}), all N columns; "
+            "activation quant + fp64 GEMM of those rows; weights quantized before timing")
+
+
+def within_tolerance(y, R):
+    """GEMM tolerance: |y-R| <= 4e-3|R| + 1e-2 rms(R) pointwise.
+    Returns the worst ratio of |y-R| to its bound (<= 1 passes)."""
+    y = np.asarray(y, np.float64)
+    R = np.asarray(R, np.float64)
+    rms = float(np.sqrt(np.mean(R * R)))
+    lim = 4e-3 * np.abs(R) + 1e-2 * rms
+    return float(np.max(np.abs(y - R) / np.maximum(lim, 1e-300)))
+
+
+def run_reference(args):
+    """The oracle, as it stands, on the host cores: one bounded row sample of
+    the workload per step.  Under torchrun only rank 0 works."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    lins = workload_linears(args.workload)
+    prepared = cpu_prepare(lins, args.ref_rows)
+    for _ in range(args.warmup):
+        cpu_step(prepared)
+    tot_t, tot_f, thr = 0.0, 0, 1
+    for _ in range(args.steps):
+        t, f, thr, _ = cpu_step(prepared)
+        tot_t += t
+        tot_f += f
+    desc = sample_desc(prepared)
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------- GPU side
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import fine_grained_block_token_b200 as fp8
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    hbm_peak, bf16_peak, peak_src = peaks()
+    fp8_peak = bf16_peak * FP8_OVER_BF16
+
+    lins = workload_linears(args.workload)
+    items = []
+    for label, xb, wb in lins:
+        M, K = xb.shape
+        N = wb.shape[0]
+        x = wl.to_torch_bf16(xb).to(dev)
+        w = wl.to_torch_bf16(wb).to(dev)
+        q_w, s_w = fp8.quant_weight(w)
+        del w
+        q_a = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev)
+        s_a = torch.empty((M, K // 128), dtype=torch.float32, device=dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws_n = fp8.workspace_bytes(M, N, K)
+        ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
+        items.append(dict(label=label, xb=xb, x=x, q_w=q_w, s_w=s_w, q_a=q_a, s_a=s_a, y=y, ws=ws,
+                          M=M, N=N, K=K))
+    torch.cuda.synchronize()
+    flops_step = sum(2 * it["M"] * it["N"] * it["K"] for it in items)
+    act_bytes_step = sum(it["M"] * it["K"] * (2 + 1) + it["M"] * (it["K"] // 128) * 4 for it in items)
+    gemm_flops_step = flops_step
+
+    def step(ev=None):
+        for i, it in enumerate(items):
+            if ev is not None:
+                ev[4 * i].record()
+            fp8.quant_act(it["x"], it["q_a"], it["s_a"])
+            if ev is not None:
+                ev[4 * i + 1].record()
+                ev[4 * i + 2].record()
+            fp8.block_linear(it["q_a"], it["s_a"], it["q_w"], it["s_w"], it["y"], it["ws"])
+            if ev is not None:
+                ev[4 * i + 3].record()
+
+    for _ in range(args.warmup):
+        step()
+    fp8.check()
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+
+    # ---- device-timed region: K steps, per-kernel events inside
+    n = len(items)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4 * n)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    t_start.record()
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record()
+    barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    act_ms = sum(e[4 * i].elapsed_time(e[4 * i + 1]) for e in evs for i in range(n))
+    gemm_ms = sum(e[4 * i + 2].elapsed_time(e[4 * i + 3]) for e in evs for i in range(n))
+    fp8.check()
+
+    # ---- end to end: pinned host inputs in, outputs back, every step
+    host_x = [wl.to_torch_bf16(it["xb"]).pin_memory() for it in items]
+    host_y = [torch.empty((it["M"], it["N"]), dtype=torch.bfloat16).pin_memory() for it in items]
+    h2d = sum(t.numel() * 2 for t in host_x)
+    d2h = sum(t.numel() * 2 for t in host_y)
+
+    def e2e_step():
+        for it, hx, hy in zip(items, host_x, host_y):
+            it["x"].copy_(hx, non_blocking=True)
+            fp8.quant_act(it["x"], it["q_a"], it["s_a"])
+            fp8.block_linear(it["q_a"], it["s_a"], it["q_w"], it["s_w"], it["y"], it["ws"])
+            hy.copy_(it["y"], non_blocking=True)
+
+    for _ in range(min(args.warmup, 3)):
+        e2e_step()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier()
+    a.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record()
+    barrier()
+    e2e_ms = a.elapsed_time(b)
+    sampler.stop()
+    fp8.check()
+
+    # max over ranks
+    vals = torch.tensor([elapsed_ms, e2e_ms, act_ms, gemm_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms, act_ms, gemm_ms = vals.tolist()
+
+    ms_per_step = elapsed_ms / args.steps
+    value = world * flops_step * args.steps / (elapsed_ms * 1e-3) / 1e12
+    e2e_value = world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    gemm_tflops = gemm_flops_step * args.steps / (gemm_ms * 1e-3) / 1e12
+    act_gbs = act_bytes_step * args.steps / (act_ms * 1e-3) / 1e9
+    launches_per_step = 2 * n
+
+    if rank == 0:
+        parity = None
+        cpu = None
+        if world == 1 and not args.no_cpu:
+            # CPU-baseline leg: the oracle on a bounded row sample of the same
+            # input bits (it quantizes them itself); the GPU rows it covers
+            # are also checked against its result.
+            prepared = cpu_prepare(lins, args.cpu_rows)
+            t, f, thr, outs = cpu_step(prepared)
+            cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                   "sample": sample_desc(prepared), "seconds": t}
+            worst = 0.0
+            for it in items:
+                rows, R = outs[it["label"]]
+                Y = it["y"][torch.as_tensor(rows, device=dev)].float().cpu().numpy()
+                worst = max(worst, within_tolerance(Y, R))
+            parity = {"rows_per_linear": args.cpu_rows, "within_tolerance": worst <= 1.0,
+                      "worst_bound_ratio": worst}
+        traffic = recorded_traffic("gemm_prefill_kernel", args.workload)
+        gemm_ms_per_launch = gemm_ms / (args.steps * n)
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3", "data": "synthetic",
+            "config": {"workload": args.workload,
+                       "linears": {it["label"]: [it["M"], it["N"], it["K"]] for it in items},
+                       "l2": "no flush: inputs of a step exceed the 126 MB L2",
+                       "parallelism": f"replicas x{world} (no data-path collective)"},
+            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak,
+                         "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
+                         "traffic": traffic,
+                         "kernel": "gemm_prefill_kernel",
+                         "peak_source": f"{peak_src} bf16 burst x {FP8_OVER_BF16} (nominal fp8/bf16)",
+                         "ms_per_launch": gemm_ms_per_launch},
+            "act_quant": {"achieved": act_gbs, "peak": hbm_peak, "unit": "GB/s",
+                          "frac": act_gbs / hbm_peak, "peak_source": f"{peak_src} copy"},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": sampler.summary(),
+            "cpu_baseline": cpu,
+            "parity": parity,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama3_prefill",
+                    choices=["llama3_prefill", "deepseek_mlp", "llama3_decode", "sweep"])
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-rows", type=int, default=32)
+    ap.add_argument("--ref-rows", type=int, default=4)
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

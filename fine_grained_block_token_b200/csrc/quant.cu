@@ -31,7 +31,7 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 }
 
 // num_groups = M * K / 128.  x: 16 uint4 per group; q: 16 uint2 per group.
-__global__ void __launch_bounds__(kAqThreads)
+__global__ void __launch_bounds__(kAqThreads, 4)
 act_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, float* __restrict__ s,
                  int64_t num_groups) {
   const int lane = threadIdx.x & 31;
@@ -52,14 +52,13 @@ act_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, float* __re
 #pragma unroll
     for (int u = 0; u < kAqUnroll; ++u) {
       const int64_t g = (p0 + u * num_warps) * 2 + half;
-      float a = amax8(v[u]);
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-      const float sc = scale_from_amax(a);
-      const float r = __frcp_rn(sc);
-      const uint2 o = quant8(v[u], sc, r);
+      uint32_t m = absmax8_bf16x2(v[u]);
+      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 8));
+      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      const float sc = scale_from_amax(absmax_halves_f32(m));
+      const uint2 o = quant8(v[u], group_scale(sc));
       if (g < num_groups) {
         q[g * 16 + l16] = o;
         if (l16 == 0) s[g] = sc;
@@ -86,22 +85,23 @@ weight_quant_kernel(const uint4* __restrict__ w, uint2* __restrict__ q, float* _
   uint4 v[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = ld_stream(w + base + static_cast<int64_t>(16 * i) * row_stride);
-  float a = 0.0f;
+  uint32_t m = absmax8_bf16x2(v[0]);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) a = fmaxf(a, amax8(v[i]));
+  for (int i = 1; i < 8; ++i) m = absmax_bf16x2(m, absmax8_bf16x2(v[i]));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  for (int o = 16; o > 0; o >>= 1) m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float a = absmax_halves_f32(m);
   if ((threadIdx.x & 31) == 0) warp_amax[threadIdx.x >> 5] = a;
   __syncthreads();
   a = warp_amax[0];
 #pragma unroll
   for (int i = 1; i < kWqThreads / 32; ++i) a = fmaxf(a, warp_amax[i]);
   const float sc = scale_from_amax(a);
-  const float r = __frcp_rn(sc);
+  const GroupScale gs = group_scale(sc);
   const int64_t qrow_stride = K / 8;  // uint2 per row
   const int64_t qbase = (bi * 128 + r0) * qrow_stride + bj * 16 + c;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) q[qbase + static_cast<int64_t>(16 * i) * qrow_stride] = quant8(v[i], sc, r);
+  for (int i = 0; i < 8; ++i) q[qbase + static_cast<int64_t>(16 * i) * qrow_stride] = quant8(v[i], gs);
   if (threadIdx.x == 0) s[bi * KB + bj] = sc;
 }
 
@@ -114,7 +114,7 @@ cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float
   const int64_t pairs = (groups + 1) / 2;
   const int64_t warps_needed = (pairs + kAqUnroll - 1) / kAqUnroll;
   const int64_t blocks_needed = (warps_needed + (kAqThreads / 32) - 1) / (kAqThreads / 32);
-  // At most 4 resident CTAs per SM worth of work per pass; larger inputs
+  // One pass of resident CTAs (4 per SM at <= 64 registers); larger inputs
   // loop inside the kernel.
   const int64_t max_blocks = static_cast<int64_t>(sm_count) * 4;
   const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);

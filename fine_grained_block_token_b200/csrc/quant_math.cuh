@@ -7,14 +7,16 @@
 //   q = e4m3_rne_satfinite(fp32(x / s))
 // The quotient x / s is formed without a per-element IEEE division: with
 // r = fp32(1 / s) (IEEE reciprocal, once per group), q0 = fp32(x * r),
-// e = fma(-q0, s, x) (exact remainder) and q = fp32(q0 + e * r).  This is
-// Markstein's correction step (P. Markstein, "Computation of elementary
+// e = fma(q0, -s, x) (the exact remainder) and q = fp32(q0 + e * r).  This
+// is Markstein's correction step (P. Markstein, "Computation of elementary
 // functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
 // 1990): with r the correctly rounded reciprocal and q0 within one ulp it
-// returns the correctly rounded quotient.  The correction maps x = -0 to
-// +0, so the sign bit of x is put back at the end (e4m3 keeps -0 as 0x80).
-// The test suite checks the result exhaustively for every (amax, x) pair of
-// bf16 values that can occur.
+// yields the correctly rounded quotient.  The three operations run as
+// packed f32x2 instructions (two elements each).  The correction maps
+// x = -0 to +0, so the sign bit of every x is OR-ed into its e4m3 code
+// (e4m3 keeps -0 as 0x80); for x != -0 the code already carries that sign.
+// The test suite replays this sequence on the host for every (amax, x)
+// pair of bf16 values and checks it gives the IEEE quotient's e4m3 code.
 #pragma once
 
 #include <cstdint>
@@ -29,46 +31,75 @@ __device__ __forceinline__ float scale_from_amax(float amax) {
   return __fdiv_rn(fmaxf(amax, kAmaxEps), kE4m3Max);
 }
 
-__device__ __forceinline__ float div_by_scale(float x, float s, float r) {
-  float q0 = __fmul_rn(x, r);
-  float e = __fmaf_rn(-q0, s, x);
-  return copysignf(__fmaf_rn(e, r, q0), x);
+// Per-group constants of the division: -s and fp32(1/s), duplicated for
+// the packed instructions.
+struct GroupScale {
+  float2 neg_s;
+  float2 rcp;
+};
+
+__device__ __forceinline__ GroupScale group_scale(float s) {
+  const float r = __frcp_rn(s);
+  GroupScale g;
+  g.neg_s = make_float2(-s, -s);
+  g.rcp = make_float2(r, r);
+  return g;
 }
 
 // Two fp32 values -> two e4m3 bytes (lo in the low byte), round to
 // nearest even, saturating to +-448.
-__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   uint16_t h;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
   return h;
 }
 
-// bf16 pair packed in a 32-bit word -> two exact fp32 values.
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// max |x| over the 8 bf16 values of a 16-byte vector.
-__device__ __forceinline__ float amax8(uint4 v) {
-  float a = fabsf(bf16lo(v.x));
-  a = fmaxf(a, fabsf(bf16hi(v.x)));
-  a = fmaxf(a, fabsf(bf16lo(v.y)));
-  a = fmaxf(a, fabsf(bf16hi(v.y)));
-  a = fmaxf(a, fabsf(bf16lo(v.z)));
-  a = fmaxf(a, fabsf(bf16hi(v.z)));
-  a = fmaxf(a, fabsf(bf16lo(v.w)));
-  a = fmaxf(a, fabsf(bf16hi(v.w)));
-  return a;
+// A bf16x2 word -> the two exact fp32 values (lo, hi).
+__device__ __forceinline__ float2 bf16x2_to_f32x2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
-__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, float s, float r) {
-  uint32_t lo = cvt_e4m3x2(div_by_scale(bf16lo(w0), s, r), div_by_scale(bf16hi(w0), s, r));
-  uint32_t hi = cvt_e4m3x2(div_by_scale(bf16lo(w1), s, r), div_by_scale(bf16hi(w1), s, r));
-  return lo | (hi << 16);
+// Element-wise max of |a| and |b| on bf16x2 words (sign of the result is
+// not meaningful; only magnitudes are used).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// |max| over the 8 bf16 values of a 16-byte vector, as a bf16x2 word whose
+// two halves both hold magnitudes (fold with absmax_bf16x2 across lanes).
+__device__ __forceinline__ uint32_t absmax8_bf16x2(uint4 v) {
+  return absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w));
+}
+
+// Larger magnitude of the two halves of a bf16x2 word, as fp32 (exact).
+__device__ __forceinline__ float absmax_halves_f32(uint32_t m) {
+  return fmaxf(__uint_as_float(m & 0x7FFF0000u), __uint_as_float((m << 16) & 0x7FFFFFFFu));
+}
+
+// Quotients x / s of a bf16x2 word, correctly rounded (see above).
+__device__ __forceinline__ float2 div2_by_scale(uint32_t w, const GroupScale& g) {
+  const float2 x = bf16x2_to_f32x2(w);
+  const float2 q0 = __fmul2_rn(x, g.rcp);
+  const float2 e = __ffma2_rn(q0, g.neg_s, x);
+  return __ffma2_rn(e, g.rcp, q0);
+}
+
+// Four bf16 (two words) -> four e4m3 codes in one word, element order kept.
+__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, const GroupScale& g) {
+  const float2 a = div2_by_scale(w0, g);
+  const float2 b = div2_by_scale(w1, g);
+  const uint32_t codes = cvt_e4m3x2(a.x, a.y) | (cvt_e4m3x2(b.x, b.y) << 16);
+  // sign bits of the four inputs (bit 15 and 31 of each word) moved to
+  // bit 7 of the matching code byte
+  const uint32_t signs = __byte_perm(w0, w1, 0x7531) & 0x80808080u;
+  return codes | signs;
 }
 
 // 8 bf16 values (16 bytes) -> 8 e4m3 codes (8 bytes), same order.
-__device__ __forceinline__ uint2 quant8(uint4 v, float s, float r) {
-  return make_uint2(quant4(v.x, v.y, s, r), quant4(v.z, v.w, s, r));
+__device__ __forceinline__ uint2 quant8(uint4 v, const GroupScale& g) {
+  return make_uint2(quant4(v.x, v.y, g), quant4(v.z, v.w, g));
 }
 
 }  // namespace fp8bl

@@ -3,9 +3,10 @@
  *
  * The kernels compute x / s for a whole 128-group with one correctly
  * rounded reciprocal r = fp32(1/s) and, per element, q0 = fp32(x*r),
- * e = fma(-q0, s, x), q = fma(e, r, q0) (Markstein's correction step),
- * and finally give q the sign bit of x (the correction turns x = -0 into
- * +0; for every other x the sign is already that of x).
+ * e = fma(q0, -s, x), q = fma(e, r, q0) (Markstein's correction step).
+ * The e4m3 code is then cvt(q) with the sign bit of x OR-ed in: the
+ * correction turns x = -0 into +0, and this program also checks that every
+ * non-zero q already carries the sign of x, so the OR changes nothing else.
  * The quantization definition wants fp32(x / s), then e4m3 rounding.  This
  * program checks, for EVERY pair the kernels can meet -- amax any
  * non-negative finite bf16 value (s = fp32(max(amax, 1e-10)/448)) and x any
@@ -45,9 +46,16 @@ static void *run(void *arg)
                 float x = bf(xm | (sg << 15));
                 float ref = x / s;
                 float q0 = x * r;
-                float e = fmaf(-q0, s, x);
-                float q = copysignf(fmaf(e, r, q0), x);
+                float e = fmaf(q0, -s, x);
+                float q = fmaf(e, r, q0);
                 j->pairs++;
+                if (q != 0.0f && (bits(q) >> 31) != (bits(x) >> 31)) {
+                    if (!j->bad) { j->bad_a = a; j->bad_x = xm | (sg << 15); }
+                    j->bad++;
+                    continue;
+                }
+                if (q == 0.0f)
+                    q = copysignf(0.0f, x);   /* the sign-bit OR on the code */
                 if (bits(q) == bits(ref))
                     continue;
                 if (fabsf(q) <= 0x1p-10f && fabsf(ref) <= 0x1p-10f &&
