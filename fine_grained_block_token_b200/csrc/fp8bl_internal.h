@@ -5,6 +5,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace fp8bl {
@@ -29,6 +30,9 @@ cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float
 cudaError_t launch_weight_quant(const void* w, int64_t N, int64_t K, void* q, float* s,
                                 cudaStream_t st);
 
+// Largest M served by the decode (swap-AB, stream-K) schedule.
+constexpr int64_t kDecodeMaxM = 64;
+
 // GEMM schedule, chosen on the host from the sizes.
 struct GemmPlan {
   int kind = 0;          // 0 = prefill tile kernel, 1 = decode (swap-AB) kernel
@@ -42,6 +46,17 @@ cudaError_t launch_block_linear(const void* q_a, const float* s_a, const void* q
                                 const float* s_w, void* y, int64_t M, int64_t N, int64_t K,
                                 const GemmPlan& plan, void* workspace, const DeviceInfo& dev,
                                 cudaStream_t st);
+
+// Decode schedule (M <= kDecodeMaxM): scratch bytes and launch.
+size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count);
+cudaError_t launch_block_linear_decode(const void* q_a, const float* s_a, const void* q_w,
+                                       const float* s_w, void* y, int64_t M, int64_t N, int64_t K,
+                                       void* workspace, const DeviceInfo& dev, cudaStream_t st);
+
+// 2-D TMA map over a row-major byte matrix [rows, cols], box box_rows x
+// box_cols, 128-byte swizzle, out-of-range elements read as zero.
+bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows, uint32_t box_cols);
 
 cudaError_t launch_block_linear_fused(const void* x, const void* q_w, const float* s_w, void* y,
                                       int64_t M, int64_t N, int64_t K, const GemmPlan& plan,

@@ -264,9 +264,21 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
   }
 }
 
+cudaError_t ensure_smem_attr() {
+  static cudaError_t st = cudaSuccess;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    st = cudaFuncSetAttribute(gemm_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              SMEM_BYTES);
+  });
+  return st;
+}
+
+}  // namespace
+
 // ------------------------------------------------------------------ host
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -296,29 +308,22 @@ bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
   return r == CUDA_SUCCESS;
 }
 
-cudaError_t ensure_smem_attr() {
-  static cudaError_t st = cudaSuccess;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    st = cudaFuncSetAttribute(gemm_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              SMEM_BYTES);
-  });
-  return st;
-}
-
-}  // namespace
-
 GemmPlan plan_block_linear(int64_t M, int64_t N, int64_t K, int sm_count, bool fused) {
-  (void)M; (void)N; (void)K; (void)sm_count;
   GemmPlan p;
   p.kind = 0;
   p.split_k = 1;
   p.workspace = 0;
+  if (M <= kDecodeMaxM) {
+    // decode sizes: swap-AB stream-K kernel + ordered reduction
+    p.kind = 1;
+    p.workspace = decode_workspace_bytes(M, N, K, sm_count);
+  }
   if (fused) {
-    // staged fused path: q_a and s_a in the workspace
+    // staged fused path: q_a and s_a in the workspace after the GEMM's own
     const int64_t qa = M * K;
     const int64_t sa = M * (K / 128) * 4;
-    p.workspace = static_cast<size_t>(((qa + 255) / 256) * 256 + sa);
+    p.workspace = ((p.workspace + 255) / 256) * 256 +
+                  static_cast<size_t>(((qa + 255) / 256) * 256 + ((sa + 255) / 256) * 256);
   }
   return p;
 }
@@ -327,8 +332,9 @@ cudaError_t launch_block_linear(const void* q_a, const float* s_a, const void* q
                                 const float* s_w, void* y, int64_t M, int64_t N, int64_t K,
                                 const GemmPlan& plan, void* workspace, const DeviceInfo& dev,
                                 cudaStream_t st) {
-  (void)plan; (void)workspace;
   if (M == 0) return cudaSuccess;
+  if (plan.kind == 1)
+    return launch_block_linear_decode(q_a, s_a, q_w, s_w, y, M, N, K, workspace, dev, st);
   cudaError_t e = ensure_smem_attr();
   if (e != cudaSuccess) return e;
   CUtensorMap ta, tb;
@@ -352,13 +358,14 @@ cudaError_t launch_block_linear_fused(const void* x, const void* q_w, const floa
                                       int64_t M, int64_t N, int64_t K, const GemmPlan& plan,
                                       void* workspace, const DeviceInfo& dev, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
-  uint8_t* qa = static_cast<uint8_t*>(workspace);
+  // staged: quantized activations in the workspace, after the GEMM's own scratch
+  (void)plan;
+  const GemmPlan gp = plan_block_linear(M, N, K, dev.sm_count, false);
+  uint8_t* qa = static_cast<uint8_t*>(workspace) + ((gp.workspace + 255) / 256) * 256;
   float* sa = reinterpret_cast<float*>(qa + ((M * K + 255) / 256) * 256);
   cudaError_t e = launch_act_quant(x, M, K, qa, sa, dev.sm_count, st);
   if (e != cudaSuccess) return e;
-  GemmPlan p2 = plan;
-  p2.workspace = 0;
-  return launch_block_linear(qa, sa, q_w, s_w, y, M, N, K, p2, nullptr, dev, st);
+  return launch_block_linear(qa, sa, q_w, s_w, y, M, N, K, gp, workspace, dev, st);
 }
 
 }  // namespace fp8bl

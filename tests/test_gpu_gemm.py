@@ -120,3 +120,40 @@ def test_fused_bit_identical(fp8):
 
 def test_no_timeout_recorded(fp8):
     fp8.check()
+
+
+@pytest.mark.parametrize("M", [1, 2, 15, 16, 17, 33, 48, 63, 64])
+def test_decode_token_counts(fp8, M):
+    """Every padded-token bucket of the decode schedule (16/32/48/64) with
+    ragged counts; K spans 24 chunks so stream-K ranges cross blocks."""
+    N, K = 1024, 3072
+    xb = wl.normal((M, K), 1.0, 0, 100 + M)
+    wb = wl.zero_blocks(wl.normal((N, K), 0.02, 1, 100 + M), 0.05)
+    y, R, _ = _run(fp8, xb, wb)
+    check_gemm(y, R, f"decode M={M}")
+
+
+def test_decode_deterministic_and_small_shapes(fp8):
+    for (M, N, K) in [(3, 128, 128), (8, 256, 384), (64, 384, 1280)]:
+        xb = wl.normal((M, K), 1.0, 0, M + K)
+        wb = wl.normal((N, K), 0.02, 1, M + K)
+        y, R, (x, q_a, s_a, q_w, s_w, _) = _run(fp8, xb, wb)
+        check_gemm(y, R, f"decode {M}x{N}x{K}")
+        y2 = fp8.block_linear(q_a, s_a, q_w, s_w)
+        y3 = fp8.block_linear(q_a, s_a, q_w, s_w)
+        torch.cuda.synchronize()
+        assert torch.equal(y2.view(torch.int16), y3.view(torch.int16))
+
+
+def test_decode_workspace_too_small(fp8):
+    M, N, K = 8, 512, 1024
+    need = fp8.workspace_bytes(M, N, K)
+    assert need > 0
+    x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((N, K), dtype=torch.bfloat16, device="cuda")
+    q_a, s_a = fp8.quant_act(x)
+    q_w, s_w = fp8.quant_weight(w)
+    small = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fp8.Fp8blError) as ei:
+        fp8.block_linear(q_a, s_a, q_w, s_w, workspace=small)
+    assert ei.value.status == 7
