@@ -1,158 +1,24 @@
 """fine_grained_block_token_b200 -- block-scaled FP8 linear layers for B200.
 
-Python binding of the C ABI in ``include/fp8bl.h`` (``libfp8bl.so``, built
-in-tree by ``fine_grained_block_token_b200.build``).  The binding only
-marshals arguments: it allocates outputs with torch on the input's device,
-passes raw device pointers, sizes and the current CUDA stream, and turns
-status codes into exceptions.  Every step of the computation runs in the
-library's CUDA kernels; there is no fallback path.  If the library is
-missing the import of this module fails.
-
-Method ("Fine-grained FP8" page of the transformers docs, opening bullet
-list): weights quantized to e4m3 with one fp32 scale per 128 x 128 block,
+Weights quantized to e4m3 with one fp32 scale per 128 x 128 block,
 activations quantized dynamically per token with one fp32 scale per group of
 128 input channels, and a GEMM that applies both scale sets per 128-deep K
-block and writes bf16.
+block and writes bf16 ("Fine-grained FP8" page of the transformers docs,
+opening bullet list).
+
+The functions below come from ``_binding`` (a ctypes binding of
+``libfp8bl.so``), loaded on first use so that the ``build`` submodule can be
+imported before the library exists.  Using any of them without the library
+raises ImportError: there is no fallback path.
 """
-from __future__ import annotations
-
-import ctypes
-import os
-
-import torch
-
 __all__ = [
-    "Fp8blError", "BLOCK", "lib_path", "quant_act", "quant_weight", "block_linear",
+    "Fp8blError", "BLOCK", "STATUS", "lib_path", "quant_act", "quant_weight", "block_linear",
     "block_linear_fused", "workspace_bytes", "fused_workspace_bytes", "check", "version",
 ]
 
-BLOCK = 128
-_HERE = os.path.dirname(os.path.abspath(__file__))
-lib_path = os.path.join(_HERE, "libfp8bl.so")
 
-if not os.path.exists(lib_path):
-    raise ImportError(
-        f"{lib_path} is missing: build it with `python -m fine_grained_block_token_b200.build`")
-
-_lib = ctypes.CDLL(lib_path)
-_i64, _vp, _sz = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
-_lib.fp8_quant_act.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
-_lib.fp8_quant_weight.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
-_lib.fp8_block_linear.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp]
-_lib.fp8_block_linear_fused.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp]
-_lib.fp8_block_linear_workspace_bytes.argtypes = [_i64, _i64, _i64]
-_lib.fp8_block_linear_workspace_bytes.restype = _sz
-_lib.fp8_block_linear_fused_workspace_bytes.argtypes = [_i64, _i64, _i64]
-_lib.fp8_block_linear_fused_workspace_bytes.restype = _sz
-_lib.fp8bl_check.argtypes = [_vp]
-_lib.fp8bl_status_string.argtypes = [ctypes.c_int]
-_lib.fp8bl_status_string.restype = ctypes.c_char_p
-_lib.fp8bl_version.restype = ctypes.c_int
-for _f in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
-           "fp8bl_check"):
-    getattr(_lib, _f).restype = ctypes.c_int
-
-STATUS = {0: "FP8BL_OK", 1: "FP8BL_ERR_NULL", 2: "FP8BL_ERR_SHAPE", 3: "FP8BL_ERR_ALIGN",
-          4: "FP8BL_ERR_ARCH", 5: "FP8BL_ERR_CUDA", 6: "FP8BL_ERR_TIMEOUT",
-          7: "FP8BL_ERR_WORKSPACE", 8: "FP8BL_ERR_OVERLAP"}
-
-
-class Fp8blError(RuntimeError):
-    def __init__(self, status: int, where: str):
-        self.status = status
-        msg = _lib.fp8bl_status_string(status).decode()
-        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
-
-
-def _ok(status: int, where: str) -> None:
-    if status != 0:
-        raise Fp8blError(status, where)
-
-
-def _stream(t: torch.Tensor):
-    return torch.cuda.current_stream(t.device).cuda_stream
-
-
-def _ptr(t):
-    return None if t is None else t.data_ptr()
-
-
-def _u8(t: torch.Tensor) -> torch.Tensor:
-    return t.view(torch.uint8) if t.dtype != torch.uint8 else t
-
-
-def version() -> int:
-    return _lib.fp8bl_version()
-
-
-def quant_act(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None):
-    """bf16 [M, K] -> (e4m3 [M, K], fp32 [M, K/128]).  Outputs may be given."""
-    M, K = x.shape
-    if q is None:
-        q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
-    if s is None:
-        s = torch.empty((M, K // BLOCK if K % BLOCK == 0 else 0), dtype=torch.float32, device=x.device)
-    _ok(_lib.fp8_quant_act(_ptr(x), M, K, _ptr(q), _ptr(s), _stream(x)), "fp8_quant_act")
-    return q, s
-
-
-def quant_weight(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None):
-    """bf16 [N, K] -> (e4m3 [N, K], fp32 [N/128, K/128])."""
-    N, K = w.shape
-    if q is None:
-        q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
-    if s is None:
-        s = torch.empty((N // BLOCK, K // BLOCK), dtype=torch.float32, device=w.device)
-    _ok(_lib.fp8_quant_weight(_ptr(w), N, K, _ptr(q), _ptr(s), _stream(w)), "fp8_quant_weight")
-    return q, s
-
-
-def workspace_bytes(M: int, N: int, K: int) -> int:
-    return int(_lib.fp8_block_linear_workspace_bytes(M, N, K))
-
-
-def fused_workspace_bytes(M: int, N: int, K: int) -> int:
-    return int(_lib.fp8_block_linear_fused_workspace_bytes(M, N, K))
-
-
-def _workspace(nbytes: int, device, given):
-    if nbytes == 0:
-        return given, 0 if given is None else given.numel() * given.element_size()
-    if given is None:
-        given = torch.empty(nbytes, dtype=torch.uint8, device=device)
-    return given, given.numel() * given.element_size()
-
-
-def block_linear(q_a, s_a, q_w, s_w, y=None, workspace=None) -> torch.Tensor:
-    """(e4m3 [M,K], fp32 [M,K/128], e4m3 [N,K], fp32 [N/128,K/128]) -> bf16 [M,N]."""
-    M, K = q_a.shape
-    N = q_w.shape[0]
-    if q_w.shape[1] != K:
-        raise ValueError("q_a and q_w disagree on K")
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
-    ws, wsb = _workspace(workspace_bytes(M, N, K), q_a.device, workspace)
-    _ok(_lib.fp8_block_linear(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
-                              _ptr(ws), wsb, _stream(q_a)), "fp8_block_linear")
-    return y
-
-
-def block_linear_fused(x, q_w, s_w, y=None, workspace=None) -> torch.Tensor:
-    """bf16 x [M,K] with quantized weights -> bf16 [M,N]; the activation
-    quantization happens inside the GEMM, bit-identical to quant_act."""
-    M, K = x.shape
-    N = q_w.shape[0]
-    if q_w.shape[1] != K:
-        raise ValueError("x and q_w disagree on K")
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    ws, wsb = _workspace(fused_workspace_bytes(M, N, K), x.device, workspace)
-    _ok(_lib.fp8_block_linear_fused(_ptr(x), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
-                                    _ptr(ws), wsb, _stream(x)), "fp8_block_linear_fused")
-    return y
-
-
-def check(device=None) -> None:
-    """Synchronise the current stream and raise if a kernel wait timed out."""
-    st = torch.cuda.current_stream(device).cuda_stream
-    _ok(_lib.fp8bl_check(st), "fp8bl_check")
+def __getattr__(name):
+    if name in __all__:
+        from . import _binding
+        return getattr(_binding, name)
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")
