@@ -13,7 +13,8 @@ raises ImportError: there is no fallback path.
 """
 __all__ = [
     "Fp8blError", "BLOCK", "STATUS", "lib_path", "quant_act", "quant_weight", "block_linear",
-    "block_linear_fused", "workspace_bytes", "fused_workspace_bytes", "check", "version",
+    "block_linear_fused", "block_linear_noalloc", "workspace_bytes", "fused_workspace_bytes",
+    "check", "version",
 ]
 
 

@@ -21,7 +21,8 @@ import torch
 
 __all__ = [
     "Fp8blError", "BLOCK", "lib_path", "quant_act", "quant_weight", "block_linear",
-    "block_linear_fused", "workspace_bytes", "fused_workspace_bytes", "check", "version",
+    "block_linear_fused", "block_linear_noalloc", "workspace_bytes", "fused_workspace_bytes",
+    "check", "version",
 ]
 
 BLOCK = 128
@@ -38,6 +39,7 @@ _lib.fp8_quant_act.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_quant_weight.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_block_linear.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp]
 _lib.fp8_block_linear_fused.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp]
+_lib.fp8_block_linear_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
 _lib.fp8_block_linear_workspace_bytes.argtypes = [_i64, _i64, _i64]
 _lib.fp8_block_linear_workspace_bytes.restype = _sz
 _lib.fp8_block_linear_fused_workspace_bytes.argtypes = [_i64, _i64, _i64]
@@ -47,7 +49,7 @@ _lib.fp8bl_status_string.argtypes = [ctypes.c_int]
 _lib.fp8bl_status_string.restype = ctypes.c_char_p
 _lib.fp8bl_version.restype = ctypes.c_int
 for _f in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
-           "fp8bl_check"):
+           "fp8_block_linear_noalloc", "fp8bl_check"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 STATUS = {0: "FP8BL_OK", 1: "FP8BL_ERR_NULL", 2: "FP8BL_ERR_SHAPE", 3: "FP8BL_ERR_ALIGN",
@@ -147,6 +149,20 @@ def block_linear_fused(x, q_w, s_w, y=None, workspace=None) -> torch.Tensor:
     ws, wsb = _workspace(fused_workspace_bytes(M, N, K), x.device, workspace)
     _ok(_lib.fp8_block_linear_fused(_ptr(x), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
                                     _ptr(ws), wsb, _stream(x)), "fp8_block_linear_fused")
+    return y
+
+
+def block_linear_noalloc(q_a, s_a, q_w, s_w, y) -> torch.Tensor:
+    """Decode-sized linear (1 <= M <= 64) with the library's built-in scratch:
+    no workspace, and nothing is allocated here or in the library, so the
+    output tensor ``y`` (bf16 [M, N]) must be given.  For callers that cannot
+    allocate device memory where they run the layer."""
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    if q_w.shape[1] != K:
+        raise ValueError("q_a and q_w disagree on K")
+    _ok(_lib.fp8_block_linear_noalloc(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
+                                      _stream(q_a)), "fp8_block_linear_noalloc")
     return y
 
 

@@ -139,6 +139,39 @@ fp8bl_status fp8_block_linear_fused(const void *x_bf16,
                                     void *workspace, size_t workspace_bytes,
                                     fp8bl_stream_t stream);
 
+/*
+ * fp8_block_linear_noalloc -- fp8_block_linear for 1 <= M <= 64 tokens
+ * (the decode sizes, whose schedule needs scratch memory) using a scratch
+ * array built into the library instead of a caller workspace.  The pages
+ * have no counterpart: this is an integration convenience.
+ *
+ * Some callers cannot allocate device memory at the point where they run
+ * the layer -- for example a serving loop whose device memory is fully
+ * reserved up front by its own pool, code that must avoid the device-wide
+ * synchronisation that cudaMalloc / cudaFree can cause, or a host program
+ * that only ever hands over the tensors it already owns.  This call lets
+ * them run the decode-sized linear with nothing but its inputs and output.
+ *
+ *   arguments as fp8_block_linear, without the workspace.
+ *   The scratch is a FP8BL_NOALLOC_SCRATCH_BYTES array in device memory that
+ *   exists on every GPU that loads the library until the process exits.
+ *   Shapes whose decode schedule needs more scratch than that return
+ *   FP8BL_ERR_WORKSPACE; M > 64 returns FP8BL_ERR_SHAPE (for M > 64,
+ *   fp8_block_linear needs no workspace: pass NULL, 0).
+ *   The first call on each device looks up the array's device address (a
+ *   CUDA runtime query), so make that first call before any stream capture.
+ *   All calls on a device share the array and leave its contents behind;
+ *   each call clears what must start at zero on `stream` first.  Calls
+ *   whose GPU work may overlap (different streams with no ordering between
+ *   them) race on the array and must not be issued.
+ *   Neither this call nor the library allocates or frees device memory.
+ */
+#define FP8BL_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+fp8bl_status fp8_block_linear_noalloc(const void *q_a, const float *s_a,
+                                      const void *q_w, const float *s_w,
+                                      void *y_bf16, int64_t M, int64_t N, int64_t K,
+                                      fp8bl_stream_t stream);
+
 /* Workspace sizes (bytes) the two linear calls need for these sizes on the
  * current device; 0 when no scratch is needed.  Never fails: invalid sizes
  * return 0 (the linear call then reports the error). */
