@@ -67,6 +67,60 @@ act_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, float* __re
   }
 }
 
+// 32-byte variant (input 32-byte aligned): a lane loads 32 contiguous bytes
+// (16 bf16) with one 256-bit load, 8 lanes own a group and a warp covers 4
+// consecutive groups (1 KB) per load instruction.  The per-group work (abs-max
+// shuffles, scale, reciprocal) is then spread over twice as many elements,
+// and each lane stores 16 codes with one 16-byte store.
+constexpr int kAq32Unroll = 2;
+
+__device__ __forceinline__ void ld_stream32(const uint4* p, uint4& a, uint4& b) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z),
+                 "=r"(b.w)
+               : "l"(p));
+}
+
+__global__ void __launch_bounds__(kAqThreads, 4)
+act_quant32_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, float* __restrict__ s,
+                   int64_t num_groups) {
+  const int lane = threadIdx.x & 31;
+  const int sub = lane >> 3;      // group within the warp's 4
+  const int l8 = lane & 7;        // 32-byte slice within the group
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kAqThreads + threadIdx.x) >> 5;
+  const int64_t num_warps = (static_cast<int64_t>(gridDim.x) * kAqThreads) >> 5;
+  const int64_t num_quads = (num_groups + 3) >> 2;
+  // The loop bound depends on the warp only: every shuffle has all lanes.
+  for (int64_t p0 = warp; p0 < num_quads; p0 += num_warps * kAq32Unroll) {
+    uint4 va[kAq32Unroll], vb[kAq32Unroll];
+#pragma unroll
+    for (int u = 0; u < kAq32Unroll; ++u) {
+      const int64_t g = (p0 + u * num_warps) * 4 + sub;
+      if (g < num_groups) {
+        ld_stream32(x + g * 16 + l8 * 2, va[u], vb[u]);
+      } else {
+        va[u] = make_uint4(0u, 0u, 0u, 0u);
+        vb[u] = va[u];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kAq32Unroll; ++u) {
+      const int64_t g = (p0 + u * num_warps) * 4 + sub;
+      uint32_t m = absmax_bf16x2(absmax8_bf16x2(va[u]), absmax8_bf16x2(vb[u]));
+      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      const float sc = scale_from_amax(absmax_halves_f32(m));
+      const GroupScale gs = group_scale(sc);
+      const uint2 lo = quant8(va[u], gs), hi = quant8(vb[u], gs);
+      if (g < num_groups) {
+        q[g * 8 + l8] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        if (l8 == 0) s[g] = sc;
+      }
+    }
+  }
+}
+
 // One CTA per 128 x 128 block.  Thread t covers 16-byte chunk (t % 16) of
 // rows (t / 16) + 16 i, i = 0..7: every load instruction of a warp reads two
 // full 256-byte row segments.
@@ -111,6 +165,16 @@ cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float
                              int sm_count, cudaStream_t st) {
   const int64_t groups = M * (K / 128);
   if (groups == 0) return cudaSuccess;
+  if ((reinterpret_cast<uintptr_t>(x) & 31) == 0) {
+    const int64_t quads = (groups + 3) / 4;
+    const int64_t warps_needed = (quads + kAq32Unroll - 1) / kAq32Unroll;
+    const int64_t blocks_needed = (warps_needed + (kAqThreads / 32) - 1) / (kAqThreads / 32);
+    const int64_t max_blocks = static_cast<int64_t>(sm_count) * 4;
+    const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
+    act_quant32_kernel<<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
+                                                      static_cast<uint4*>(q), s, groups);
+    return cudaGetLastError();
+  }
   const int64_t pairs = (groups + 1) / 2;
   const int64_t warps_needed = (pairs + kAqUnroll - 1) / kAqUnroll;
   const int64_t blocks_needed = (warps_needed + (kAqThreads / 32) - 1) / (kAqThreads / 32);

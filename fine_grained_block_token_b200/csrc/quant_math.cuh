@@ -15,8 +15,13 @@
 // packed f32x2 instructions (two elements each).  The correction maps
 // x = -0 to +0, so the sign bit of every x is OR-ed into its e4m3 code
 // (e4m3 keeps -0 as 0x80); for x != -0 the code already carries that sign.
-// The test suite replays this sequence on the host for every (amax, x)
-// pair of bf16 values and checks it gives the IEEE quotient's e4m3 code.
+// The scale itself is formed with the same correction step against the
+// constant R = fp32(1/448): q0 = fp32(a * R), e = fma(q0, -448, a),
+// s = fp32(q0 + e * R).
+// The test suite replays both sequences on the host: the scale for every
+// amax a bf16 input can produce (and the eps floor) against the IEEE
+// quotient a / 448, and the element quotient for every (amax, x) pair of
+// bf16 values against the e4m3 code of the IEEE quotient x / s.
 #pragma once
 
 #include <cstdint>
@@ -26,9 +31,13 @@ namespace fp8bl {
 
 constexpr float kE4m3Max = 448.0f;
 constexpr float kAmaxEps = 1e-10f;
+constexpr float kRcpE4m3Max = 0x1.24924ap-9f;   // fp32(1 / 448)
 
 __device__ __forceinline__ float scale_from_amax(float amax) {
-  return __fdiv_rn(fmaxf(amax, kAmaxEps), kE4m3Max);
+  const float a = fmaxf(amax, kAmaxEps);
+  const float q0 = __fmul_rn(a, kRcpE4m3Max);
+  const float e = __fmaf_rn(q0, -kE4m3Max, a);
+  return __fmaf_rn(e, kRcpE4m3Max, q0);
 }
 
 // Per-group constants of the division: -s and fp32(1/s), duplicated for

@@ -17,6 +17,12 @@
  * rounded) and multiplication, with gradual underflow, exactly as the GPU
  * instructions the kernel uses (div.rn, rcp.rn, mul.rn, fma.rn, no flush).
  *
+ * The scale s itself is formed on the GPU with the same correction step
+ * against the constant R = fp32(1/448): q0 = fp32(a*R), e = fma(q0,-448,a),
+ * s = fma(e, R, q0), a = max(amax, 1e-10).  This program first checks that
+ * s equals the IEEE quotient a / 448 for every amax (printing
+ * "scales <n> bad <m>"), then uses it for the element check.
+ *
  * Usage: div_exhaustive <nthreads>.  Prints "pairs <n> bad <m>".
  */
 #include <math.h>
@@ -31,15 +37,23 @@ static int g_nt;
 static float bf(uint32_t h) { uint32_t b = h << 16; float f; memcpy(&f, &b, 4); return f; }
 static uint32_t bits(float f) { uint32_t b; memcpy(&b, &f, 4); return b; }
 
-typedef struct { int t; uint64_t pairs, bad; uint32_t bad_a, bad_x; } job;
+typedef struct { int t; uint64_t pairs, bad, scale_bad; uint32_t bad_a, bad_x; } job;
 
 static void *run(void *arg)
 {
     job *j = (job *)arg;
     volatile float eps = 1e-10f, m448 = 448.0f, one = 1.0f;
+    const float R = one / m448;
     for (uint32_t a = (uint32_t)j->t; a <= 0x7F7Fu; a += (uint32_t)g_nt) {
         float amax = bf(a);
-        float s = fmaxf(amax, eps) / m448;
+        float av = fmaxf(amax, eps);
+        float sq0 = av * R;
+        float se = fmaf(sq0, -m448, av);
+        float s = fmaf(se, R, sq0);
+        if (bits(s) != bits(av / m448)) {
+            j->scale_bad++;
+            continue;
+        }
         float r = one / s;
         for (uint32_t xm = 0; xm <= a; ++xm) {
             for (uint32_t sg = 0; sg < 2; ++sg) {
@@ -81,15 +95,17 @@ int main(int argc, char **argv)
         jobs[t].t = t;
         pthread_create(&th[t], 0, run, &jobs[t]);
     }
-    uint64_t pairs = 0, bad = 0;
+    uint64_t pairs = 0, bad = 0, scale_bad = 0;
     uint32_t ba = 0, bx = 0;
     for (int t = 0; t < g_nt; ++t) {
         pthread_join(th[t], 0);
         pairs += jobs[t].pairs;
+        scale_bad += jobs[t].scale_bad;
         if (jobs[t].bad && !bad) { ba = jobs[t].bad_a; bx = jobs[t].bad_x; }
         bad += jobs[t].bad;
     }
+    printf("scales 32640 bad %llu\n", (unsigned long long)scale_bad);
     printf("pairs %llu bad %llu first amax 0x%04x x 0x%04x\n",
            (unsigned long long)pairs, (unsigned long long)bad, ba, bx);
-    return bad ? 1 : 0;
+    return (bad || scale_bad) ? 1 : 0;
 }

@@ -93,3 +93,19 @@ def test_weight_quant_shapes(fp8, N, K):
 def test_weight_quant_full_size(fp8):
     _, wbits = wl.deepseek_mlp("up")        # W [18432, 7168], 1% zero blocks
     _check_weight(fp8, wbits)
+
+
+def test_act_quant_16_byte_aligned_input(fp8):
+    """Inputs that are 16- but not 32-byte aligned take the 16-byte kernel;
+    codes and scales must be identical to the oracle as well."""
+    M, K = 77, 1536
+    bits = wl.student_t_outliers(M, K, 3.0, 0.01, 100.0)
+    base = torch.empty(M * K + 64, dtype=torch.bfloat16, device="cuda")
+    x = base[8:8 + M * K].view(M, K)                    # +16 bytes
+    assert x.data_ptr() % 32 == 16
+    x.copy_(wl.to_torch_bf16(bits).cuda())
+    q, s = fp8.quant_act(x)
+    torch.cuda.synchronize()
+    qo, so = oracle.quant_act(bits, nthreads=8)
+    assert np.array_equal(f32(s).view(np.uint32), so.view(np.uint32))
+    assert np.array_equal(u8(q), qo)
