@@ -157,3 +157,36 @@ def test_decode_workspace_too_small(fp8):
     with pytest.raises(fp8.Fp8blError) as ei:
         fp8.block_linear(q_a, s_a, q_w, s_w, workspace=small)
     assert ei.value.status == 7
+
+
+@pytest.mark.parametrize("M", [512, 16384])
+def test_full_size_sweep_unfused_and_fused(fp8, M):
+    """Sweep workload: X [M, 7168] Student-t(3) with outlier channels and
+    zeroed groups against W [2048, 7168]; the fused entry point must equal the
+    unfused one bit for bit, and both meet the tolerance on sampled rows."""
+    xb = wl.sweep_x(M)
+    wb = wl.sweep_w()
+    rows = _sample_rows(M, 16, seed=M)
+    y, R, (x, q_a, s_a, q_w, s_w, y_full) = _run(fp8, xb, wb, rows=rows)
+    check_gemm(y, R, f"sweep M={M}")
+    y_fused = fp8.block_linear_fused(x, q_w, s_w)
+    torch.cuda.synchronize()
+    assert torch.equal(y_full.view(torch.int16), y_fused.view(torch.int16))
+
+
+def test_full_size_deepseek_down(fp8):
+    xb, wb = wl.deepseek_mlp("down")          # X [8192, 18432], W [7168, 18432]
+    rows = _sample_rows(xb.shape[0], 8, seed=3)
+    y, R, _ = _run(fp8, xb, wb, rows=rows)
+    check_gemm(y, R, "deepseek down")
+
+
+def test_fused_prefill_size_bit_identical(fp8):
+    xb, wb = wl.llama3_prefill("down")        # X [4096, 14336], W [4096, 14336]
+    x, w = to_dev(xb), to_dev(wb)
+    q_w, s_w = fp8.quant_weight(w)
+    q_a, s_a = fp8.quant_act(x)
+    y1 = fp8.block_linear(q_a, s_a, q_w, s_w)
+    y2 = fp8.block_linear_fused(x, q_w, s_w)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
