@@ -127,7 +127,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    {
       uint32_t issued_mask = 0, phase_mask = 0;
       uint32_t c = 0;
       int blk = static_cast<int>(u_begin / KB);
@@ -135,24 +135,32 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
       for (int64_t u = u_begin; u < u_end; ++u, ++c, (++kb == KB ? (kb = 0, ++blk) : 0)) {
         const int s = c % DSTAGES;
         const uint32_t ph = (c / DSTAGES) & 1u;
-        if (!ptx::mbar_wait(empty_bar(s), ph ^ 1u)) {
-          record_error(args.err, kErrTimeoutProducer);
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(empty_bar(s), ph ^ 1u))) {
+          if (lane == 0) record_error(args.err, kErrTimeoutProducer);
           break;
         }
-        ptx::mbar_arrive_expect_tx(full_bar(s), STAGE_TX);
-        ptx::tma_load_2d(smem_base + DSMEM_W_OFF + s * W_BYTES, &tmap_w, full_bar(s), kb * DBK,
-                         blk * DBM);
-        ptx::tma_load_2d(smem_base + DSMEM_X_OFF + s * X_BYTES, &tmap_x, full_bar(s), kb * DBK, 0);
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(full_bar(s), STAGE_TX);
+          ptx::tma_load_2d(smem_base + DSMEM_W_OFF + s * W_BYTES, &tmap_w, full_bar(s), kb * DBK,
+                           blk * DBM);
+          ptx::tma_load_2d(smem_base + DSMEM_X_OFF + s * X_BYTES, &tmap_x, full_bar(s), kb * DBK, 0);
+        }
+        __syncwarp();
         issued_mask |= 1u << s;
         phase_mask = (phase_mask & ~(1u << s)) | (ph << s);
       }
-      for (int s = 0; s < DSTAGES; ++s)
-        if (((issued_mask >> s) & 1u) && !ptx::mbar_wait(full_bar(s), (phase_mask >> s) & 1u))
-          record_error(args.err, kErrTimeoutProducer);
+      if (lane == 0)
+        for (int s = 0; s < DSTAGES; ++s)
+          if (((issued_mask >> s) & 1u) && !ptx::mbar_wait(full_bar(s), (phase_mask >> s) & 1u))
+            record_error(args.err, kErrTimeoutProducer);
+      __syncwarp();
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
+    // The whole warp runs the loop (the wait results are made warp-uniform
+    // with a vote) and lane 0 issues: measured on B200, a loop run by lane 0
+    // alone with a data-dependent exit costs ~600 cycles per chunk.
+    {
       uint32_t c = 0;
       bool issued = false;
       for (int64_t u = u_begin; u < u_end; ++u, ++c) {
@@ -160,27 +168,31 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         const uint32_t sph = (c / DSTAGES) & 1u;
         const int buf = c % DTBUFS;
         const uint32_t bph = (c / DTBUFS) & 1u;
-        if (!ptx::mbar_wait_spin(tempty_bar(buf), bph ^ 1u) ||
-            !ptx::mbar_wait_spin(full_bar(s), sph)) {
-          record_error(args.err, kErrTimeoutMma);
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(tempty_bar(buf), bph ^ 1u) &&
+                                         ptx::mbar_wait_spin(full_bar(s), sph))) {
+          if (lane == 0) record_error(args.err, kErrTimeoutMma);
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t w_addr = smem_base + DSMEM_W_OFF + s * W_BYTES;
-        const uint32_t x_addr = smem_base + DSMEM_X_OFF + s * X_BYTES;
-        const uint32_t d = tmem_base + static_cast<uint32_t>(buf * MAX_MPAD);
+        if (lane == 0) {
+          const uint32_t w_addr = smem_base + DSMEM_W_OFF + s * W_BYTES;
+          const uint32_t x_addr = smem_base + DSMEM_X_OFF + s * X_BYTES;
+          const uint32_t d = tmem_base + static_cast<uint32_t>(buf * MAX_MPAD);
 #pragma unroll
-        for (int k = 0; k < DBK / DUMMA_K; ++k)
-          ptx::mma_f8f6f4(d, ptx::sdesc_kmajor_sw128(w_addr + k * DUMMA_K),
-                          ptx::sdesc_kmajor_sw128(x_addr + k * DUMMA_K), IDESC, k > 0 ? 1u : 0u);
-        ptx::mma_commit(tfull_bar(buf));
-        ptx::mma_commit(empty_bar(s));
+          for (int k = 0; k < DBK / DUMMA_K; ++k)
+            ptx::mma_f8f6f4(d, ptx::sdesc_kmajor_sw128(w_addr + k * DUMMA_K),
+                            ptx::sdesc_kmajor_sw128(x_addr + k * DUMMA_K), IDESC, k > 0 ? 1u : 0u);
+          ptx::mma_commit(tfull_bar(buf));
+          ptx::mma_commit(empty_bar(s));
+        }
+        __syncwarp();
         issued = true;
       }
-      if (issued) {
+      if (issued && lane == 0) {
         ptx::mma_commit(drain_bar);
         if (!ptx::mbar_wait(drain_bar, 0)) record_error(args.err, kErrTimeoutMma);
       }
+      __syncwarp();
     }
   } else if (warp >= 4) {
     // ----------------------------------------------------------- promotion

@@ -13,9 +13,13 @@
 // running together share the same weight columns.  12 warps:
 //   warp 0      TMA producer: A tile 128x128 and W tile 256x128 (e4m3,
 //               128-byte swizzle) into a 4-deep shared-memory ring.
-//   warp 1      MMA issuer (one thread): per chunk, 4 MMAs (M=128, N=256,
-//               K=32) into one of two 256-column TMEM buffers, then commits
-//               to release the stage and to mark the buffer full.
+//   warp 1      MMA issuer: the whole warp runs the loop and waits (the
+//               wait results made warp-uniform by a vote), lane 0 issues
+//               4 MMAs per chunk (M=128, N=256, K=32) into one of two
+//               256-column TMEM buffers, then commits to release the stage
+//               and to mark the buffer full.  (A loop run by lane 0 alone,
+//               with a data-dependent exit, measured ~600 cycles per
+//               iteration on B200 whatever it waited for.)
 //   warp 2      owns the TMEM allocation (512 columns).
 //   warps 4-11  promotion: warp w reads TMEM lanes 32 (w % 4) .. +31 (its
 //               rows) and column half (w - 4) / 4 (one 128-wide weight
@@ -23,9 +27,18 @@
 //               the last load has landed, and adds partial * s_a[row, j] *
 //               s_w[nblk, j] into 128 fp32 registers with packed f32x2
 //               FMAs; after the last chunk it converts to bf16 and stores.
-// Measured on B200 (see the design notes): this layout, a CTA-pair 256x256
-// tile and 16-warp promotion variants all reach the same throughput, set by
-// the 1 kW power limit with the promotion work included.
+// What bounds it (measured on B200): every 128-deep chunk leaves a 128 KB
+// fp32 partial in TMEM that must be read into registers before the buffer
+// can take the chunk after next.  tcgen05.ld is latency-bound (a 64-column
+// load takes ~250 cycles; one warp moves at most ~36 B/cycle), so the read
+// rate equals the bytes in flight / ~250 cycles, and with the 128x256 fp32
+// accumulator occupying half the register file the promotion warps cannot
+// keep the ~64 KB in flight that the tensor core's 512 cycles per chunk
+// require.  Variants with two MMA-issuing warps, 64-column loads, 16
+// promotion warps, four 128-column TMEM buffers or CTA-pair tiles all land
+// at the same ~1.0-1.1 M flop per cycle (about 45% of the tensor core's
+// rate); the concurrent TMEM reads, FMAs and the power limit do not slow
+// the MMAs themselves.
 // Every mbarrier wait is bounded in time; on expiry the kernel records an
 // error code in the error word, drains what it started and exits cleanly.
 #include <cstdint>
@@ -151,7 +164,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
+    {
       uint32_t c = 0;
       bool ok = true, issued = false;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
@@ -160,30 +173,35 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
           const uint32_t sph = (c / STAGES) & 1u;
           const int buf = c & 1;
           const uint32_t bph = (c >> 1) & 1u;
-          if (!ptx::mbar_wait(tempty_bar(buf), bph ^ 1u) || !ptx::mbar_wait(full_bar(s), sph)) {
-            record_error(args.err, kErrTimeoutMma);
-            ok = false;
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait_spin(tempty_bar(buf), bph ^ 1u) &&
+                                           ptx::mbar_wait_spin(full_bar(s), sph));
+          if (!ok) {
+            if (lane == 0) record_error(args.err, kErrTimeoutMma);
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t a_addr = smem_base + SMEM_A_OFF + s * A_BYTES;
-          const uint32_t b_addr = smem_base + SMEM_B_OFF + s * B_BYTES;
-          const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+          if (lane == 0) {
+            const uint32_t a_addr = smem_base + SMEM_A_OFF + s * A_BYTES;
+            const uint32_t b_addr = smem_base + SMEM_B_OFF + s * B_BYTES;
+            const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
-            ptx::mma_f8f6f4(d, ptx::sdesc_kmajor_sw128(a_addr + k * UMMA_K),
-                            ptx::sdesc_kmajor_sw128(b_addr + k * UMMA_K), IDESC, k > 0 ? 1u : 0u);
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              ptx::mma_f8f6f4(d, ptx::sdesc_kmajor_sw128(a_addr + k * UMMA_K),
+                              ptx::sdesc_kmajor_sw128(b_addr + k * UMMA_K), IDESC, k > 0 ? 1u : 0u);
+            }
+            ptx::mma_commit(empty_bar(s));
+            ptx::mma_commit(tfull_bar(buf));
           }
-          ptx::mma_commit(empty_bar(s));
-          ptx::mma_commit(tfull_bar(buf));
+          __syncwarp();
           issued = true;
         }
       }
-      if (issued) {
+      if (issued && lane == 0) {
         // All MMAs finish before the TMEM they write is released.
         ptx::mma_commit(drain_bar);
         if (!ptx::mbar_wait(drain_bar, 0)) record_error(args.err, kErrTimeoutMma);
       }
+      __syncwarp();
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
@@ -214,7 +232,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
         if (kb + 2 < num_kb) { sa2 = __ldg(sa_row + kb + 2); sw2 = __ldg(sw_row + kb + 2); }
         const int buf = c & 1;
         const uint32_t bph = (c >> 1) & 1u;
-        if (!ptx::mbar_wait(tfull_bar(buf), bph)) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(tfull_bar(buf), bph))) {
           record_error(args.err, kErrTimeoutEpilogue);
           ok = false;
           break;
