@@ -35,7 +35,8 @@ constexpr int64_t kDecodeMaxM = 64;
 
 // GEMM schedule, chosen on the host from the sizes.
 struct GemmPlan {
-  int kind = 0;          // 0 = prefill tile kernel, 1 = decode (swap-AB) kernel
+  int kind = 0;          // 0 = prefill tile kernel, 1 = decode (swap-AB) kernel,
+                         // 2 = fused prefill kernel (activation quantization in the tiles)
   int split_k = 1;       // number of K slices (decode / small grids)
   size_t workspace = 0;  // bytes of fp32 partials needed
 };
@@ -61,6 +62,12 @@ bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
 cudaError_t launch_block_linear_fused(const void* x, const void* q_w, const float* s_w, void* y,
                                       int64_t M, int64_t N, int64_t K, const GemmPlan& plan,
                                       void* workspace, const DeviceInfo& dev, cudaStream_t st);
+
+// Fused prefill kernel (plan kind 2): activation quantization inside the
+// GEMM's tiles; no workspace.
+cudaError_t launch_block_linear_fused_tiles(const void* x, const void* q_w, const float* s_w,
+                                            void* y, int64_t M, int64_t N, int64_t K,
+                                            const DeviceInfo& dev, cudaStream_t st);
 
 // Error codes a kernel writes into the error word (first error wins).
 enum KernelError : int {

@@ -336,8 +336,12 @@ GemmPlan plan_block_linear(int64_t M, int64_t N, int64_t K, int sm_count, bool f
     p.kind = 1;
     p.workspace = decode_workspace_bytes(M, N, K, sm_count);
   }
-  if (fused) {
-    // staged fused path: q_a and s_a in the workspace after the GEMM's own
+  if (fused && p.kind == 0) {
+    // prefill sizes: the activation tile is quantized inside the GEMM
+    p.kind = 2;
+  } else if (fused) {
+    // decode sizes: quantize first (a few KB) into the workspace, after the
+    // GEMM's own scratch, then run the decode schedule
     const int64_t qa = M * K;
     const int64_t sa = M * (K / 128) * 4;
     p.workspace = ((p.workspace + 255) / 256) * 256 +
@@ -376,8 +380,8 @@ cudaError_t launch_block_linear_fused(const void* x, const void* q_w, const floa
                                       int64_t M, int64_t N, int64_t K, const GemmPlan& plan,
                                       void* workspace, const DeviceInfo& dev, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
+  if (plan.kind == 2) return launch_block_linear_fused_tiles(x, q_w, s_w, y, M, N, K, dev, st);
   // staged: quantized activations in the workspace, after the GEMM's own scratch
-  (void)plan;
   const GemmPlan gp = plan_block_linear(M, N, K, dev.sm_count, false);
   uint8_t* qa = static_cast<uint8_t*>(workspace) + ((gp.workspace + 255) / 256) * 256;
   float* sa = reinterpret_cast<float*>(qa + ((M * K + 255) / 256) * 256);
