@@ -28,7 +28,10 @@
 //                once every CTA's MMA has released stage s (multicast commit).
 //   warp 1       MMA issuer (warp-wide loop, lane 0 issues): 4 MMAs per chunk
 //                (M=128, N=256, K=32) into one of two 256-column TMEM buffers.
-//   warp 2       TMEM owner.
+//   warp 2       TMEM owner, then the slice sender: once the quantizers
+//                have written their rows, bulk-copies them (and the scales)
+//                into the other CTAs' shared memory, completion counted in
+//                bytes on the receivers' barriers (no multicast).
 //   warps 4-11   promotion as in the unfused kernel, s_a from the ring.
 // Registers: the block launches with 512 x 128; warps 0-3 drop to 40, the
 // promotion warpgroups take 176 and the quantizers 120 (sum = launch total).
@@ -76,8 +79,10 @@ constexpr int SMEM_X_OFF = SMEM_B_OFF + STAGES * B_BYTES;
 constexpr int SMEM_SA_OFF = SMEM_X_OFF + XSLOTS * X_BYTES;
 constexpr int SMEM_BAR_OFF = SMEM_SA_OFF + SA_SLOTS * BM * 4;
 // xfull[X], xempty[X], wfull[S], wempty[S], aempty[S], qdone[S], tfull[2],
-// tempty[2], sfull[SA], drain
-constexpr int NUM_BARS = 2 * XSLOTS + 4 * STAGES + 4 + SA_SLOTS + 1;
+// tempty[2], sfull[SA], drain, slice[S]
+constexpr int NUM_BARS = 2 * XSLOTS + 5 * STAGES + 4 + SA_SLOTS + 1;
+constexpr uint32_t SLICE_BYTES = QROWS * 128;      // one CTA's rows of codes
+constexpr uint32_t SCALE_BYTES = QROWS * 4;        // and their scales
 constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NUM_BARS * 8;
 constexpr int SMEM_BYTES = SMEM_MISC_OFF + 16 + 1024;   // + slack for 1024-byte alignment
 
@@ -89,6 +94,16 @@ struct FusedArgs {
 };
 
 __device__ __forceinline__ void record_error(int* err, int code) { atomicCAS(err, 0, code); }
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -117,6 +132,7 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
   auto tempty = [&](uint32_t b) { return bar_base + 8u * (2 * XSLOTS + 4 * STAGES + 2 + b); };
   auto sfull = [&](uint32_t k) { return bar_base + 8u * (2 * XSLOTS + 4 * STAGES + 4 + k); };
   const uint32_t drain_bar = bar_base + 8u * (2 * XSLOTS + 4 * STAGES + 4 + SA_SLOTS);
+  auto slice = [&](uint32_t s) { return bar_base + 8u * (2 * XSLOTS + 4 * STAGES + 5 + SA_SLOTS + s); };
   const uint32_t sa_base = smem_base + SMEM_SA_OFF;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SMEM_MISC_OFF);
 
@@ -140,14 +156,15 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(wfull(s), 1);
       ptx::mbar_init(wempty(s), 1);
-      ptx::mbar_init(aempty(s), CL);                       // one commit per CTA
-      ptx::mbar_init(qdone(s), CL * NUM_QUANT_WARPS);      // every quantizer warp
+      ptx::mbar_init(aempty(s), CL);                  // one commit per CTA
+      ptx::mbar_init(qdone(s), 1);                    // local arrival + remote bytes
+      ptx::mbar_init(slice(s), NUM_QUANT_WARPS);      // this CTA's rows written
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(tfull(b), 1);
       ptx::mbar_init(tempty(b), NUM_EPI_WARPS);
     }
-    for (int k = 0; k < SA_SLOTS; ++k) ptx::mbar_init(sfull(k), CL * NUM_QUANT_WARPS);
+    for (int k = 0; k < SA_SLOTS; ++k) ptx::mbar_init(sfull(k), 1);
     ptx::mbar_init(drain_bar, 1);
     ptx::fence_barrier_init();
     ptx::prefetch_tmap(&tmap_x);
@@ -176,7 +193,7 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
         const uint32_t xs = c % XSLOTS;
         const uint32_t ph = (c / XSLOTS) & 1u;
         if (c >= XSLOTS) {
-          ok = __all_sync(0xffffffffu, ptx::mbar_wait_spin(xempty(xs), ph ^ 1u));
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(xempty(xs), ph ^ 1u));
           if (!ok) {
             if (lane == 0) record_error(args.err, kErrTimeoutProducer);
             break;
@@ -211,7 +228,7 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
         const uint32_t s = c % STAGES;
         const uint32_t ph = (c / STAGES) & 1u;
         if (c >= STAGES) {
-          ok = __all_sync(0xffffffffu, ptx::mbar_wait_spin(wempty(s), ph ^ 1u));
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(wempty(s), ph ^ 1u));
           if (!ok) {
             if (lane == 0) record_error(args.err, kErrTimeoutProducer);
             break;
@@ -241,7 +258,7 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
         const uint32_t sph = (c / STAGES) & 1u;
         const uint32_t buf = c & 1u;
         const uint32_t bph = (c >> 1) & 1u;
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait_spin_cluster(qdone(s), sph) &&
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait_spin(qdone(s), sph) &&
                                          ptx::mbar_wait_spin(wfull(s), sph) &&
                                          ptx::mbar_wait_spin(tempty(buf), bph ^ 1u));
         if (!ok) {
@@ -271,6 +288,39 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
       if (!ptx::mbar_wait(drain_bar, 0)) record_error(args.err, kErrTimeoutMma);
     }
     __syncwarp();
+  } else if (warp == 2) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+    // ----------------------------------------------------- slice sender
+    // Once this CTA's quantizers have written their rows of chunk c, send
+    // the slice (codes and scales) to the other CTAs, counted in bytes on
+    // their barriers, and arrive locally expecting the other three slices.
+    uint32_t c = 0;
+    bool ok = true;
+    for (int u = cluster_id; u < num_units && ok; u += num_clusters) {
+      for (int kb = 0; kb < num_kb; ++kb, ++c) {
+        const uint32_t s = c % STAGES;
+        const uint32_t slot = c % SA_SLOTS;
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait_spin(slice(s), (c / STAGES) & 1u));
+        if (!ok) {
+          if (lane == 0) record_error(args.err, kErrTimeoutProducer);
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t a_src = smem_base + SMEM_A_OFF + s * A_BYTES + rank * SLICE_BYTES;
+          const uint32_t s_src = sa_base + (slot * BM + rank * QROWS) * 4u;
+          for (uint32_t k = 1; k < CL; ++k) {
+            const uint32_t dst = (rank + k) % CL;
+            ptx::bulk_copy_s2s(ptx::map_to_cta(a_src, dst), a_src, SLICE_BYTES,
+                               ptx::map_to_cta(qdone(s), dst));
+            ptx::bulk_copy_s2s(ptx::map_to_cta(s_src, dst), s_src, SCALE_BYTES,
+                               ptx::map_to_cta(sfull(slot), dst));
+          }
+          ptx::mbar_arrive_expect_tx(qdone(s), (CL - 1) * SLICE_BYTES);
+          ptx::mbar_arrive_expect_tx(sfull(slot), (CL - 1) * SCALE_BYTES);
+        }
+        __syncwarp();
+      }
+    }
   } else if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
   } else if (warp >= FIRST_QUANT_WARP) {
@@ -326,21 +376,15 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
           ok = false;
           break;
         }
-        const uint32_t adst = smem_base + SMEM_A_OFF + s * A_BYTES + rt * 128u;
-        const uint32_t sdst = sa_base + ((c % SA_SLOTS) * BM + rt) * 4u;
+        const uint32_t astage = smem_base + SMEM_A_OFF + s * A_BYTES;
+        const uint32_t slot = c % SA_SLOTS;
 #pragma unroll
-        for (uint32_t k = 0; k < CL; ++k) {
-#pragma unroll
-          for (uint32_t t = 0; t < 2; ++t)
-            ptx::st_cluster_v4(ptx::map_to_cta(adst + (((2u * part + t) ^ sw) << 4), k), code[t]);
-          if (part == 0) ptx::st_cluster_f32(ptx::map_to_cta(sdst, k), scale);
-        }
-        ptx::fence_proxy_async_cluster();   // codes visible to every CTA's tensor core
+        for (uint32_t t = 0; t < 2; ++t)
+          sts128(astage + rt * 128u + (((2u * part + t) ^ sw) << 4), code[t]);
+        if (part == 0) sts32(sa_base + (slot * BM + rt) * 4u, __float_as_uint(scale));
+        ptx::fence_proxy_async_smem();   // visible to the tensor core and the bulk copies
         __syncwarp();
-        if (lane < CL) {
-          ptx::mbar_arrive_remote(ptx::map_to_cta(qdone(s), static_cast<uint32_t>(lane)));
-          ptx::mbar_arrive_remote(ptx::map_to_cta(sfull(c % SA_SLOTS), static_cast<uint32_t>(lane)));
-        }
+        if (lane == 0) ptx::mbar_arrive(slice(s));
       }
     }
   } else {
@@ -374,8 +418,7 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
         const uint32_t buf = c & 1u;
         const uint32_t bph = (c >> 1) & 1u;
         if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(tfull(buf), bph) &&
-                                         ptx::mbar_wait_spin_cluster(sfull(c % SA_SLOTS),
-                                                                     (c / SA_SLOTS) & 1u))) {
+                                         ptx::mbar_wait_spin(sfull(c % SA_SLOTS), (c / SA_SLOTS) & 1u))) {
           if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
           ok = false;
           break;

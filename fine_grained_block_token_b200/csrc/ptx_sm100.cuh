@@ -282,50 +282,16 @@ __device__ __forceinline__ uint32_t map_to_cta(uint32_t addr, uint32_t rank) {
   return r;
 }
 
-// Stores into (possibly another CTA's) shared memory at a shared::cluster address.
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-               "r"(v.z), "r"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(addr), "r"(__float_as_uint(v)) : "memory");
-}
-
-// Orders this thread's generic-proxy shared-memory writes (local or in other
-// CTAs of the cluster) before later async-proxy accesses (the tensor core).
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
-}
-
-// Arrive on an mbarrier in any CTA of the cluster, releasing this thread's
-// prior writes at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
-// Bounded polling wait (as mbar_wait_spin) with cluster-scope acquire, for
-// barriers that other CTAs of the cluster arrive on.
-__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to
+// `dst` in any CTA of the cluster; completion is counted in bytes on the
+// mbarrier `bar` of the destination CTA (both shared::cluster addresses).
+// Not a multicast operation.
+__device__ __forceinline__ void bulk_copy_s2s(uint32_t dst, uint32_t src, uint32_t bytes,
+                                              uint32_t bar) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
       : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_spin_cluster(uint32_t bar, uint32_t parity,
-                                                       uint64_t limit_cycles = 1ull << 32) {
-  if (mbar_test_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = clock64();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_test_wait_cluster(bar, parity)) return true;
-    if ((i & 255u) == 0 && clock64() - t0 > limit_cycles) return false;
-  }
 }
 
 // Arrive (once) on the mbarrier at shared offset `bar` in every CTA of
