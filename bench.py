@@ -14,8 +14,12 @@ Prints ONE JSON line (rank 0).  `value` is whole-job TFLOP/s (2 M N K per
 linear, all ranks) over the device-timed K steps (CUDA events, max over
 ranks).  `e2e` repeats the measurement through the public API with the
 inputs copied from pinned host memory and the outputs copied back inside
-every step.  `roofline` covers the dominant kernel (the block-scaled GEMM)
-against the measured peaks in MEASURED_PEAKS.json.  `cpu_baseline` and
+every step.  `roofline` covers the dominant kernel (the block-scaled GEMM;
+for the decode workload the weight-streaming decode kernel, against HBM)
+against the measured peaks in MEASURED_PEAKS.json, from a second pass with
+events around every kernel.  `fused` times fp8_block_linear_fused (the
+activation quantization inside the GEMM) on the same inputs and checks its
+output equals the two-call path bit for bit.  `cpu_baseline` and
 `--impl reference` time the plain CPU oracle on a bounded row sample.
 """
 from __future__ import annotations
@@ -295,18 +299,27 @@ def run_ours(args):
     sampler.start()
     time.sleep(0.3)
 
-    # ---- device-timed region: K steps, per-kernel events inside
+    # ---- device-timed region: K whole steps, nothing else on the stream
     n = len(items)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4 * n)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     barrier()
     t_start.record()
     for k in range(args.steps):
-        step(evs[k])
+        step()
     t_end.record()
     barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
+    fp8.check()
+
+    # ---- the same K steps again with events around every kernel, for the
+    # per-kernel rates (the event records themselves cost a few us each,
+    # which matters next to decode-sized kernels, hence the separate pass)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4 * n)] for _ in range(args.steps)]
+    barrier()
+    for k in range(args.steps):
+        step(evs[k])
+    barrier()
     act_ms = sum(e[4 * i].elapsed_time(e[4 * i + 1]) for e in evs for i in range(n))
     gemm_ms = sum(e[4 * i + 2].elapsed_time(e[4 * i + 3]) for e in evs for i in range(n))
     fp8.check()
@@ -336,14 +349,41 @@ def run_ours(args):
     b.record()
     barrier()
     e2e_ms = a.elapsed_time(b)
+    # ---- the fused entry point (activation quantization inside the GEMM)
+    # on the same inputs and steps; its output must equal the two-call one
+    y_ref = [it["y"].clone() for it in items]
+    fws = []
+    for it in items:
+        nb = fp8.fused_workspace_bytes(it["M"], it["N"], it["K"])
+        fws.append(torch.empty(max(nb, 16), dtype=torch.uint8, device=dev))
+
+    def fused_step():
+        for it, w in zip(items, fws):
+            fp8.block_linear_fused(it["x"], it["q_w"], it["s_w"], it["y"], w)
+
+    for _ in range(min(args.warmup, 3)):
+        fused_step()
+    torch.cuda.synchronize()
+    fused_identical = all(torch.equal(r.view(torch.int16), it["y"].view(torch.int16))
+                          for r, it in zip(y_ref, items))
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier()
+    a.record()
+    for _ in range(args.steps):
+        fused_step()
+    b.record()
+    barrier()
+    fused_ms = a.elapsed_time(b)
     sampler.stop()
     fp8.check()
 
     # max over ranks
-    vals = torch.tensor([elapsed_ms, e2e_ms, act_ms, gemm_ms], dtype=torch.float64, device=dev)
+    vals = torch.tensor([elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms], dtype=torch.float64,
+                        device=dev)
     if world > 1:
         dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms, act_ms, gemm_ms = vals.tolist()
+    elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms = vals.tolist()
 
     ms_per_step = elapsed_ms / args.steps
     value = world * flops_step * args.steps / (elapsed_ms * 1e-3) / 1e12
@@ -351,6 +391,14 @@ def run_ours(args):
     gemm_tflops = gemm_flops_step * args.steps / (gemm_ms * 1e-3) / 1e12
     act_gbs = act_bytes_step * args.steps / (act_ms * 1e-3) / 1e9
     launches_per_step = 2 * n
+    fused_value = world * flops_step * args.steps / (fused_ms * 1e-3) / 1e12
+    decode = args.workload == "llama3_decode"
+    # decode linears are bound by streaming the weights: algorithmic bytes =
+    # codes + block scales of W, codes + group scales of X, bf16 Y
+    gemm_bytes_step = sum(it["N"] * it["K"] + (it["N"] // 128) * (it["K"] // 128) * 4 +
+                          it["M"] * it["K"] + it["M"] * (it["K"] // 128) * 4 + 2 * it["M"] * it["N"]
+                          for it in items)
+    gemm_gbs = gemm_bytes_step * args.steps / (gemm_ms * 1e-3) / 1e9
 
     if rank == 0:
         parity = None
@@ -381,16 +429,25 @@ def run_ours(args):
                        "linears": {it["label"]: [it["M"], it["N"], it["K"]] for it in items},
                        "l2": "no flush: inputs of a step exceed the 126 MB L2",
                        "parallelism": f"replicas x{world} (no data-path collective)"},
-            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak,
-                         "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
-                         "traffic": traffic,
-                         "kernel": "gemm_prefill_kernel",
-                         "peak_source": f"{peak_src} bf16 burst x {FP8_OVER_BF16} (nominal fp8/bf16)",
-                         "ms_per_launch": gemm_ms_per_launch},
+            "roofline": ({"bound": "hbm", "achieved": gemm_gbs, "peak": hbm_peak,
+                          "unit": "GB/s", "frac": gemm_gbs / hbm_peak, "traffic": None,
+                          "kernel": "decode_kernel", "peak_source": f"{peak_src} copy",
+                          "ms_per_launch": gemm_ms_per_launch,
+                          "tflops": gemm_tflops} if decode else
+                         {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak,
+                          "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
+                          "traffic": traffic,
+                          "kernel": "gemm_prefill_kernel",
+                          "peak_source": f"{peak_src} bf16 burst x {FP8_OVER_BF16} (nominal fp8/bf16)",
+                          "ms_per_launch": gemm_ms_per_launch}),
             "act_quant": {"achieved": act_gbs, "peak": hbm_peak, "unit": "GB/s",
                           "frac": act_gbs / hbm_peak, "peak_source": f"{peak_src} copy"},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "fused": {"value": fused_value, "unit": "TFLOP/s", "ms_per_step": fused_ms / args.steps,
+                      "vs_two_call": ms_per_step / (fused_ms / args.steps),
+                      "kernel": "decode_kernel after act_quant (staged)" if decode else "gemm_fused_kernel",
+                      "identical_to_two_call": fused_identical},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary(),
             "cpu_baseline": cpu,

@@ -190,3 +190,25 @@ def test_fused_prefill_size_bit_identical(fp8):
     y2 = fp8.block_linear_fused(x, q_w, s_w)
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("M,N,K", [(8192, 2048, 1024), (4096, 4096, 2048), (640, 1280, 1152)])
+def test_fused_repeated_runs_bit_identical(fp8, M, N, K):
+    """The fused kernel at sizes where each CTA cluster processes several
+    (row band, group of N-tiles) units -- with a partly empty last group
+    (N = 1280) and an odd chunk count (K = 1152) -- run ten times: Y must
+    equal the unfused result every time.  A hand-off race between the fused
+    kernel's warps or CTAs shows up as an intermittent mismatch."""
+    xb = wl.sweep_x(M, K)
+    wb = wl.normal((N, K), 0.02, 1, M + N + K)
+    x, w = to_dev(xb), to_dev(wb)
+    q_w, s_w = fp8.quant_weight(w)
+    q_a, s_a = fp8.quant_act(x)
+    y1 = fp8.block_linear(q_a, s_a, q_w, s_w)
+    y2 = torch.empty_like(y1)
+    for rep in range(10):
+        y2.fill_(0)
+        fp8.block_linear_fused(x, q_w, s_w, y2)
+        torch.cuda.synchronize()
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), (M, N, K, rep)
+    fp8.check()
