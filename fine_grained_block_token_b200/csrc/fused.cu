@@ -90,8 +90,24 @@ struct FusedArgs {
   const float* s_w;
   __nv_bfloat16* y;
   int M, N, K;
+  int group_m;       // row bands per raster group (see unit_coords)
   int* err;
 };
+
+// Unit u -> (row band, group of CL N-tiles).  Row bands are taken in groups
+// of group_m; within a group the N-groups are outer and the bands inner, so
+// the clusters running together share a few activation bands (which stay in
+// L2 while every N-group passes over them) and a few weight groups.
+__device__ __forceinline__ void unit_coords(int u, int num_m, int num_g, int group_m, int& m_blk,
+                                            int& g) {
+  const int per_group = group_m * num_g;
+  const int grp = u / per_group;
+  const int base = grp * group_m;
+  const int gm = min(group_m, num_m - base);
+  const int idx = u - grp * per_group;
+  g = idx / gm;
+  m_blk = base + idx % gm;
+}
 
 __device__ __forceinline__ void record_error(int* err, int code) { atomicCAS(err, 0, code); }
 
@@ -187,7 +203,8 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
     uint32_t c = 0;
     bool ok = true;
     for (int u = cluster_id; u < num_units && ok; u += num_clusters) {
-      const int m_blk = u % num_m;
+      int m_blk, g;
+      unit_coords(u, num_m, num_g, args.group_m, m_blk, g);
       const int row0 = m_blk * BM + static_cast<int>(rank) * QROWS;
       for (int kb = 0; kb < num_kb; ++kb, ++c) {
         const uint32_t xs = c % XSLOTS;
@@ -223,7 +240,9 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
     uint32_t c = 0;
     bool ok = true;
     for (int u = cluster_id; u < num_units && ok; u += num_clusters) {
-      const int n_blk = (u / num_m) * CL + static_cast<int>(rank);
+      int m_blk, g;
+      unit_coords(u, num_m, num_g, args.group_m, m_blk, g);
+      const int n_blk = g * CL + static_cast<int>(rank);
       for (int kb = 0; kb < num_kb; ++kb, ++c) {
         const uint32_t s = c % STAGES;
         const uint32_t ph = (c / STAGES) & 1u;
@@ -399,8 +418,9 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
     uint32_t c = 0;
     bool ok = true;
     for (int u = cluster_id; u < num_units && ok; u += num_clusters) {
-      const int m_blk = u % num_m;
-      const int n_blk = (u / num_m) * CL + static_cast<int>(rank);
+      int m_blk, g;
+      unit_coords(u, num_m, num_g, args.group_m, m_blk, g);
+      const int n_blk = g * CL + static_cast<int>(rank);
       const int row = m_blk * BM + r;
       const int nb = n_blk * 2 + half;
       const bool row_ok = row < M;
@@ -520,6 +540,13 @@ cudaError_t launch_block_linear_fused_tiles(const void* x, const void* q_w, cons
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
+  // row bands per raster group: their bf16 activations (128 x K x 2 bytes
+  // each) fit in ~40 MB of L2
+  const int64_t num_m = (M + BM - 1) / BM;
+  const int64_t band_bytes = static_cast<int64_t>(BM) * K * 2;
+  int64_t gm = (int64_t{40} << 20) / band_bytes;
+  gm = gm < 1 ? 1 : (gm > num_m ? num_m : gm);
+  a.group_m = static_cast<int>(gm);
   a.err = dev.error_flag;
   const int64_t units = ((M + BM - 1) / BM) * ((((N + BN - 1) / BN) + CL - 1) / CL);
   const int clusters = static_cast<int>(units < max_clusters ? units : max_clusters);
