@@ -8,6 +8,7 @@
 
 #include "../../include/fp8bl.h"
 #include "fp8bl_internal.h"
+#include "ptx_sm100.cuh"
 
 namespace fp8bl {
 namespace {
@@ -195,6 +196,35 @@ fp8bl_status fp8_block_linear_fused(const void* x_bf16, const void* q_w, const f
   }
   return from_cuda(launch_block_linear_fused(x_bf16, q_w, s_w, y_bf16, M, N, K, plan, workspace,
                                              *d, as_cuda(stream)));
+}
+
+namespace fp8bl {
+namespace {
+// One thread waits on a freshly initialised mbarrier (phase 0 never
+// completes) with the kernels' bounded waits; on expiry it records the
+// timeout exactly as the GEMM and quantization kernels do.
+__global__ void selftest_wait_kernel(uint64_t limit_cycles, int kind, int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    const uint32_t b = ptx::smem_u32(&bar);
+    ptx::mbar_init(b, 1);
+    ptx::fence_barrier_init();
+    const bool ok = kind == 0 ? ptx::mbar_wait(b, 0, limit_cycles)
+                              : ptx::mbar_wait_spin(b, 0, limit_cycles);
+    if (!ok) atomicCAS(err, 0, kErrTimeoutSelftest);
+  }
+}
+}  // namespace
+}  // namespace fp8bl
+
+fp8bl_status fp8bl_selftest_wait_timeout(uint64_t limit_cycles, int kind, fp8bl_stream_t stream) {
+  if (limit_cycles == 0 || limit_cycles > (uint64_t{1} << 32) || (kind != 0 && kind != 1))
+    return FP8BL_ERR_SHAPE;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, as_cuda(stream)>>>(limit_cycles, kind, d->error_flag);
+  return from_cuda(cudaGetLastError());
 }
 
 fp8bl_status fp8bl_check(fp8bl_stream_t stream) {

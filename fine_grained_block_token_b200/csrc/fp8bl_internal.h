@@ -75,6 +75,7 @@ enum KernelError : int {
   kErrTimeoutProducer = 1,
   kErrTimeoutMma = 2,
   kErrTimeoutEpilogue = 3,
+  kErrTimeoutSelftest = 4,
 };
 
 }  // namespace fp8bl

@@ -183,6 +183,21 @@ size_t fp8_block_linear_fused_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * FP8BL_OK (or FP8BL_ERR_CUDA if the synchronisation itself failed). */
 fp8bl_status fp8bl_check(fp8bl_stream_t stream);
 
+/*
+ * fp8bl_selftest_wait_timeout -- exercises the kernels' failure detection
+ * (no counterpart on the pages).  Enqueues on `stream` a one-thread kernel
+ * that waits on an mbarrier nothing ever arrives on, with the bounded wait
+ * the library's kernels use, limited to `limit_cycles` SM clock cycles
+ * (kind 0: the suspending wait, kind 1: the polling wait).  When the limit
+ * runs out the kernel records a timeout in the library's error word and
+ * returns, so the next fp8bl_check(stream) returns FP8BL_ERR_TIMEOUT (and
+ * clears it) and the device stays usable.  No memory is touched besides
+ * the error word.
+ *   limit_cycles: 1 .. 2^32;  kind: 0 or 1;  otherwise FP8BL_ERR_SHAPE.
+ */
+fp8bl_status fp8bl_selftest_wait_timeout(uint64_t limit_cycles, int kind,
+                                          fp8bl_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char *fp8bl_status_string(fp8bl_status status);
 

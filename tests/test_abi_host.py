@@ -123,3 +123,14 @@ def test_workspace_query_never_fails(lib):
     f.restype = ctypes.c_size_t
     assert f(4, 100, 128) == 0
     assert f(-1, 128, 128) == 0
+
+
+def test_selftest_wait_timeout_rejects_bad_arguments(lib):
+    """The failure-detection self-test validates its arguments on the host."""
+    f = lib.fp8bl_selftest_wait_timeout
+    f.argtypes = [ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    assert f(0, 0, None) == 2
+    assert f((1 << 32) + 1, 0, None) == 2
+    assert f(1000, 2, None) == 2
+    assert f(1000, -1, None) == 2
