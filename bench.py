@@ -198,10 +198,36 @@ def within_tolerance(y, R):
     return float(np.max(np.abs(y - R) / np.maximum(lim, 1e-300)))
 
 
+# ------------------------------------------------------ multi-process host
+
+def rank_info():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(values, device, world: int):
+    """Element-wise maximum of `values` over all ranks (device-timed numbers
+    are reported as the slowest rank's).  `device` is where the collective
+    runs: the GPU under NCCL, the CPU under gloo."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(world: int, work_per_step: float, steps: int, elapsed_ms: float) -> float:
+    """Replicas: every rank runs the same steps, so the job does world x the
+    work of one rank in the slowest rank's time (weak scaling)."""
+    return world * work_per_step * steps / (elapsed_ms * 1e-3)
+
+
 def run_reference(args):
     """The oracle, as it stands, on the host cores: one bounded row sample of
     the workload per step.  Under torchrun only rank 0 works."""
-    rank = int(os.environ.get("RANK", "0"))
+    _, rank, _ = rank_info()
     if rank != 0:
         return 0
     lins = workload_linears(args.workload)
@@ -236,9 +262,7 @@ def run_ours(args):
 
     import fine_grained_block_token_b200 as fp8
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_info()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -379,19 +403,16 @@ def run_ours(args):
     fp8.check()
 
     # max over ranks
-    vals = torch.tensor([elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms], dtype=torch.float64,
-                        device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms = vals.tolist()
+    elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms = max_over_ranks(
+        [elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms], dev, world)
 
     ms_per_step = elapsed_ms / args.steps
-    value = world * flops_step * args.steps / (elapsed_ms * 1e-3) / 1e12
-    e2e_value = world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_rate(world, flops_step, args.steps, elapsed_ms) / 1e12
+    e2e_value = whole_job_rate(world, flops_step, e2e_steps, e2e_ms) / 1e12
     gemm_tflops = gemm_flops_step * args.steps / (gemm_ms * 1e-3) / 1e12
     act_gbs = act_bytes_step * args.steps / (act_ms * 1e-3) / 1e9
     launches_per_step = 2 * n
-    fused_value = world * flops_step * args.steps / (fused_ms * 1e-3) / 1e12
+    fused_value = whole_job_rate(world, flops_step, args.steps, fused_ms) / 1e12
     decode = args.workload == "llama3_decode"
     # decode linears are bound by streaming the weights: algorithmic bytes =
     # codes + block scales of W, codes + group scales of X, bf16 Y
