@@ -249,7 +249,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         // After a timed-out wait this warp stops touching TMEM but keeps
         // walking its range, so that every named barrier below is reached
         // by all four promotion warps.
-        if (ok && !ptx::mbar_wait(tfull_bar(buf), bph)) {
+        if (ok && !ptx::mbar_wait_spin(tfull_bar(buf), bph)) {
           record_error(args.err, kErrTimeoutEpilogue);
           ok = false;
         }
@@ -285,16 +285,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                          (static_cast<int64_t>(g) * args.maxseg + (blk - first_blk)) * (MPAD * 128);
 #pragma unroll
             for (int m = 0; m < MPAD; ++m) dst[m * 128 + n_local] = acc[m];
-            // publish the partial and count this CTA in; the last one reduces
-            __threadfence();
+            // publish the partial and count this CTA in; the last one reduces.
+            // The barrier orders every thread's stores before one thread's
+            // fence + atomic (the fence is cumulative), as a grid-wide
+            // barrier does; the last CTA fences again before reading.
             ptx::named_barrier_sync(1, 128);
             __shared__ int last_flag;
             const int g_lo = static_cast<int>(((blk_u0 + 1) * args.G - 1) / args.units);
             const int g_hi = static_cast<int>(((blk_u0 + KB) * args.G - 1) / args.units);
-            if (threadIdx.x == 128) last_flag = atomicAdd(args.counters + blk, 1) == g_hi - g_lo;
+            if (threadIdx.x == 128) {
+              __threadfence();
+              last_flag = atomicAdd(args.counters + blk, 1) == g_hi - g_lo;
+              if (last_flag) __threadfence();
+            }
             ptx::named_barrier_sync(1, 128);
             if (last_flag) {
-              __threadfence();
               // sum the block's partials in increasing CTA order; the loads
               // of UR partials are in flight together
               constexpr int UR = MPAD <= 16 ? 4 : (MPAD <= 32 ? 2 : 1);
