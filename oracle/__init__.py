@@ -11,7 +11,9 @@ encoder written from the format definition); this module compiles it with gcc
 Sources (transformers docs, "Fine-grained FP8" page):
   * opening bullet list -- 128 x 128 weight blocks, per-token activation
     groups of 128 along the input channel;
-  * "DeepGEMM fast path" section -- the dynamic activation scheme.
+  * "DeepGEMM fast path" section -- the dynamic activation scheme;
+  * "UE8M0 scale format" section -- power-of-two scales stored as
+    float8_e8m0fnu (the ``*_ue8m0`` functions).
 The readings the pages leave open (scale formula, rounding, eps) are stated
 in the header comment of ``fp8bl_oracle.c``.
 """
@@ -68,6 +70,16 @@ def bind(path: str):
     lib.oracle_block_linear_rows.argtypes = [vp, vp, vp, vp, i64, i64, i64,
                                                  vp, i64, vp, ip]
     lib.oracle_block_linear_rows.restype = ctypes.c_int
+    lib.oracle_ue8m0_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_ue8m0_decode.restype = ctypes.c_double
+    lib.oracle_ue8m0_from_amax.argtypes = [ctypes.c_float]
+    lib.oracle_ue8m0_from_amax.restype = ctypes.c_uint8
+    lib.oracle_quant_act_ue8m0_rows.argtypes = [vp, i64, i64, vp, vp, i64, i64]
+    lib.oracle_quant_act_ue8m0_rows.restype = None
+    lib.oracle_quant_act_ue8m0.argtypes = [vp, i64, i64, vp, vp, ip]
+    lib.oracle_quant_act_ue8m0.restype = None
+    lib.oracle_quant_weight_ue8m0.argtypes = [vp, i64, i64, vp, vp]
+    lib.oracle_quant_weight_ue8m0.restype = None
     return lib
 
 
@@ -187,6 +199,75 @@ def block_linear(q_a, s_a, q_w, s_w, rows=None, nthreads: int = 1) -> np.ndarray
         if rc != 0:
             raise MemoryError("oracle allocation failed")
     return y
+
+
+# ------------------------------------------------------------ UE8M0 scales
+# "Fine-grained FP8" page, "UE8M0 scale format" section: scales kept as
+# float8_e8m0fnu (scale_fmt="ue8m0").  Readings R6-R8 in fp8bl_oracle.c:
+# the scale is the fp32 scale rounded up to a power of two 2^e, stored as
+# the byte e + 127, and q = e4m3(x * 2^-e).
+
+
+def ue8m0_decode(codes) -> np.ndarray:
+    """fp64 values 2^(c - 127) of ue8m0 codes (NaN for 255)."""
+    lib = _load()
+    c = np.asarray(codes, dtype=np.uint8)
+    table = np.array([lib.oracle_ue8m0_decode(i) for i in range(256)], dtype=np.float64)
+    return table[c]
+
+
+def ue8m0_from_amax(amax: float) -> int:
+    """ue8m0 code of the scale of a group whose largest magnitude is ``amax``."""
+    return int(_load().oracle_ue8m0_from_amax(float(np.float32(amax))))
+
+
+def quant_act_ue8m0(x_bf16, nthreads: int = 1):
+    """Per-token 1 x 128 activation quantization with UE8M0 scales.
+
+    Returns (q uint8 [M, K] e4m3 codes, s uint8 [M, K/128] ue8m0 codes)."""
+    x = _as_bf16_bits(x_bf16)
+    M, K = x.shape
+    if K % BLOCK:
+        raise ValueError("K must be a multiple of 128")
+    q = np.empty((M, K), dtype=np.uint8)
+    s = np.empty((M, K // BLOCK), dtype=np.uint8)
+    if M:
+        _load().oracle_quant_act_ue8m0(_ptr(x), M, K, _ptr(q), _ptr(s), int(nthreads))
+    return q, s
+
+
+def quant_act_ue8m0_rows(x_bf16, m0: int, m1: int):
+    """UE8M0 quantization of rows m0..m1-1 only (single thread)."""
+    x = _as_bf16_bits(x_bf16)
+    M, K = x.shape
+    sub = np.ascontiguousarray(x[m0:m1])
+    q = np.empty((m1 - m0, K), dtype=np.uint8)
+    s = np.empty((m1 - m0, K // BLOCK), dtype=np.uint8)
+    if m1 > m0:
+        _load().oracle_quant_act_ue8m0_rows(_ptr(sub), m1 - m0, K, _ptr(q), _ptr(s), 0, m1 - m0)
+    return q, s
+
+
+def quant_weight_ue8m0(w_bf16):
+    """128 x 128 block weight quantization with UE8M0 scales.
+
+    Returns (q uint8 [N, K], s uint8 [N/128, K/128] ue8m0 codes)."""
+    w = _as_bf16_bits(w_bf16)
+    N, K = w.shape
+    if N % BLOCK or K % BLOCK:
+        raise ValueError("N and K must be multiples of 128")
+    q = np.empty((N, K), dtype=np.uint8)
+    s = np.empty((N // BLOCK, K // BLOCK), dtype=np.uint8)
+    _load().oracle_quant_weight_ue8m0(_ptr(w), N, K, _ptr(q), _ptr(s))
+    return q, s
+
+
+def block_linear_ue8m0(q_a, c_a, q_w, c_w, rows=None, nthreads: int = 1) -> np.ndarray:
+    """fp64 result of the block-scaled linear whose scales are ue8m0 codes:
+    the same sum as ``block_linear`` with s = 2^(c - 127) (exact in fp32)."""
+    s_a = ue8m0_decode(c_a).astype(np.float32)
+    s_w = ue8m0_decode(c_w).astype(np.float32)
+    return block_linear(q_a, s_a, q_w, s_w, rows=rows, nthreads=nthreads)
 
 
 def bf16_rne(y: np.ndarray) -> np.ndarray:

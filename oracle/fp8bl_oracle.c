@@ -185,6 +185,106 @@ void oracle_quant_weight(const uint16_t *w, int64_t N, int64_t K,
     }
 }
 
+/* ------------------------------------------------- UE8M0 scale variant
+ *
+ * "Fine-grained FP8" page, "UE8M0 scale format" section: DeepSeek-V4-style
+ * checkpoints keep the FP8 weight scales as packed float8_e8m0fnu values
+ * instead of float32 (scale_fmt="ue8m0"), and on Blackwell the DeepGEMM
+ * expert kernels accept only these.  The section gives neither how a scale
+ * becomes a power of two nor a layout.  Readings used here:
+ *   R6  a ue8m0 code c is an unsigned biased exponent: value 2^(c - 127),
+ *       c = 255 is NaN (the float8_e8m0fnu format); no sign, no zero.
+ *   R7  the scale of a group or block is the smallest power of two
+ *       s = 2^e with max(amax, EPS) <= 448 * s, i.e. the fp32 scale of R3
+ *       rounded UP to a power of two, so the largest element still maps
+ *       inside +-448 and nothing saturates; stored as c = e + 127, one byte
+ *       per scale, in the same [M, K/128] and [N/128, K/128] grids.
+ *   R8  q = encode(RN32(x * 2^-e)): the product is exact in fp64 and is
+ *       rounded once to fp32 (the only rounding besides the e4m3 one; it
+ *       matters only when x * 2^-e underflows fp32, where e4m3 gives 0).
+ *   The GEMM is R5 with s = 2^(c - 127).
+ */
+
+/* R6 */
+double oracle_ue8m0_decode(uint8_t c)
+{
+    if (c == 255)
+        return NAN;
+    return ldexp(1.0, (int)c - 127);
+}
+
+/* R7: the least e with a <= 448 * 2^e, found by exact comparisons
+ * (448 * 2^e is exact in fp64, and so is the fp32 amax). */
+uint8_t oracle_ue8m0_from_amax(float amax)
+{
+    double a = amax > OR_AMAX_EPS ? (double)amax : (double)OR_AMAX_EPS;
+    int e;
+    frexp(a / 448.0, &e);                   /* starting guess */
+    while (ldexp(448.0, e - 1) >= a)
+        --e;
+    while (ldexp(448.0, e) < a)
+        ++e;
+    return (uint8_t)(e + 127);
+}
+
+/* R8 for one value, given the group's code c. */
+static uint8_t encode_pow2(float x, uint8_t c)
+{
+    double v = (double)x * ldexp(1.0, 127 - (int)c);   /* exact */
+    return oracle_e4m3_encode((float)v);
+}
+
+/* Activation quantization with UE8M0 scales, rows m0 .. m1-1.
+ * x: bf16 [M, K]; q: e4m3 [M, K]; s: ue8m0 codes [M, K/128]. */
+void oracle_quant_act_ue8m0_rows(const uint16_t *x, int64_t M, int64_t K,
+                                 uint8_t *q, uint8_t *s, int64_t m0, int64_t m1)
+{
+    (void)M;
+    int64_t G = K / OR_BLOCK;
+    for (int64_t m = m0; m < m1; ++m) {
+        for (int64_t g = 0; g < G; ++g) {
+            const uint16_t *xg = x + m * K + g * OR_BLOCK;
+            float amax = 0.0f;
+            for (int i = 0; i < OR_BLOCK; ++i) {
+                float a = fabsf(bf16_to_f32(xg[i]));
+                if (a > amax)
+                    amax = a;
+            }
+            uint8_t c = oracle_ue8m0_from_amax(amax);
+            s[m * G + g] = c;
+            for (int i = 0; i < OR_BLOCK; ++i)
+                q[m * K + g * OR_BLOCK + i] = encode_pow2(bf16_to_f32(xg[i]), c);
+        }
+    }
+}
+
+/* Weight quantization with UE8M0 scales, one per 128 x 128 block.
+ * w: bf16 [N, K]; q: e4m3 [N, K]; s: ue8m0 codes [N/128, K/128]. */
+void oracle_quant_weight_ue8m0(const uint16_t *w, int64_t N, int64_t K,
+                               uint8_t *q, uint8_t *s)
+{
+    int64_t NB = N / OR_BLOCK, KB = K / OR_BLOCK;
+    for (int64_t bi = 0; bi < NB; ++bi) {
+        for (int64_t bj = 0; bj < KB; ++bj) {
+            float amax = 0.0f;
+            for (int r = 0; r < OR_BLOCK; ++r)
+                for (int c = 0; c < OR_BLOCK; ++c) {
+                    float a = fabsf(bf16_to_f32(
+                        w[(bi * OR_BLOCK + r) * K + bj * OR_BLOCK + c]));
+                    if (a > amax)
+                        amax = a;
+                }
+            uint8_t code = oracle_ue8m0_from_amax(amax);
+            s[bi * KB + bj] = code;
+            for (int r = 0; r < OR_BLOCK; ++r)
+                for (int c = 0; c < OR_BLOCK; ++c) {
+                    int64_t idx = (bi * OR_BLOCK + r) * K + bj * OR_BLOCK + c;
+                    q[idx] = encode_pow2(bf16_to_f32(w[idx]), code);
+                }
+        }
+    }
+}
+
 /* ----------------------------------------------------------------- GEMM */
 
 /* R5 for the output rows listed in rows[0 .. nrows-1] (all N columns).
@@ -279,18 +379,22 @@ typedef struct {
     int64_t M, K;
     uint8_t *q;
     float *s;
+    uint8_t *s8;        /* UE8M0 codes instead of s when not NULL */
     int64_t m0, m1;
 } qa_job;
 
 static void *qa_rows(void *arg)
 {
     qa_job *j = (qa_job *)arg;
-    oracle_quant_act_rows(j->x, j->M, j->K, j->q, j->s, j->m0, j->m1);
+    if (j->s8)
+        oracle_quant_act_ue8m0_rows(j->x, j->M, j->K, j->q, j->s8, j->m0, j->m1);
+    else
+        oracle_quant_act_rows(j->x, j->M, j->K, j->q, j->s, j->m0, j->m1);
     return NULL;
 }
 
-void oracle_quant_act(const uint16_t *x, int64_t M, int64_t K, uint8_t *q,
-                      float *s, int nthreads)
+static void quant_act_threads(const uint16_t *x, int64_t M, int64_t K,
+                              uint8_t *q, float *s, uint8_t *s8, int nthreads)
 {
     if (nthreads < 1)
         nthreads = 1;
@@ -305,10 +409,22 @@ void oracle_quant_act(const uint16_t *x, int64_t M, int64_t K, uint8_t *q,
         int64_t m0 = t * per, m1 = (t + 1) * per;
         if (m0 > M) m0 = M;
         if (m1 > M) m1 = M;
-        qa_job j = {x, M, K, q, s, m0, m1};
+        qa_job j = {x, M, K, q, s, s8, m0, m1};
         jobs[t] = j;
         pthread_create(&th[t], NULL, qa_rows, &jobs[t]);
     }
     for (int t = 0; t < nthreads; ++t)
         pthread_join(th[t], NULL);
+}
+
+void oracle_quant_act(const uint16_t *x, int64_t M, int64_t K, uint8_t *q,
+                      float *s, int nthreads)
+{
+    quant_act_threads(x, M, K, q, s, NULL, nthreads);
+}
+
+void oracle_quant_act_ue8m0(const uint16_t *x, int64_t M, int64_t K,
+                            uint8_t *q, uint8_t *s, int nthreads)
+{
+    quant_act_threads(x, M, K, q, NULL, s, nthreads);
 }

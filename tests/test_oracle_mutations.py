@@ -16,6 +16,7 @@ import oracle
 import workloads as wl
 from tests import test_oracle_gemm as tg
 from tests import test_oracle_quant as tq
+from tests import test_oracle_ue8m0 as tu
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
                    "oracle", "fp8bl_oracle.c")
@@ -94,3 +95,32 @@ def test_real_oracle_passes_same_checks():
     tg.test_gemm_vs_exact_rationals(256)
     assert np.all(np.isfinite(oracle.block_linear(*tg._random_case(2, 128, 128, 0))))
     assert wl.tiny()[0].shape == (32, 512)
+
+
+UE8M0_MUTANTS = [
+    # rounds the exponent down at exact powers of two (<= instead of <)
+    ("while (ldexp(448.0, e) < a)", "while (ldexp(448.0, e) <= a)"),
+    # floor instead of ceil: the largest element may exceed 448
+    ("while (ldexp(448.0, e - 1) >= a)\n        --e;\n    while (ldexp(448.0, e) < a)\n        ++e;",
+     "e = (int)floor(log2(a / 448.0));"),
+    # bias 128 instead of 127 when storing
+    ("return (uint8_t)(e + 127);", "return (uint8_t)(e + 128);"),
+    # multiplies by 2^e instead of 2^-e
+    ("double v = (double)x * ldexp(1.0, 127 - (int)c);", "double v = (double)x * ldexp(1.0, (int)c - 127);"),
+    # decode without the bias
+    ("return ldexp(1.0, (int)c - 127);", "return ldexp(1.0, (int)c - 126);"),
+]
+
+
+@pytest.mark.parametrize("old,new", UE8M0_MUTANTS)
+def test_ue8m0_pins_catch(tmp_path, monkeypatch, old, new):
+    lib = _build_mutant(tmp_path, old, new)
+    monkeypatch.setattr(oracle, "_lib", lib)
+    checks = [
+        tu.test_decode_all_codes_vs_torch,
+        lambda: tu.test_scale_code_at_binade_edges(3),
+        tu.test_scale_code_vs_frexp_random,
+        tu.test_act_vs_library_composition,
+        tu.test_weight_vs_library_composition,
+    ]
+    assert any(_fails(c) for c in checks)
