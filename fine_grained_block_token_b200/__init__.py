@@ -4,7 +4,9 @@ Weights quantized to e4m3 with one fp32 scale per 128 x 128 block,
 activations quantized dynamically per token with one fp32 scale per group of
 128 input channels, and a GEMM that applies both scale sets per 128-deep K
 block and writes bf16 ("Fine-grained FP8" page of the transformers docs,
-opening bullet list).
+opening bullet list).  The ``*_ue8m0`` functions are the power-of-two scale
+variant of the page's "UE8M0 scale format" section (float8_e8m0fnu scales),
+whose GEMM runs on the tensor core's block-scaled MMA.
 
 The functions below come from ``_binding`` (a ctypes binding of
 ``libfp8bl.so``), loaded on first use so that the ``build`` submodule can be
@@ -14,7 +16,7 @@ raises ImportError: there is no fallback path.
 __all__ = [
     "Fp8blError", "BLOCK", "STATUS", "lib_path", "quant_act", "quant_weight", "block_linear",
     "block_linear_fused", "block_linear_noalloc", "workspace_bytes", "fused_workspace_bytes",
-    "check", "version",
+    "check", "version", "quant_act_ue8m0", "quant_weight_ue8m0", "block_linear_ue8m0",
 ]
 
 

@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "Fp8blError", "BLOCK", "lib_path", "quant_act", "quant_weight", "block_linear",
     "block_linear_fused", "block_linear_noalloc", "workspace_bytes", "fused_workspace_bytes",
-    "check", "version",
+    "check", "version", "quant_act_ue8m0", "quant_weight_ue8m0", "block_linear_ue8m0",
 ]
 
 BLOCK = 128
@@ -44,12 +44,16 @@ _lib.fp8_block_linear_workspace_bytes.argtypes = [_i64, _i64, _i64]
 _lib.fp8_block_linear_workspace_bytes.restype = _sz
 _lib.fp8_block_linear_fused_workspace_bytes.argtypes = [_i64, _i64, _i64]
 _lib.fp8_block_linear_fused_workspace_bytes.restype = _sz
+_lib.fp8_quant_act_ue8m0.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
+_lib.fp8_quant_weight_ue8m0.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
+_lib.fp8_block_linear_ue8m0.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
 _lib.fp8bl_check.argtypes = [_vp]
 _lib.fp8bl_status_string.argtypes = [ctypes.c_int]
 _lib.fp8bl_status_string.restype = ctypes.c_char_p
 _lib.fp8bl_version.restype = ctypes.c_int
 for _f in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
-           "fp8_block_linear_noalloc", "fp8bl_check"):
+           "fp8_block_linear_noalloc", "fp8bl_check", "fp8_quant_act_ue8m0",
+           "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 STATUS = {0: "FP8BL_OK", 1: "FP8BL_ERR_NULL", 2: "FP8BL_ERR_SHAPE", 3: "FP8BL_ERR_ALIGN",
@@ -105,6 +109,52 @@ def quant_weight(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor
         s = torch.empty((N // BLOCK, K // BLOCK), dtype=torch.float32, device=w.device)
     _ok(_lib.fp8_quant_weight(_ptr(w), N, K, _ptr(q), _ptr(s), _stream(w)), "fp8_quant_weight")
     return q, s
+
+
+# UE8M0 variant ("UE8M0 scale format" section): scales are float8_e8m0fnu
+# codes (one byte, value 2^(code - 127)), the fp32 scale rounded up to a
+# power of two.
+
+
+def quant_act_ue8m0(x: torch.Tensor, q: torch.Tensor | None = None,
+                    s: torch.Tensor | None = None):
+    """bf16 [M, K] -> (e4m3 [M, K], float8_e8m0fnu [M, K/128])."""
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    if s is None:
+        s = torch.empty((M, K // BLOCK if K % BLOCK == 0 else 0), dtype=torch.float8_e8m0fnu,
+                        device=x.device)
+    _ok(_lib.fp8_quant_act_ue8m0(_ptr(x), M, K, _ptr(q), _ptr(s), _stream(x)),
+        "fp8_quant_act_ue8m0")
+    return q, s
+
+
+def quant_weight_ue8m0(w: torch.Tensor, q: torch.Tensor | None = None,
+                       s: torch.Tensor | None = None):
+    """bf16 [N, K] -> (e4m3 [N, K], float8_e8m0fnu [N/128, K/128])."""
+    N, K = w.shape
+    if q is None:
+        q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
+    if s is None:
+        s = torch.empty((N // BLOCK, K // BLOCK), dtype=torch.float8_e8m0fnu, device=w.device)
+    _ok(_lib.fp8_quant_weight_ue8m0(_ptr(w), N, K, _ptr(q), _ptr(s), _stream(w)),
+        "fp8_quant_weight_ue8m0")
+    return q, s
+
+
+def block_linear_ue8m0(q_a, s_a, q_w, s_w, y=None) -> torch.Tensor:
+    """(e4m3 [M,K], e8m0 [M,K/128], e4m3 [N,K], e8m0 [N/128,K/128]) -> bf16 [M,N],
+    on the tensor core's block-scaled MMA."""
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    if q_w.shape[1] != K:
+        raise ValueError("q_a and q_w disagree on K")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
+    _ok(_lib.fp8_block_linear_ue8m0(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
+                                    _stream(q_a)), "fp8_block_linear_ue8m0")
+    return y
 
 
 def workspace_bytes(M: int, N: int, K: int) -> int:

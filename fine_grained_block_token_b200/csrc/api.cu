@@ -82,7 +82,7 @@ const char* fp8bl_status_string(fp8bl_status s) {
     case FP8BL_OK: return "ok";
     case FP8BL_ERR_NULL: return "a required pointer is NULL";
     case FP8BL_ERR_SHAPE: return "invalid sizes (need K, N multiples of 128, within limits)";
-    case FP8BL_ERR_ALIGN: return "pointer not 16-byte aligned (4-byte for scales)";
+    case FP8BL_ERR_ALIGN: return "pointer not 16-byte aligned (4-byte for fp32 scales)";
     case FP8BL_ERR_ARCH: return "current device is not compute capability 10.0 (sm_100)";
     case FP8BL_ERR_CUDA: return "CUDA call failed";
     case FP8BL_ERR_TIMEOUT: return "a kernel wait ran out of time";
@@ -196,6 +196,61 @@ fp8bl_status fp8_block_linear_fused(const void* x_bf16, const void* q_w, const f
   }
   return from_cuda(launch_block_linear_fused(x_bf16, q_w, s_w, y_bf16, M, N, K, plan, workspace,
                                              *d, as_cuda(stream)));
+}
+
+fp8bl_status fp8_quant_act_ue8m0(const void* x_bf16, int64_t M, int64_t K, void* q_e4m3,
+                                 uint8_t* s_ue8m0, fp8bl_stream_t stream) {
+  if (!dim_ok(M, true) || !dim_ok(K, false) || K % FP8BL_BLOCK) return FP8BL_ERR_SHAPE;
+  if (M == 0) return FP8BL_OK;
+  if (!x_bf16 || !q_e4m3 || !s_ue8m0) return FP8BL_ERR_NULL;
+  if (!aligned(x_bf16, 16) || !aligned(q_e4m3, 16)) return FP8BL_ERR_ALIGN;
+  const size_t nx = static_cast<size_t>(M * K) * 2, nq = static_cast<size_t>(M * K),
+               ns = static_cast<size_t>(M * (K / 128));
+  if (overlap(x_bf16, nx, q_e4m3, nq) || overlap(x_bf16, nx, s_ue8m0, ns) ||
+      overlap(q_e4m3, nq, s_ue8m0, ns))
+    return FP8BL_ERR_OVERLAP;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  return from_cuda(
+      launch_act_quant_ue8m0(x_bf16, M, K, q_e4m3, s_ue8m0, d->sm_count, as_cuda(stream)));
+}
+
+fp8bl_status fp8_quant_weight_ue8m0(const void* w_bf16, int64_t N, int64_t K, void* q_e4m3,
+                                    uint8_t* s_ue8m0, fp8bl_stream_t stream) {
+  if (!dim_ok(N, false) || !dim_ok(K, false) || N % FP8BL_BLOCK || K % FP8BL_BLOCK)
+    return FP8BL_ERR_SHAPE;
+  if (!w_bf16 || !q_e4m3 || !s_ue8m0) return FP8BL_ERR_NULL;
+  if (!aligned(w_bf16, 16) || !aligned(q_e4m3, 16)) return FP8BL_ERR_ALIGN;
+  const size_t nw = static_cast<size_t>(N * K) * 2, nq = static_cast<size_t>(N * K),
+               ns = static_cast<size_t>((N / 128) * (K / 128));
+  if (overlap(w_bf16, nw, q_e4m3, nq) || overlap(w_bf16, nw, s_ue8m0, ns) ||
+      overlap(q_e4m3, nq, s_ue8m0, ns))
+    return FP8BL_ERR_OVERLAP;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  return from_cuda(launch_weight_quant_ue8m0(w_bf16, N, K, q_e4m3, s_ue8m0, as_cuda(stream)));
+}
+
+fp8bl_status fp8_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                    const uint8_t* s_w, void* y_bf16, int64_t M, int64_t N,
+                                    int64_t K, fp8bl_stream_t stream) {
+  if (!linear_dims_ok(M, N, K)) return FP8BL_ERR_SHAPE;
+  if (M == 0) return FP8BL_OK;
+  if (!q_a || !s_a || !q_w || !s_w || !y_bf16) return FP8BL_ERR_NULL;
+  if (!aligned(q_a, 16) || !aligned(q_w, 16) || !aligned(y_bf16, 16)) return FP8BL_ERR_ALIGN;
+  const size_t ny = static_cast<size_t>(M * N) * 2;
+  if (overlap(y_bf16, ny, q_a, static_cast<size_t>(M * K)) ||
+      overlap(y_bf16, ny, q_w, static_cast<size_t>(N * K)) ||
+      overlap(y_bf16, ny, s_a, static_cast<size_t>(M * (K / 128))) ||
+      overlap(y_bf16, ny, s_w, static_cast<size_t>((N / 128) * (K / 128))))
+    return FP8BL_ERR_OVERLAP;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  return from_cuda(
+      launch_block_linear_ue8m0(q_a, s_a, q_w, s_w, y_bf16, M, N, K, *d, as_cuda(stream)));
 }
 
 namespace fp8bl {

@@ -30,6 +30,19 @@ cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float
 cudaError_t launch_weight_quant(const void* w, int64_t N, int64_t K, void* q, float* s,
                                 cudaStream_t st);
 
+// UE8M0 variants of both ("UE8M0 scale format"): one byte per scale, the
+// code e + 127 of the power-of-two scale 2^e.
+cudaError_t launch_act_quant_ue8m0(const void* x, int64_t M, int64_t K, void* q, uint8_t* s,
+                                   int sm_count, cudaStream_t st);
+cudaError_t launch_weight_quant_ue8m0(const void* w, int64_t N, int64_t K, void* q, uint8_t* s,
+                                      cudaStream_t st);
+
+// Block-scaled GEMM with UE8M0 scales on the hardware block-scaled MMA
+// (tcgen05.mma kind::mxf8f6f4.block_scale); no workspace.
+cudaError_t launch_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                      const uint8_t* s_w, void* y, int64_t M, int64_t N,
+                                      int64_t K, const DeviceInfo& dev, cudaStream_t st);
+
 // Largest M served by the decode (swap-AB, stream-K) schedule.
 constexpr int64_t kDecodeMaxM = 64;
 

@@ -1,0 +1,365 @@
+// Block-scaled FP8 GEMM with UE8M0 (power-of-two) scales on the hardware
+// block-scaled MMA of sm_100a:
+//   y = bf16( sum_j 2^(ea[m,j]-127) 2^(ew[n/128,j]-127) (A_j W_j^T) )
+//
+// "Fine-grained FP8" page, "UE8M0 scale format" section: checkpoints in the
+// DeepSeek-V4 style keep their FP8 scales as float8_e8m0fnu, and that is
+// the only scale format the Blackwell DeepGEMM expert kernels accept.  The
+// reason is this instruction: tcgen05.mma kind::mxf8f6f4.block_scale
+// multiplies every 32-deep K slice of A and B by a per-row ue8m0 scale
+// factor read from tensor memory, inside the tensor core.  The per-128-K
+// scales of the fine-grained scheme become four equal per-32-K factors, so
+// the accumulator runs across the whole K extent in TMEM and no promotion
+// by CUDA cores is needed (the fp32-scale kernel spends its time there).
+//
+// One CTA per SM (persistent), output tile 128 (M) x 256 (N), tiles visited
+// M-fastest.  12 warps:
+//   warp 0      TMA producer: A 128x128 and W 256x128 e4m3 tiles (128-byte
+//               swizzle) into a 4-deep shared-memory ring.
+//   warp 3      scale-factor builder: for the same stage, writes the 128
+//               activation-row and 256 weight-row scale bytes, each
+//               replicated 4x (one per 32-K slice), in the tensor core's
+//               scale-factor layout (per 128 rows: 512 bytes, row r at byte
+//               16 (r % 32) + 4 (r / 32) + slice), fences them for the async
+//               proxy and arrives on the stage's full barrier.  Its global
+//               loads run four stages ahead of the stores.
+//   warp 1      MMA issuer (whole warp loops and waits, lane 0 issues): per
+//               stage, 3 tcgen05.cp (32 rows x 16 bytes, broadcast to the 4
+//               lane quarters) move the scale factors into TMEM columns
+//               256..259 (A) and 264..271 (B), then 4 block-scaled MMAs
+//               (M=128, N=256, K=32, scale-factor id = slice) accumulate
+//               into columns 0..255; copies and MMAs run in issue order.
+//   warp 2      owns the TMEM allocation (512 columns).
+//   warps 4-11  epilogue: after the tile's last MMA, warp w reads TMEM lanes
+//               32 (w % 4) .. +31 and columns 128 ((w - 4) / 4) .. +127 with
+//               two 64-column loads, releases the accumulator, and converts
+//               and stores the bf16 row segment.
+// A single 256-column accumulator plus the scale-factor columns is what fits
+// in TMEM, so the MMAs of the next tile wait for the epilogue's TMEM reads
+// (not for its stores).
+// Every mbarrier wait is bounded in time; on expiry the kernel records an
+// error code in the error word, drains what it started and exits cleanly.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <mutex>
+
+#include "fp8bl_internal.h"
+#include "ptx_sm100.cuh"
+
+namespace fp8bl {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;
+constexpr int STAGES = 4;
+constexpr int UMMA_K = 32;
+constexpr int A_BYTES = BM * BK;
+constexpr int B_BYTES = BN * BK;
+constexpr int SFA_BYTES = 512;            // 128 rows x 4 slices
+constexpr int SFB_BYTES = 1024;           // 256 rows x 4 slices
+constexpr int TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;
+constexpr uint32_t SFA_COL = 256;
+constexpr uint32_t SFB_COL = 264;
+constexpr int NUM_THREADS = 384;
+constexpr int NUM_EPI_WARPS = 8;
+constexpr uint32_t IDESC = ptx::idesc_mxf8_e4m3_ue8m0(BM, BN);
+constexpr uint32_t kUnitScale = 127;      // ue8m0 code of 1.0, for rows past M or N
+
+constexpr int SMEM_A_OFF = 0;
+constexpr int SMEM_B_OFF = SMEM_A_OFF + STAGES * A_BYTES;
+constexpr int SMEM_SFA_OFF = SMEM_B_OFF + STAGES * B_BYTES;
+constexpr int SMEM_SFB_OFF = SMEM_SFA_OFF + STAGES * SFA_BYTES;
+constexpr int SMEM_BAR_OFF = SMEM_SFB_OFF + STAGES * SFB_BYTES;
+constexpr int NUM_BARS = 2 * STAGES + 3;  // full, empty, tfull, tempty, drain
+constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NUM_BARS * 8;
+constexpr int SMEM_BYTES = SMEM_MISC_OFF + 16 + 1024;  // + slack for 1024-byte alignment
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(STAGES == 4, "the scale-factor builder's prefetch ring has one entry per stage");
+static_assert(SFB_COL + 8 <= TMEM_COLS && SFA_COL + 4 <= SFB_COL, "TMEM columns");
+
+struct GemmArgs {
+  const uint8_t* s_a;   // ue8m0 [M, K/128]
+  const uint8_t* s_w;   // ue8m0 [N/128, K/128]
+  __nv_bfloat16* y;
+  int M, N, K;
+  int* err;
+};
+
+__device__ __forceinline__ void record_error(int* err, int code) { atomicCAS(err, 0, code); }
+
+__device__ __forceinline__ uint32_t rep4(uint32_t b) { return b * 0x01010101u; }
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                  const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t smem_base = ptx::smem_u32(smem);
+  const uint32_t bar_base = smem_base + SMEM_BAR_OFF;
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  const uint32_t tfull_bar = bar_base + 8u * (2 * STAGES);
+  const uint32_t tempty_bar = bar_base + 8u * (2 * STAGES + 1);
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 2);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SMEM_MISC_OFF);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int M = args.M, N = args.N, K = args.K;
+  const int num_m = (M + BM - 1) / BM;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_kb = K / BK;
+  const int num_tiles = num_m * num_n;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full_bar(s), 2);     // TMA producer + scale-factor builder
+      ptx::mbar_init(empty_bar(s), 1);
+    }
+    ptx::mbar_init(tfull_bar, 1);
+    ptx::mbar_init(tempty_bar, NUM_EPI_WARPS);
+    ptx::mbar_init(drain_bar, 1);
+    ptx::fence_barrier_init();
+    ptx::prefetch_tmap(&tmap_a);
+    ptx::prefetch_tmap(&tmap_b);
+  }
+  if (warp == 2) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_holder), TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int last_phase[STAGES];
+      for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
+      uint32_t c = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m_blk = tile % num_m, n_blk = tile / num_m;
+        for (int kb = 0; kb < num_kb; ++kb, ++c) {
+          const int s = c % STAGES;
+          const uint32_t ph = (c / STAGES) & 1u;
+          if (!ptx::mbar_wait(empty_bar(s), ph ^ 1u)) {
+            record_error(args.err, kErrTimeoutProducer);
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
+          ptx::tma_load_2d(smem_base + SMEM_A_OFF + s * A_BYTES, &tmap_a, full_bar(s), kb * BK,
+                           m_blk * BM);
+          ptx::tma_load_2d(smem_base + SMEM_B_OFF + s * B_BYTES, &tmap_b, full_bar(s), kb * BK,
+                           n_blk * BN);
+          last_phase[s] = static_cast<int>(ph);
+        }
+      }
+      // Every load this thread issued lands before the CTA may exit.  The
+      // full barrier also needs the scale-factor builder's arrival, which
+      // precedes any later phase, so waiting on the phase suffices.
+      for (int s = 0; s < STAGES; ++s)
+        if (last_phase[s] >= 0 && !ptx::mbar_wait(full_bar(s), static_cast<uint32_t>(last_phase[s])))
+          record_error(args.err, kErrTimeoutProducer);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------ scale-factor builder
+    // Chunk c of this CTA = (its (c / num_kb)-th tile, K block c % num_kb),
+    // in the producer's order.  Loads for chunk c + STAGES are issued right
+    // after chunk c is stored, so each load has four stages to land.
+    const int my_tiles =
+        static_cast<int>(blockIdx.x) < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const uint32_t total = static_cast<uint32_t>(my_tiles) * static_cast<uint32_t>(num_kb);
+    const int nblk_count = N / 128;
+    auto load = [&](uint32_t c, uint32_t (&a)[4], uint32_t (&b)[2]) {
+      const int tile = static_cast<int>(blockIdx.x + (c / num_kb) * gridDim.x);
+      const int kb = static_cast<int>(c % num_kb);
+      const int m_blk = tile % num_m, n_blk = tile / num_m;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int row = m_blk * BM + lane + 32 * j;
+        a[j] = row < M ? __ldg(args.s_a + static_cast<int64_t>(row) * num_kb + kb) : kUnitScale;
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int nb = n_blk * 2 + h;
+        b[h] = nb < nblk_count ? __ldg(args.s_w + static_cast<int64_t>(nb) * num_kb + kb)
+                               : kUnitScale;
+      }
+    };
+    uint32_t ra[STAGES][4], rb[STAGES][2];
+#pragma unroll
+    for (int i = 0; i < STAGES; ++i)
+      if (static_cast<uint32_t>(i) < total) load(static_cast<uint32_t>(i), ra[i], rb[i]);
+    bool ok = true;
+    for (uint32_t c0 = 0; c0 < total && ok; c0 += STAGES) {
+#pragma unroll
+      for (int i = 0; i < STAGES; ++i) {
+        const uint32_t c = c0 + i;     // c % STAGES == i
+        if (c >= total) break;
+        const uint32_t ph = (c / STAGES) & 1u;
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(empty_bar(i), ph ^ 1u))) {
+          if (lane == 0) record_error(args.err, kErrTimeoutProducer);
+          ok = false;
+          break;
+        }
+        const uint32_t sfa = smem_base + SMEM_SFA_OFF + i * SFA_BYTES + lane * 16;
+        const uint32_t sfb = smem_base + SMEM_SFB_OFF + i * SFB_BYTES + lane * 16;
+        st_shared_v4(sfa, rep4(ra[i][0]), rep4(ra[i][1]), rep4(ra[i][2]), rep4(ra[i][3]));
+        const uint32_t b0 = rep4(rb[i][0]), b1 = rep4(rb[i][1]);
+        st_shared_v4(sfb, b0, b0, b0, b0);
+        st_shared_v4(sfb + 512, b1, b1, b1, b1);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(full_bar(i));
+        if (c + STAGES < total) load(c + STAGES, ra[i], rb[i]);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    uint32_t c = 0, t_local = 0;
+    bool ok = true, issued = false;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t_local) {
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait_spin(tempty_bar, (t_local & 1u) ^ 1u));
+      if (!ok) {
+        if (lane == 0) record_error(args.err, kErrTimeoutMma);
+        break;
+      }
+      for (int kb = 0; kb < num_kb; ++kb, ++c) {
+        const int s = c % STAGES;
+        const uint32_t sph = (c / STAGES) & 1u;
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait_spin(full_bar(s), sph));
+        if (!ok) {
+          if (lane == 0) record_error(args.err, kErrTimeoutMma);
+          break;
+        }
+        ptx::tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a_addr = smem_base + SMEM_A_OFF + s * A_BYTES;
+          const uint32_t b_addr = smem_base + SMEM_B_OFF + s * B_BYTES;
+          const uint32_t sfa_addr = smem_base + SMEM_SFA_OFF + s * SFA_BYTES;
+          const uint32_t sfb_addr = smem_base + SMEM_SFB_OFF + s * SFB_BYTES;
+          ptx::tmem_cp_32x128b_warpx4(tmem_base + SFA_COL, ptx::sdesc_rows16_noswizzle(sfa_addr));
+          ptx::tmem_cp_32x128b_warpx4(tmem_base + SFB_COL, ptx::sdesc_rows16_noswizzle(sfb_addr));
+          ptx::tmem_cp_32x128b_warpx4(tmem_base + SFB_COL + 4,
+                                      ptx::sdesc_rows16_noswizzle(sfb_addr + 512));
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            ptx::mma_mxf8f6f4_block_scale(
+                tmem_base + ACC_COL, ptx::sdesc_kmajor_sw128(a_addr + k * UMMA_K),
+                ptx::sdesc_kmajor_sw128(b_addr + k * UMMA_K), IDESC | ptx::idesc_sf_ids(k, k),
+                tmem_base + SFA_COL, tmem_base + SFB_COL, (kb | k) != 0 ? 1u : 0u);
+          }
+          ptx::mma_commit(empty_bar(s));
+          if (kb == num_kb - 1) ptx::mma_commit(tfull_bar);
+        }
+        __syncwarp();
+        issued = true;
+      }
+    }
+    if (issued && lane == 0) {
+      // All MMAs finish before the TMEM they write is released.
+      ptx::mma_commit(drain_bar);
+      if (!ptx::mbar_wait(drain_bar, 0)) record_error(args.err, kErrTimeoutMma);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int nblk_count = N / 128;
+    uint32_t t_local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t_local) {
+      const int m_blk = tile % num_m, n_blk = tile / num_m;
+      const int row = m_blk * BM + quarter * 32 + lane;
+      const int nb = n_blk * 2 + half;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(tfull_bar, t_local & 1u))) {
+        if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
+        break;
+      }
+      ptx::tc_fence_after();
+      uint32_t v0[64], v1[64];
+      const uint32_t tb = tmem_base + lane_off + ACC_COL + static_cast<uint32_t>(half * 128);
+      ptx::tmem_ld_32x32b_x64(tb, v0);
+      ptx::tmem_ld_32x32b_x64(tb + 64, v1);
+      ptx::tmem_ld_wait();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(tempty_bar);
+      if (row < M && nb < nblk_count) {
+        uint4* dst = reinterpret_cast<uint4*>(args.y + static_cast<int64_t>(row) * N + nb * 128);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint32_t* src = j < 8 ? v0 + 8 * j : v1 + 8 * (j - 8);
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 p = __float22bfloat162_rn(
+                make_float2(__uint_as_float(src[2 * i]), __uint_as_float(src[2 * i + 1])));
+            o[i] = *reinterpret_cast<uint32_t*>(&p);
+          }
+          dst[j] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+cudaError_t ensure_smem_attr() {
+  static cudaError_t st = cudaSuccess;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    st = cudaFuncSetAttribute(gemm_ue8m0_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              SMEM_BYTES);
+  });
+  return st;
+}
+
+}  // namespace
+
+cudaError_t launch_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                      const uint8_t* s_w, void* y, int64_t M, int64_t N,
+                                      int64_t K, const DeviceInfo& dev, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  cudaError_t e = ensure_smem_attr();
+  if (e != cudaSuccess) return e;
+  CUtensorMap ta, tb;
+  if (!make_tmap_u8(&ta, q_a, M, K, BM, BK) || !make_tmap_u8(&tb, q_w, N, K, BN, BK))
+    return cudaErrorInvalidValue;
+  GemmArgs a;
+  a.s_a = s_a;
+  a.s_w = s_w;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.err = dev.error_flag;
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  gemm_ue8m0_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, a);
+  return cudaGetLastError();
+}
+
+}  // namespace fp8bl

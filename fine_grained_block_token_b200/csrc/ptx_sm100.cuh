@@ -193,6 +193,33 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
+// D[tmem] (+)= (A * 2^sfa) (B * 2^sfb)^T with per-32-K block scale factors
+// read from tensor memory: e4m3 x e4m3 -> fp32, scale factors ue8m0, one
+// CTA.  The scale-factor ids (which byte of each 32-bit TMEM word) travel
+// in the instruction descriptor; sfa_tmem / sfb_tmem are plain column
+// addresses.
+__device__ __forceinline__ void mma_mxf8f6f4_block_scale(uint32_t d_tmem, uint64_t a_desc,
+                                                         uint64_t b_desc, uint32_t idesc,
+                                                         uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+      "r"(sfb_tmem)
+      : "memory");
+}
+
+// Shared -> tensor memory copy of 32 rows x 128 bits, broadcast to all four
+// 32-lane quarters: row r of the source lands in lanes r, 32 + r, 64 + r and
+// 96 + r, columns taddr .. taddr + 3.  Ordered with the MMAs this thread
+// issues (same tcgen05 pipeline).
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
+               : "memory");
+}
+
 // Arrive (once) on `bar` when all previously issued MMAs of this thread
 // have completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -320,6 +347,31 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t smem_addr) {
   d |= (uint64_t)1u << 46;
   d |= (uint64_t)2u << 61;
   return d;
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte block stored without
+// swizzle, rows 16 bytes apart (the source of tmem_cp_32x128b_warpx4):
+// start address >> 4 in bits 0-13, leading byte offset 16 >> 4 in 16-29,
+// stride byte offset 128 >> 4 (between 8-row core matrices) in 32-45,
+// version 1 in bits 46-47, swizzle mode 0 (none) in bits 61-63.
+__device__ __forceinline__ uint64_t sdesc_rows16_noswizzle(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(16u >> 4) << 16;
+  d |= (uint64_t)(128u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  return d;
+}
+
+// Instruction descriptor, kind::mxf8f6f4 with block scaling: A = B = e4m3
+// (format 0 in bits 7-9 and 10-12), both K-major, N >> 3 in bits 17-22,
+// scale-factor format 1 (ue8m0) in bit 23, M >> 4 in bits 24-28.  The
+// scale-factor ids go in bits 4-5 (B) and 29-30 (A); K = 32 per MMA.
+__host__ __device__ constexpr uint32_t idesc_mxf8_e4m3_ue8m0(uint32_t M, uint32_t N) {
+  return ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_sf_ids(uint32_t sfa_id, uint32_t sfb_id) {
+  return (sfa_id << 29) | (sfb_id << 4);
 }
 
 // Instruction descriptor, kind::f8f6f4, A = B = e4m3, D = fp32, both

@@ -10,6 +10,12 @@
 // writes 8 bytes of codes per lane (the warp writes 256 contiguous bytes)
 // plus one scale.  Each warp keeps UNROLL pairs of groups in flight so the
 // SM has enough bytes outstanding to run at HBM bandwidth.
+//
+// Every kernel is instantiated twice: kPow2 = false writes fp32 scales
+// (s = amax / 448), kPow2 = true writes UE8M0 codes (the "UE8M0 scale
+// format" section of the same page: the scale rounded up to a power of two,
+// one byte each) and multiplies by the exact power of two instead of
+// dividing.
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -30,9 +36,38 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   return v;
 }
 
+// Per-group constants of either scale format, from the group's amax.
+template <bool kPow2>
+struct GroupQuant;
+
+template <>
+struct GroupQuant<false> {
+  float s;
+  GroupScale g;
+  __device__ __forceinline__ explicit GroupQuant(float amax)
+      : s(scale_from_amax(amax)), g(group_scale(s)) {}
+  __device__ __forceinline__ uint2 quant(uint4 v) const { return quant8(v, g); }
+  __device__ __forceinline__ void store_scale(void* out, int64_t i) const {
+    static_cast<float*>(out)[i] = s;
+  }
+};
+
+template <>
+struct GroupQuant<true> {
+  uint32_t code;
+  float2 inv;
+  __device__ __forceinline__ explicit GroupQuant(float amax)
+      : code(ue8m0_from_amax(amax)), inv(ue8m0_inverse2(code)) {}
+  __device__ __forceinline__ uint2 quant(uint4 v) const { return quant8_pow2(v, inv); }
+  __device__ __forceinline__ void store_scale(void* out, int64_t i) const {
+    static_cast<uint8_t*>(out)[i] = static_cast<uint8_t>(code);
+  }
+};
+
 // num_groups = M * K / 128.  x: 16 uint4 per group; q: 16 uint2 per group.
+template <bool kPow2>
 __global__ void __launch_bounds__(kAqThreads, 4)
-act_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, float* __restrict__ s,
+act_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, void* __restrict__ s,
                  int64_t num_groups) {
   const int lane = threadIdx.x & 31;
   const int half = lane >> 4;
@@ -57,11 +92,11 @@ act_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, float* __re
       m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 4));
       m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 2));
       m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      const float sc = scale_from_amax(absmax_halves_f32(m));
-      const uint2 o = quant8(v[u], group_scale(sc));
+      const GroupQuant<kPow2> gq(absmax_halves_f32(m));
+      const uint2 o = gq.quant(v[u]);
       if (g < num_groups) {
         q[g * 16 + l16] = o;
-        if (l16 == 0) s[g] = sc;
+        if (l16 == 0) gq.store_scale(s, g);
       }
     }
   }
@@ -81,8 +116,9 @@ __device__ __forceinline__ void ld_stream32(const uint4* p, uint4& a, uint4& b) 
                : "l"(p));
 }
 
+template <bool kPow2>
 __global__ void __launch_bounds__(kAqThreads, 4)
-act_quant32_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, float* __restrict__ s,
+act_quant32_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, void* __restrict__ s,
                    int64_t num_groups) {
   const int lane = threadIdx.x & 31;
   const int sub = lane >> 3;      // group within the warp's 4
@@ -110,12 +146,11 @@ act_quant32_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, float* __
       m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 4));
       m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 2));
       m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      const float sc = scale_from_amax(absmax_halves_f32(m));
-      const GroupScale gs = group_scale(sc);
-      const uint2 lo = quant8(va[u], gs), hi = quant8(vb[u], gs);
+      const GroupQuant<kPow2> gq(absmax_halves_f32(m));
+      const uint2 lo = gq.quant(va[u]), hi = gq.quant(vb[u]);
       if (g < num_groups) {
         q[g * 8 + l8] = make_uint4(lo.x, lo.y, hi.x, hi.y);
-        if (l8 == 0) s[g] = sc;
+        if (l8 == 0) gq.store_scale(s, g);
       }
     }
   }
@@ -126,8 +161,9 @@ act_quant32_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, float* __
 // full 256-byte row segments.
 constexpr int kWqThreads = 256;
 
+template <bool kPow2>
 __global__ void __launch_bounds__(kWqThreads)
-weight_quant_kernel(const uint4* __restrict__ w, uint2* __restrict__ q, float* __restrict__ s,
+weight_quant_kernel(const uint4* __restrict__ w, uint2* __restrict__ q, void* __restrict__ s,
                     int64_t K, int64_t KB) {
   __shared__ float warp_amax[kWqThreads / 32];
   const int64_t blk = blockIdx.x;
@@ -150,19 +186,21 @@ weight_quant_kernel(const uint4* __restrict__ w, uint2* __restrict__ q, float* _
   a = warp_amax[0];
 #pragma unroll
   for (int i = 1; i < kWqThreads / 32; ++i) a = fmaxf(a, warp_amax[i]);
-  const float sc = scale_from_amax(a);
-  const GroupScale gs = group_scale(sc);
+  const GroupQuant<kPow2> gq(a);
   const int64_t qrow_stride = K / 8;  // uint2 per row
   const int64_t qbase = (bi * 128 + r0) * qrow_stride + bj * 16 + c;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) q[qbase + static_cast<int64_t>(16 * i) * qrow_stride] = quant8(v[i], gs);
-  if (threadIdx.x == 0) s[bi * KB + bj] = sc;
+  for (int i = 0; i < 8; ++i) q[qbase + static_cast<int64_t>(16 * i) * qrow_stride] = gq.quant(v[i]);
+  if (threadIdx.x == 0) gq.store_scale(s, bi * KB + bj);
 }
 
 }  // namespace
 
-cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float* s,
-                             int sm_count, cudaStream_t st) {
+namespace {
+
+template <bool kPow2>
+cudaError_t act_quant(const void* x, int64_t M, int64_t K, void* q, void* s, int sm_count,
+                      cudaStream_t st) {
   const int64_t groups = M * (K / 128);
   if (groups == 0) return cudaSuccess;
   if ((reinterpret_cast<uintptr_t>(x) & 31) == 0) {
@@ -171,8 +209,8 @@ cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float
     const int64_t blocks_needed = (warps_needed + (kAqThreads / 32) - 1) / (kAqThreads / 32);
     const int64_t max_blocks = static_cast<int64_t>(sm_count) * 4;
     const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
-    act_quant32_kernel<<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
-                                                      static_cast<uint4*>(q), s, groups);
+    act_quant32_kernel<kPow2><<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
+                                                             static_cast<uint4*>(q), s, groups);
     return cudaGetLastError();
   }
   const int64_t pairs = (groups + 1) / 2;
@@ -182,20 +220,42 @@ cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float
   // loop inside the kernel.
   const int64_t max_blocks = static_cast<int64_t>(sm_count) * 4;
   const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
-  act_quant_kernel<<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
-                                                  static_cast<uint2*>(q), s, groups);
+  act_quant_kernel<kPow2><<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
+                                                         static_cast<uint2*>(q), s, groups);
   return cudaGetLastError();
 }
 
-cudaError_t launch_weight_quant(const void* w, int64_t N, int64_t K, void* q, float* s,
-                                cudaStream_t st) {
+template <bool kPow2>
+cudaError_t weight_quant(const void* w, int64_t N, int64_t K, void* q, void* s, cudaStream_t st) {
   const int64_t KB = K / 128;
   const int64_t blocks = (N / 128) * KB;
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
-  weight_quant_kernel<<<static_cast<unsigned>(blocks), kWqThreads, 0, st>>>(
+  weight_quant_kernel<kPow2><<<static_cast<unsigned>(blocks), kWqThreads, 0, st>>>(
       static_cast<const uint4*>(w), static_cast<uint2*>(q), s, K, KB);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float* s,
+                             int sm_count, cudaStream_t st) {
+  return act_quant<false>(x, M, K, q, s, sm_count, st);
+}
+
+cudaError_t launch_act_quant_ue8m0(const void* x, int64_t M, int64_t K, void* q, uint8_t* s,
+                                   int sm_count, cudaStream_t st) {
+  return act_quant<true>(x, M, K, q, s, sm_count, st);
+}
+
+cudaError_t launch_weight_quant(const void* w, int64_t N, int64_t K, void* q, float* s,
+                                cudaStream_t st) {
+  return weight_quant<false>(w, N, K, q, s, st);
+}
+
+cudaError_t launch_weight_quant_ue8m0(const void* w, int64_t N, int64_t K, void* q, uint8_t* s,
+                                      cudaStream_t st) {
+  return weight_quant<true>(w, N, K, q, s, st);
 }
 
 }  // namespace fp8bl

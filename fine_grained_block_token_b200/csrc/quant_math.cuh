@@ -111,4 +111,40 @@ __device__ __forceinline__ uint2 quant8(uint4 v, const GroupScale& g) {
   return make_uint2(quant4(v.x, v.y, g), quant4(v.z, v.w, g));
 }
 
+// ------------------------------------------------------ UE8M0 scales
+// "Fine-grained FP8" page, "UE8M0 scale format" section: scales stored as
+// float8_e8m0fnu.  The scale of a group is the smallest power of two 2^e
+// with max(amax, 1e-10) <= 448 * 2^e, kept as the byte e + 127.  With
+// t = fp32(max(amax, 1e-10) / 448) (the correctly rounded quotient above),
+// e = ceil(log2 t) is t's unbiased exponent plus one when t's mantissa is
+// non-zero: for fp32 amax the rounded quotient never lands on a power of two
+// that the exact quotient lies above (the nearest fp32 values to 448 * 2^k
+// are more than half an ulp of 2^k away after the division), and the test
+// suite replays this for every amax a bf16 input can produce.
+__device__ __forceinline__ uint32_t ue8m0_from_amax(float amax) {
+  const uint32_t t = __float_as_uint(scale_from_amax(amax));   // positive, normal
+  return (t >> 23) + ((t & 0x7FFFFFu) != 0u ? 1u : 0u);
+}
+
+// 2^-e for the code c = e + 127, as fp32 bits (254 - c) << 23; codes stay
+// within 85 .. 247, so the result is a normal number.
+__device__ __forceinline__ float2 ue8m0_inverse2(uint32_t code) {
+  const float r = __uint_as_float((254u - code) << 23);
+  return make_float2(r, r);
+}
+
+// Four bf16 (two words) -> four e4m3 codes of x * 2^-e (an exact product
+// unless it underflows, where the code is a zero of x's sign).
+__device__ __forceinline__ uint32_t quant4_pow2(uint32_t w0, uint32_t w1, float2 inv) {
+  const float2 a = __fmul2_rn(bf16x2_to_f32x2(w0), inv);
+  const float2 b = __fmul2_rn(bf16x2_to_f32x2(w1), inv);
+  const uint32_t codes = cvt_e4m3x2(a.x, a.y) | (cvt_e4m3x2(b.x, b.y) << 16);
+  const uint32_t signs = __byte_perm(w0, w1, 0x7531) & 0x80808080u;
+  return codes | signs;
+}
+
+__device__ __forceinline__ uint2 quant8_pow2(uint4 v, float2 inv) {
+  return make_uint2(quant4_pow2(v.x, v.y, inv), quant4_pow2(v.z, v.w, inv));
+}
+
 }  // namespace fp8bl

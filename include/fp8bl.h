@@ -172,6 +172,44 @@ fp8bl_status fp8_block_linear_noalloc(const void *q_a, const float *s_a,
                                       void *y_bf16, int64_t M, int64_t N, int64_t K,
                                       fp8bl_stream_t stream);
 
+/*
+ * UE8M0 (power-of-two) scale variant.
+ * Passage: "Fine-grained FP8" page, "UE8M0 scale format" section
+ * (DeepSeek-V4-style checkpoints keep FP8 scales as packed float8_e8m0fnu,
+ * scale_fmt="ue8m0"; on Blackwell the DeepGEMM expert kernels accept only
+ * that format).  The page fixes neither the rounding to a power of two nor a
+ * layout; this library implements:
+ *   - the scale of a group or block is the smallest power of two 2^e with
+ *     max(amax, FP8BL_AMAX_EPS) <= 448 * 2^e (the fp32 scale rounded up);
+ *   - it is stored as one byte, the float8_e8m0fnu code e + 127 (value
+ *     2^(code - 127)), in the same row-major grids as the fp32 scales:
+ *     [M, K/128] for activations, [N/128, K/128] for weights;
+ *   - q = e4m3(x * 2^-e): an exact product, then round to nearest even;
+ *   - the linear runs on the tensor core's block-scaled MMA, which applies
+ *     the two scales per 32-deep slice of K and accumulates the whole K
+ *     extent in fp32; y is rounded once to bf16.
+ * Codes stay within 85 .. 247 for finite bf16 inputs.  The scale arrays
+ * have no alignment requirement; the other rules are those of the fp32
+ * calls above.
+ */
+fp8bl_status fp8_quant_act_ue8m0(const void *x_bf16, int64_t M, int64_t K,
+                                 void *q_e4m3, uint8_t *s_ue8m0,
+                                 fp8bl_stream_t stream);
+fp8bl_status fp8_quant_weight_ue8m0(const void *w_bf16, int64_t N, int64_t K,
+                                    void *q_e4m3, uint8_t *s_ue8m0,
+                                    fp8bl_stream_t stream);
+/*
+ *   q_a  in : e4m3 [M, K]              s_a in : ue8m0 codes [M, K/128]
+ *   q_w  in : e4m3 [N, K]              s_w in : ue8m0 codes [N/128, K/128]
+ *   y_bf16 out: bf16 [M, N]
+ *   M >= 0, N, K > 0 and multiples of 128, all <= FP8BL_MAX_DIM.  Scale
+ *   codes must be finite (not 255).  No workspace.
+ */
+fp8bl_status fp8_block_linear_ue8m0(const void *q_a, const uint8_t *s_a,
+                                    const void *q_w, const uint8_t *s_w,
+                                    void *y_bf16, int64_t M, int64_t N, int64_t K,
+                                    fp8bl_stream_t stream);
+
 /* Workspace sizes (bytes) the two linear calls need for these sizes on the
  * current device; 0 when no scratch is needed.  Never fails: invalid sizes
  * return 0 (the linear call then reports the error). */

@@ -31,7 +31,8 @@ def lib():
 def test_header_declares_expected_calls():
     names = _declared()
     for n in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
-              "fp8_block_linear_workspace_bytes", "fp8bl_check", "fp8bl_status_string"):
+              "fp8_block_linear_workspace_bytes", "fp8bl_check", "fp8bl_status_string",
+              "fp8_quant_act_ue8m0", "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0"):
         assert n in names
 
 
@@ -104,6 +105,34 @@ def test_fused_argument_errors(lib):
     assert f(x, w, sw, y, 4, 128, 120, None, 0, None) == 2
     assert f(x, None, sw, y, 4, 128, 128, None, 0, None) == 1
     assert f(x, w, sw, x, 4, 128, 128, None, 0, None) == 8
+
+
+def test_ue8m0_argument_errors(lib):
+    fa = lib.fp8_quant_act_ue8m0
+    fa.argtypes = [V, ctypes.c_int64, ctypes.c_int64, V, V, V]
+    g = _p(0x10000)
+    assert fa(g, 4, 100, _p(0x20000), _p(0x30000), None) == 2     # K % 128
+    assert fa(g, 0, 128, None, None, None) == 0                   # empty M
+    assert fa(g, 4, 128, _p(0x20000), None, None) == 1            # null scales
+    assert fa(_p(0x10008), 4, 128, _p(0x20000), _p(0x30000), None) == 3
+    # byte scales need no alignment: a misaligned scale pointer is accepted
+    # by the checks and reaches the device query (no GPU here: CUDA / ARCH)
+    assert fa(g, 4, 128, _p(0x20000), _p(0x30001), None) in (4, 5)
+    assert fa(g, 4, 128, _p(0x20000), _p(0x10010), None) == 8     # scales overlap x
+    fw = lib.fp8_quant_weight_ue8m0
+    fw.argtypes = [V, ctypes.c_int64, ctypes.c_int64, V, V, V]
+    assert fw(g, 100, 128, _p(0x200000), _p(0x300000), None) == 2
+    assert fw(g, 128, 128, None, _p(0x300000), None) == 1
+    fl = lib.fp8_block_linear_ue8m0
+    fl.argtypes = [V, V, V, V, V, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, V]
+    a, sa, w, sw, y = (_p(0x1000000 * (i + 1)) for i in range(5))
+    assert fl(a, sa, w, sw, y, 4, 100, 128, None) == 2
+    assert fl(a, sa, w, sw, y, 4, 128, 130, None) == 2
+    assert fl(a, sa, w, sw, y, 0, 128, 128, None) == 0
+    assert fl(a, None, w, sw, y, 4, 128, 128, None) == 1
+    assert fl(a, sa, w, sw, _p(0x5000008), 4, 128, 128, None) == 3
+    assert fl(a, sa, w, sw, a, 4, 128, 128, None) == 8
+    assert fl(a, sa, w, sw, sw, 4, 128, 128, None) == 8           # y over the weight scales
 
 
 def test_valid_call_without_gpu_reports_cuda_error(lib):
