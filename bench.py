@@ -19,7 +19,10 @@ for the decode workload the weight-streaming decode kernel, against HBM)
 against the measured peaks in MEASURED_PEAKS.json, from a second pass with
 events around every kernel.  `fused` times fp8_block_linear_fused (the
 activation quantization inside the GEMM) on the same inputs and checks its
-output equals the two-call path bit for bit.  `cpu_baseline` and
+output equals the two-call path bit for bit.  `ue8m0` times the
+power-of-two scale variant (ue8m0 activation quantization + the GEMM on the
+tensor core's block-scaled MMA) on the same inputs, with its GEMM's
+roofline and an oracle check of sampled rows.  `cpu_baseline` and
 `--impl reference` time the plain CPU oracle on a bounded row sample.
 """
 from __future__ import annotations
@@ -76,9 +79,17 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def gemm_source_sha() -> str:
+KERNEL_SOURCES = {
+    "gemm_prefill_kernel": ("gemm.cu", "ptx_sm100.cuh", "quant_math.cuh"),
+    "gemm_ue8m0_kernel": ("gemm_ue8m0.cu", "ptx_sm100.cuh"),
+}
+
+
+def gemm_source_sha(kernel: str = "gemm_prefill_kernel") -> str:
+    """Hash of the sources a kernel is compiled from (its traffic entry in
+    profiles/traffic.txt is valid only while this matches)."""
     h = hashlib.sha256()
-    for f in ("gemm.cu", "ptx_sm100.cuh", "quant_math.cuh"):
+    for f in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(ROOT, "fine_grained_block_token_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -89,7 +100,7 @@ def recorded_traffic(kernel: str, workload: str):
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    sha = gemm_source_sha()
+    sha = gemm_source_sha(kernel)
     for line in open(p):
         if line.startswith("#") or not line.strip():
             continue
@@ -186,6 +197,32 @@ def sample_desc(prepared):
     n = len(prepared[0][1]) if prepared else 0
     return (f"{n} random rows per linear ({', '.join(p[0] for p in prepared)}), all N columns; "
             "activation quant + fp64 GEMM of those rows; weights quantized before timing")
+
+
+def decode_workload(name: str) -> bool:
+    return name == "llama3_decode"
+
+
+def ue8m0_parity(u8_items, lins, rows_per_linear: int, dev):
+    """The UE8M0 leg's output on a few sampled rows against the oracle, which
+    quantizes those rows of the same input bits itself (weights: the GPU's
+    codes, held bit-exact to the oracle by the test suite)."""
+    import torch
+    import oracle
+    worst = 0.0
+    for u, (label, xb, _) in zip(u8_items, lins):
+        M = xb.shape[0]
+        rows = np.unique(np.linspace(0, M - 1, rows_per_linear).astype(np.int64))
+        per_row = [oracle.quant_act_ue8m0_rows(xb, int(r), int(r) + 1) for r in rows]
+        qa = np.concatenate([q for q, _ in per_row])
+        ca = np.concatenate([c for _, c in per_row])
+        qw = u["q_w"].view(torch.uint8).cpu().numpy()
+        cw = u["s_w"].view(torch.uint8).cpu().numpy()
+        R = oracle.block_linear_ue8m0(qa, ca, qw, cw, nthreads=os.cpu_count() or 1)
+        Y = u["y"][torch.as_tensor(rows, device=dev)].float().cpu().numpy()
+        worst = max(worst, within_tolerance(Y, R))
+    return {"rows_per_linear": rows_per_linear, "within_tolerance": worst <= 1.0,
+            "worst_bound_ratio": worst}
 
 
 def within_tolerance(y, R):
@@ -423,12 +460,60 @@ def run_ours(args):
     b.record()
     barrier()
     fused_ms = a.elapsed_time(b)
+
+    # ---- the UE8M0 (power-of-two scale) variant on the same inputs:
+    # activation quantization with ue8m0 scales + the GEMM on the tensor
+    # core's block-scaled MMA, same steps; then a per-kernel event pass
+    u8_items = []
+    ue8m0_ms = ue8m0_gemm_ms = None
+    if not decode_workload(args.workload):
+        for it in items:
+            w = wl.to_torch_bf16(next(wb for lb, _, wb in lins if lb == it["label"])).to(dev)
+            q_w8, s_w8 = fp8.quant_weight_ue8m0(w)
+            del w
+            u8_items.append(dict(it=it, q_w=q_w8, s_w=s_w8,
+                                 q_a=torch.empty_like(it["q_a"]),
+                                 s_a=torch.empty((it["M"], it["K"] // 128), dtype=torch.float8_e8m0fnu,
+                                                 device=dev),
+                                 y=torch.empty_like(it["y"])))
+
+        def ue8m0_step(ev=None):
+            for i, u in enumerate(u8_items):
+                fp8.quant_act_ue8m0(u["it"]["x"], u["q_a"], u["s_a"])
+                if ev is not None:
+                    ev[2 * i].record()
+                fp8.block_linear_ue8m0(u["q_a"], u["s_a"], u["q_w"], u["s_w"], u["y"])
+                if ev is not None:
+                    ev[2 * i + 1].record()
+
+        for _ in range(min(args.warmup, 3)):
+            ue8m0_step()
+        torch.cuda.synchronize()
+        u8_graph = None if args.eager else capture(ue8m0_step)
+        run_u8 = (lambda: u8_graph.replay()) if u8_graph is not None else ue8m0_step
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        barrier()
+        a.record()
+        for _ in range(args.steps):
+            run_u8()
+        b.record()
+        barrier()
+        ue8m0_ms = a.elapsed_time(b)
+        evs8 = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(args.steps)]
+        barrier()
+        for k in range(args.steps):
+            ue8m0_step(evs8[k])
+        barrier()
+        ue8m0_gemm_ms = sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs8 for i in range(n))
+        del u8_graph
     sampler.stop()
     fp8.check()
 
     # max over ranks
-    elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms = max_over_ranks(
-        [elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms], dev, world)
+    elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms, ue8m0_ms, ue8m0_gemm_ms = max_over_ranks(
+        [elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms, ue8m0_ms or 0.0, ue8m0_gemm_ms or 0.0],
+        dev, world)
 
     ms_per_step = elapsed_ms / args.steps
     value = whole_job_rate(world, flops_step, args.steps, elapsed_ms) / 1e12
@@ -463,6 +548,18 @@ def run_ours(args):
                 worst = max(worst, within_tolerance(Y, R))
             parity = {"rows_per_linear": args.cpu_rows, "within_tolerance": worst <= 1.0,
                       "worst_bound_ratio": worst}
+        ue8m0 = None
+        if u8_items:
+            u8_gemm_tf = gemm_flops_step * args.steps / (ue8m0_gemm_ms * 1e-3) / 1e12
+            ue8m0 = {"value": whole_job_rate(world, flops_step, args.steps, ue8m0_ms) / 1e12,
+                     "unit": "TFLOP/s", "ms_per_step": ue8m0_ms / args.steps,
+                     "vs_fp32_scales": ms_per_step / (ue8m0_ms / args.steps),
+                     "gemm": {"kernel": "gemm_ue8m0_kernel", "achieved": u8_gemm_tf, "peak": fp8_peak,
+                              "unit": "TFLOP/s", "frac": u8_gemm_tf / fp8_peak,
+                              "ms_per_launch": ue8m0_gemm_ms / (args.steps * n),
+                              "traffic": recorded_traffic("gemm_ue8m0_kernel", args.workload)}}
+            if world == 1 and not args.no_cpu:
+                ue8m0["parity"] = ue8m0_parity(u8_items, lins, args.ue8m0_rows, dev)
         traffic = recorded_traffic("gemm_prefill_kernel", args.workload)
         gemm_ms_per_launch = gemm_ms / (args.steps * n)
         line = {
@@ -494,6 +591,7 @@ def run_ours(args):
                       "vs_two_call": ms_per_step / (fused_ms / args.steps),
                       "kernel": "decode_kernel after act_quant (staged)" if decode else "gemm_fused_kernel",
                       "identical_to_two_call": fused_identical},
+            "ue8m0": ue8m0,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary(),
             "cpu_baseline": cpu,
@@ -501,6 +599,7 @@ def run_ours(args):
         }
         print(json.dumps(line))
     del graph, fused_graph   # released before the process group goes away
+    u8_items.clear()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -519,6 +618,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-rows", type=int, default=32)
     ap.add_argument("--ref-rows", type=int, default=4)
+    ap.add_argument("--ue8m0-rows", type=int, default=4,
+                    help="rows per linear of the UE8M0 leg checked against the oracle")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch every step's kernels one by one")
     args = ap.parse_args()

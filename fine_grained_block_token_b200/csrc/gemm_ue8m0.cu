@@ -16,26 +16,28 @@
 // M-fastest.  12 warps:
 //   warp 0      TMA producer: A 128x128 and W 256x128 e4m3 tiles (128-byte
 //               swizzle) into a 4-deep shared-memory ring.
-//   warp 3      scale-factor builder: for the same stage, writes the 128
-//               activation-row and 256 weight-row scale bytes, each
-//               replicated 4x (one per 32-K slice), in the tensor core's
-//               scale-factor layout (per 128 rows: 512 bytes, row r at byte
-//               16 (r % 32) + 4 (r / 32) + slice), fences them for the async
-//               proxy and arrives on the stage's full barrier.  Its global
-//               loads run four stages ahead of the stores.
-//   warp 1      MMA issuer (whole warp loops and waits, lane 0 issues): per
-//               stage, 3 tcgen05.cp (32 rows x 16 bytes, broadcast to the 4
-//               lane quarters) move the scale factors into TMEM columns
-//               256..259 (A) and 264..271 (B), then 4 block-scaled MMAs
-//               (M=128, N=256, K=32, scale-factor id = slice) accumulate
-//               into columns 0..255; copies and MMAs run in issue order.
+//   warp 1      MMA issuer (whole warp loops and waits, lane 0 issues): 4
+//               block-scaled MMAs per 128-deep stage (M=128, N=256, K=32,
+//               scale-factor id = 32-K slice) into TMEM columns 0..255,
+//               reading the stage's scale factors from its own 16 TMEM
+//               columns (256 + 16 s ...).
 //   warp 2      owns the TMEM allocation (512 columns).
+//   warps 4-7   scale-factor writers, then epilogue: warp 4 + q writes lane
+//               quarter q of the stage's scale-factor columns with one
+//               tcgen05.st -- the tensor core's layout: per lane l, column j
+//               (0..3) holds activation row 32 j + l's scale replicated 4x
+//               (one byte per 32-K slice), columns 4..7 and 8..11 the two
+//               weight blocks' scales -- and arrives on the stage's full
+//               barrier.  They stay up to 4 stages ahead of the MMAs; at a
+//               tile's end they first fill the next tile's first 4 stages.
+//               (Writing from registers keeps the copies off the tensor
+//               pipe: three tcgen05.cp per stage cost ~180 cycles of it.)
 //   warps 4-11  epilogue: after the tile's last MMA, warp w reads TMEM lanes
 //               32 (w % 4) .. +31 and columns 128 ((w - 4) / 4) .. +127 with
 //               two 64-column loads, releases the accumulator, and converts
 //               and stores the bf16 row segment.
-// A single 256-column accumulator plus the scale-factor columns is what fits
-// in TMEM, so the MMAs of the next tile wait for the epilogue's TMEM reads
+// A single 256-column accumulator is what fits next to the scale-factor
+// columns, so the MMAs of the next tile wait for the epilogue's TMEM reads
 // (not for its stores).
 // Every mbarrier wait is bounded in time; on expiry the kernel records an
 // error code in the error word, drains what it started and exits cleanly.
@@ -58,28 +60,25 @@ constexpr int STAGES = 4;
 constexpr int UMMA_K = 32;
 constexpr int A_BYTES = BM * BK;
 constexpr int B_BYTES = BN * BK;
-constexpr int SFA_BYTES = 512;            // 128 rows x 4 slices
-constexpr int SFB_BYTES = 1024;           // 256 rows x 4 slices
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t SFA_COL = 256;
-constexpr uint32_t SFB_COL = 264;
+constexpr uint32_t SF_COL0 = 256;         // stage s: columns SF_COL0 + 16 s .. + 15
+constexpr uint32_t SFA_COL = 0;           // offsets within a stage's columns
+constexpr uint32_t SFB_COL = 4;
 constexpr int NUM_THREADS = 384;
 constexpr int NUM_EPI_WARPS = 8;
+constexpr int NUM_SF_WARPS = 4;           // warps 4..7, one per TMEM lane quarter
 constexpr uint32_t IDESC = ptx::idesc_mxf8_e4m3_ue8m0(BM, BN);
 constexpr uint32_t kUnitScale = 127;      // ue8m0 code of 1.0, for rows past M or N
 
 constexpr int SMEM_A_OFF = 0;
 constexpr int SMEM_B_OFF = SMEM_A_OFF + STAGES * A_BYTES;
-constexpr int SMEM_SFA_OFF = SMEM_B_OFF + STAGES * B_BYTES;
-constexpr int SMEM_SFB_OFF = SMEM_SFA_OFF + STAGES * SFA_BYTES;
-constexpr int SMEM_BAR_OFF = SMEM_SFB_OFF + STAGES * SFB_BYTES;
+constexpr int SMEM_BAR_OFF = SMEM_B_OFF + STAGES * B_BYTES;
 constexpr int NUM_BARS = 2 * STAGES + 3;  // full, empty, tfull, tempty, drain
 constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NUM_BARS * 8;
 constexpr int SMEM_BYTES = SMEM_MISC_OFF + 16 + 1024;  // + slack for 1024-byte alignment
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(STAGES == 4, "the scale-factor builder's prefetch ring has one entry per stage");
-static_assert(SFB_COL + 8 <= TMEM_COLS && SFA_COL + 4 <= SFB_COL, "TMEM columns");
+static_assert(SF_COL0 >= ACC_COL + BN && SF_COL0 + 16 * STAGES <= TMEM_COLS, "TMEM columns");
 
 struct GemmArgs {
   const uint8_t* s_a;   // ue8m0 [M, K/128]
@@ -93,12 +92,6 @@ __device__ __forceinline__ void record_error(int* err, int code) { atomicCAS(err
 
 __device__ __forceinline__ uint32_t rep4(uint32_t b) { return b * 0x01010101u; }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
@@ -125,7 +118,7 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(full_bar(s), 2);     // TMA producer + scale-factor builder
+      ptx::mbar_init(full_bar(s), 1 + NUM_SF_WARPS);   // TMA producer + scale-factor writers
       ptx::mbar_init(empty_bar(s), 1);
     }
     ptx::mbar_init(tfull_bar, 1);
@@ -170,64 +163,11 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
       }
       // Every load this thread issued lands before the CTA may exit.  The
-      // full barrier also needs the scale-factor builder's arrival, which
-      // precedes any later phase, so waiting on the phase suffices.
+      // full barrier also needs the scale-factor writers' arrivals, which
+      // precede any later phase, so waiting on the phase suffices.
       for (int s = 0; s < STAGES; ++s)
         if (last_phase[s] >= 0 && !ptx::mbar_wait(full_bar(s), static_cast<uint32_t>(last_phase[s])))
           record_error(args.err, kErrTimeoutProducer);
-    }
-  } else if (warp == 3) {
-    // ------------------------------------------------ scale-factor builder
-    // Chunk c of this CTA = (its (c / num_kb)-th tile, K block c % num_kb),
-    // in the producer's order.  Loads for chunk c + STAGES are issued right
-    // after chunk c is stored, so each load has four stages to land.
-    const int my_tiles =
-        static_cast<int>(blockIdx.x) < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const uint32_t total = static_cast<uint32_t>(my_tiles) * static_cast<uint32_t>(num_kb);
-    const int nblk_count = N / 128;
-    auto load = [&](uint32_t c, uint32_t (&a)[4], uint32_t (&b)[2]) {
-      const int tile = static_cast<int>(blockIdx.x + (c / num_kb) * gridDim.x);
-      const int kb = static_cast<int>(c % num_kb);
-      const int m_blk = tile % num_m, n_blk = tile / num_m;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int row = m_blk * BM + lane + 32 * j;
-        a[j] = row < M ? __ldg(args.s_a + static_cast<int64_t>(row) * num_kb + kb) : kUnitScale;
-      }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int nb = n_blk * 2 + h;
-        b[h] = nb < nblk_count ? __ldg(args.s_w + static_cast<int64_t>(nb) * num_kb + kb)
-                               : kUnitScale;
-      }
-    };
-    uint32_t ra[STAGES][4], rb[STAGES][2];
-#pragma unroll
-    for (int i = 0; i < STAGES; ++i)
-      if (static_cast<uint32_t>(i) < total) load(static_cast<uint32_t>(i), ra[i], rb[i]);
-    bool ok = true;
-    for (uint32_t c0 = 0; c0 < total && ok; c0 += STAGES) {
-#pragma unroll
-      for (int i = 0; i < STAGES; ++i) {
-        const uint32_t c = c0 + i;     // c % STAGES == i
-        if (c >= total) break;
-        const uint32_t ph = (c / STAGES) & 1u;
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(empty_bar(i), ph ^ 1u))) {
-          if (lane == 0) record_error(args.err, kErrTimeoutProducer);
-          ok = false;
-          break;
-        }
-        const uint32_t sfa = smem_base + SMEM_SFA_OFF + i * SFA_BYTES + lane * 16;
-        const uint32_t sfb = smem_base + SMEM_SFB_OFF + i * SFB_BYTES + lane * 16;
-        st_shared_v4(sfa, rep4(ra[i][0]), rep4(ra[i][1]), rep4(ra[i][2]), rep4(ra[i][3]));
-        const uint32_t b0 = rep4(rb[i][0]), b1 = rep4(rb[i][1]);
-        st_shared_v4(sfb, b0, b0, b0, b0);
-        st_shared_v4(sfb + 512, b1, b1, b1, b1);
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(full_bar(i));
-        if (c + STAGES < total) load(c + STAGES, ra[i], rb[i]);
-      }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
@@ -251,18 +191,13 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
         if (lane == 0) {
           const uint32_t a_addr = smem_base + SMEM_A_OFF + s * A_BYTES;
           const uint32_t b_addr = smem_base + SMEM_B_OFF + s * B_BYTES;
-          const uint32_t sfa_addr = smem_base + SMEM_SFA_OFF + s * SFA_BYTES;
-          const uint32_t sfb_addr = smem_base + SMEM_SFB_OFF + s * SFB_BYTES;
-          ptx::tmem_cp_32x128b_warpx4(tmem_base + SFA_COL, ptx::sdesc_rows16_noswizzle(sfa_addr));
-          ptx::tmem_cp_32x128b_warpx4(tmem_base + SFB_COL, ptx::sdesc_rows16_noswizzle(sfb_addr));
-          ptx::tmem_cp_32x128b_warpx4(tmem_base + SFB_COL + 4,
-                                      ptx::sdesc_rows16_noswizzle(sfb_addr + 512));
+          const uint32_t sf = tmem_base + SF_COL0 + 16u * static_cast<uint32_t>(s);
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
             ptx::mma_mxf8f6f4_block_scale(
                 tmem_base + ACC_COL, ptx::sdesc_kmajor_sw128(a_addr + k * UMMA_K),
                 ptx::sdesc_kmajor_sw128(b_addr + k * UMMA_K), IDESC | ptx::idesc_sf_ids(k, k),
-                tmem_base + SFA_COL, tmem_base + SFB_COL, (kb | k) != 0 ? 1u : 0u);
+                sf + SFA_COL, sf + SFB_COL, (kb | k) != 0 ? 1u : 0u);
           }
           ptx::mma_commit(empty_bar(s));
           if (kb == num_kb - 1) ptx::mma_commit(tfull_bar);
@@ -278,13 +213,70 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------ scale-factor writers + epilogue
     const int quarter = warp & 3;
     const int half = (warp - 4) >> 2;
+    const bool sf_writer = warp < 4 + NUM_SF_WARPS;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int nblk_count = N / 128;
+    // Chunk c of this CTA = (its (c / num_kb)-th tile, K block c % num_kb),
+    // in the producer's order.
+    const int my_tiles =
+        static_cast<int>(blockIdx.x) < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const uint32_t total = static_cast<uint32_t>(my_tiles) * static_cast<uint32_t>(num_kb);
+    uint32_t c_sf = 0;   // next chunk whose scale factors this warp writes
+    bool ok = true;
+    auto write_sf = [&](uint32_t c) -> bool {
+      const int tile = static_cast<int>(blockIdx.x + (c / num_kb) * gridDim.x);
+      const int kb = static_cast<int>(c % num_kb);
+      const int m_blk = tile % num_m, n_blk = tile / num_m;
+      // loads first: they land while the slot is still in use
+      uint32_t v[16];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int row = m_blk * BM + 32 * j + lane;
+        v[j] = row < M ? __ldg(args.s_a + static_cast<int64_t>(row) * num_kb + kb) : kUnitScale;
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int nb = n_blk * 2 + h;
+        v[4 + 4 * h] = nb < nblk_count ? __ldg(args.s_w + static_cast<int64_t>(nb) * num_kb + kb)
+                                       : kUnitScale;
+      }
+      const int s = c % STAGES;
+      const uint32_t ph = (c / STAGES) & 1u;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(empty_bar(s), ph ^ 1u))) return false;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = rep4(v[j]);
+      const uint32_t b0 = rep4(v[4]), b1 = rep4(v[8]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[4 + j] = b0;
+        v[8 + j] = b1;
+        v[12 + j] = 0u;
+      }
+      ptx::tmem_st_32x32b_x16(tmem_base + lane_off + SF_COL0 + 16u * static_cast<uint32_t>(s), v);
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(full_bar(s));
+      return true;
+    };
     uint32_t t_local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t_local) {
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t_local) {
+      if (sf_writer) {
+        // this tile's stages and the next tile's first STAGES stages (their
+        // slots are freed by this tile's MMAs, not by its epilogue)
+        const uint32_t upto = (t_local + 1) * static_cast<uint32_t>(num_kb) + STAGES;
+        for (; c_sf < total && c_sf < upto; ++c_sf) {
+          if (!write_sf(c_sf)) {
+            if (lane == 0) record_error(args.err, kErrTimeoutProducer);
+            ok = false;
+            break;
+          }
+        }
+        if (!ok) break;
+      }
       const int m_blk = tile % num_m, n_blk = tile / num_m;
       const int row = m_blk * BM + quarter * 32 + lane;
       const int nb = n_blk * 2 + half;
