@@ -14,6 +14,8 @@ Sources (transformers docs, "Fine-grained FP8" page):
   * "DeepGEMM fast path" section -- the dynamic activation scheme;
   * "UE8M0 scale format" section -- power-of-two scales stored as
     float8_e8m0fnu (the ``*_ue8m0`` functions).
+Row-wise FP8 (the ``*_rowwise`` functions): "BFL (fp8r / nvfp4)" page of the
+diffusers docs, first bullet of its list and its "Kernels" table.
 The readings the pages leave open (scale formula, rounding, eps) are stated
 in the header comment of ``fp8bl_oracle.c``.
 """
@@ -80,6 +82,10 @@ def bind(path: str):
     lib.oracle_quant_act_ue8m0.restype = None
     lib.oracle_quant_weight_ue8m0.argtypes = [vp, i64, i64, vp, vp]
     lib.oracle_quant_weight_ue8m0.restype = None
+    lib.oracle_quant_rowwise_rows.argtypes = [vp, i64, vp, vp, i64, i64]
+    lib.oracle_quant_rowwise_rows.restype = None
+    lib.oracle_linear_rowwise_rows.argtypes = [vp, vp, vp, vp, i64, i64, vp, i64, vp]
+    lib.oracle_linear_rowwise_rows.restype = ctypes.c_int
     return lib
 
 
@@ -268,6 +274,47 @@ def block_linear_ue8m0(q_a, c_a, q_w, c_w, rows=None, nthreads: int = 1) -> np.n
     s_a = ue8m0_decode(c_a).astype(np.float32)
     s_w = ue8m0_decode(c_w).astype(np.float32)
     return block_linear(q_a, s_a, q_w, s_w, rows=rows, nthreads=nthreads)
+
+
+# ------------------------------------------------------ row-wise FP8 (fp8r)
+# "BFL (fp8r / nvfp4)" page: one fp32 scale per weight row and per
+# activation row.  Readings R9-R10 in fp8bl_oracle.c.
+
+
+def quant_rowwise(x_bf16, r0: int = 0, r1: int | None = None):
+    """Row-wise e4m3 quantization of rows r0..r1-1 of a bf16 [R, K] matrix.
+
+    Returns (q uint8 [r1 - r0, K], s float32 [r1 - r0])."""
+    x = _as_bf16_bits(x_bf16)
+    R, K = x.shape
+    r1 = R if r1 is None else r1
+    sub = np.ascontiguousarray(x[r0:r1])
+    q = np.empty((r1 - r0, K), dtype=np.uint8)
+    s = np.empty((r1 - r0,), dtype=np.float32)
+    if r1 > r0:
+        _load().oracle_quant_rowwise_rows(_ptr(sub), K, _ptr(q), _ptr(s), 0, r1 - r0)
+    return q, s
+
+
+def linear_rowwise(q_a, s_a, q_w, s_w, rows=None) -> np.ndarray:
+    """fp64 result of the row-wise scaled linear for the given rows.
+
+    q_a uint8 [M, K], s_a float32 [M], q_w uint8 [N, K], s_w float32 [N]."""
+    q_a = np.ascontiguousarray(q_a, dtype=np.uint8)
+    q_w = np.ascontiguousarray(q_w, dtype=np.uint8)
+    s_a = np.ascontiguousarray(s_a, dtype=np.float32)
+    s_w = np.ascontiguousarray(s_w, dtype=np.float32)
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    if q_w.shape[1] != K or s_a.shape != (M,) or s_w.shape != (N,):
+        raise ValueError("shape mismatch")
+    r = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    y = np.empty((len(r), N), dtype=np.float64)
+    if len(r):
+        if _load().oracle_linear_rowwise_rows(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), N, K,
+                                              _ptr(r), len(r), _ptr(y)) != 0:
+            raise MemoryError("oracle allocation failed")
+    return y
 
 
 def bf16_rne(y: np.ndarray) -> np.ndarray:

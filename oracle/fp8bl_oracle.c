@@ -285,6 +285,68 @@ void oracle_quant_weight_ue8m0(const uint16_t *w, int64_t N, int64_t K,
     }
 }
 
+/* ------------------------------------------------- row-wise FP8 (fp8r)
+ *
+ * "BFL (fp8r / nvfp4)" page, first bullet of its list: each quantized
+ * linear keeps an E4M3 weight and one fp32 weight scale per row, and the
+ * activations are quantized to E4M3 per row at run time; its "Kernels"
+ * table runs the product as a scaled matmul with row-wise scales.  The page
+ * gives no scale formula; the readings of R3/R4 carry over with one group
+ * per row:
+ *   R9   s[r] = RN32(max(amax over row r, EPS) / 448), q = encode(RN32(x / s[r]))
+ *        for activation rows (tokens) and weight rows (output channels);
+ *   R10  y[m,n] = s_a[m] * s_w[n] * sum over all k of dec(q_a[m,k]) * dec(q_w[n,k]),
+ *        in fp64 (the sum is exact: integer multiples of 2^-18 below 2^18,
+ *        at most 2^17 terms, < 53 bits).
+ */
+
+/* R9 for rows r0 .. r1-1 of a bf16 [R, K] matrix; s: fp32 [R]. */
+void oracle_quant_rowwise_rows(const uint16_t *x, int64_t K, uint8_t *q,
+                               float *s, int64_t r0, int64_t r1)
+{
+    for (int64_t r = r0; r < r1; ++r) {
+        const uint16_t *xr = x + r * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(bf16_to_f32(xr[k]));
+            if (a > amax)
+                amax = a;
+        }
+        float sc = scale_from_amax(amax);
+        s[r] = sc;
+        for (int64_t k = 0; k < K; ++k)
+            q[r * K + k] = oracle_e4m3_encode(bf16_to_f32(xr[k]) / sc);
+    }
+}
+
+/* R10 for the output rows listed in rows[0 .. nrows-1]; y fp64 [nrows, N]. */
+int oracle_linear_rowwise_rows(const uint8_t *qa, const float *sa,
+                               const uint8_t *qw, const float *sw,
+                               int64_t N, int64_t K,
+                               const int64_t *rows, int64_t nrows, double *y)
+{
+    double dec[256];
+    for (int c = 0; c < 256; ++c)
+        dec[c] = oracle_e4m3_decode((uint8_t)c);
+    double *arow = (double *)malloc((size_t)K * sizeof(double));
+    if (!arow)
+        return -1;
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t m = rows[r];
+        for (int64_t k = 0; k < K; ++k)
+            arow[k] = dec[qa[m * K + k]];
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t *wr = qw + n * K;
+            double b = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                b += arow[k] * dec[wr[k]];
+            y[r * N + n] = (double)sa[m] * (double)sw[n] * b;
+        }
+    }
+    free(arow);
+    return 0;
+}
+
 /* ----------------------------------------------------------------- GEMM */
 
 /* R5 for the output rows listed in rows[0 .. nrows-1] (all N columns).

@@ -16,6 +16,7 @@ import oracle
 import workloads as wl
 from tests import test_oracle_gemm as tg
 from tests import test_oracle_quant as tq
+from tests import test_oracle_rowwise as trw
 from tests import test_oracle_ue8m0 as tu
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
@@ -122,5 +123,31 @@ def test_ue8m0_pins_catch(tmp_path, monkeypatch, old, new):
         tu.test_scale_code_vs_frexp_random,
         tu.test_act_vs_library_composition,
         tu.test_weight_vs_library_composition,
+    ]
+    assert any(_fails(c) for c in checks)
+
+
+ROWWISE_MUTANTS = [
+    # amax over the first 128 elements only (the block rule leaking in)
+    ("        for (int64_t k = 0; k < K; ++k) {\n            float a = fabsf(bf16_to_f32(xr[k]));",
+     "        for (int64_t k = 0; k < (K < 128 ? K : 128); ++k) {\n            float a = fabsf(bf16_to_f32(xr[k]));"),
+    # weight scale of the wrong index (the activation row's)
+    ("y[r * N + n] = (double)sa[m] * (double)sw[n] * b;", "y[r * N + n] = (double)sa[m] * (double)sw[m % N] * b;"),
+    # dropped last k term
+    ("            for (int64_t k = 0; k < K; ++k)\n                b += arow[k] * dec[wr[k]];",
+     "            for (int64_t k = 0; k + 1 < K; ++k)\n                b += arow[k] * dec[wr[k]];"),
+]
+
+
+@pytest.mark.parametrize("old,new", ROWWISE_MUTANTS)
+def test_rowwise_pins_catch(tmp_path, monkeypatch, old, new):
+    lib = _build_mutant(tmp_path, old, new)
+    monkeypatch.setattr(oracle, "_lib", lib)
+    checks = [
+        lambda: trw.test_quant_vs_library_composition(5, 4096, 1),
+        trw.test_row_max_maps_to_448,
+        trw.test_linear_vs_exact_rationals,
+        trw.test_unit_scales_reduce_to_integer_matmul,
+        trw.test_scale_index_per_row_and_column,
     ]
     assert any(_fails(c) for c in checks)
