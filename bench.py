@@ -19,10 +19,11 @@ for the decode workload the weight-streaming decode kernel, against HBM)
 against the measured peaks in MEASURED_PEAKS.json, from a second pass with
 events around every kernel.  `fused` times fp8_block_linear_fused (the
 activation quantization inside the GEMM) on the same inputs and checks its
-output equals the two-call path bit for bit.  `ue8m0` times the
-power-of-two scale variant (ue8m0 activation quantization + the GEMM on the
-tensor core's block-scaled MMA) on the same inputs, with its GEMM's
-roofline and an oracle check of sampled rows.  `cpu_baseline` and
+output equals the two-call path bit for bit.  `ue8m0` and `fp8r` time the
+two other scale formats on the same inputs (power-of-two scales on the
+tensor core's block-scaled MMA; one fp32 scale per activation row and weight
+row), each with its GEMM's roofline and an oracle check of sampled rows.
+`cpu_baseline` and
 `--impl reference` time the plain CPU oracle on a bounded row sample.
 """
 from __future__ import annotations
@@ -82,6 +83,7 @@ def peaks():
 KERNEL_SOURCES = {
     "gemm_prefill_kernel": ("gemm.cu", "ptx_sm100.cuh", "quant_math.cuh"),
     "gemm_ue8m0_kernel": ("gemm_ue8m0.cu", "ptx_sm100.cuh"),
+    "gemm_rowwise_kernel": ("gemm_rowwise.cu", "ptx_sm100.cuh"),
 }
 
 
@@ -203,22 +205,29 @@ def decode_workload(name: str) -> bool:
     return name == "llama3_decode"
 
 
-def ue8m0_parity(u8_items, lins, rows_per_linear: int, dev):
-    """The UE8M0 leg's output on a few sampled rows against the oracle, which
+def variant_parity(name: str, v_items, lins, rows_per_linear: int, dev):
+    """A variant leg's output on a few sampled rows against the oracle, which
     quantizes those rows of the same input bits itself (weights: the GPU's
-    codes, held bit-exact to the oracle by the test suite)."""
+    codes and scales, held bit-exact to the oracle by the test suite)."""
     import torch
     import oracle
     worst = 0.0
-    for u, (label, xb, _) in zip(u8_items, lins):
+    for u, (label, xb, _) in zip(v_items, lins):
         M = xb.shape[0]
         rows = np.unique(np.linspace(0, M - 1, rows_per_linear).astype(np.int64))
-        per_row = [oracle.quant_act_ue8m0_rows(xb, int(r), int(r) + 1) for r in rows]
+        if name == "ue8m0":
+            per_row = [oracle.quant_act_ue8m0_rows(xb, int(r), int(r) + 1) for r in rows]
+        else:
+            per_row = [oracle.quant_rowwise(xb, int(r), int(r) + 1) for r in rows]
         qa = np.concatenate([q for q, _ in per_row])
-        ca = np.concatenate([c for _, c in per_row])
+        sa = np.concatenate([c for _, c in per_row])
         qw = u["q_w"].view(torch.uint8).cpu().numpy()
-        cw = u["s_w"].view(torch.uint8).cpu().numpy()
-        R = oracle.block_linear_ue8m0(qa, ca, qw, cw, nthreads=os.cpu_count() or 1)
+        if name == "ue8m0":
+            sw = u["s_w"].view(torch.uint8).cpu().numpy()
+            R = oracle.block_linear_ue8m0(qa, sa, qw, sw, nthreads=os.cpu_count() or 1)
+        else:
+            sw = u["s_w"].cpu().numpy()
+            R = oracle.linear_rowwise(qa, sa, qw, sw)
         Y = u["y"][torch.as_tensor(rows, device=dev)].float().cpu().numpy()
         worst = max(worst, within_tolerance(Y, R))
     return {"rows_per_linear": rows_per_linear, "within_tolerance": worst <= 1.0,
@@ -461,59 +470,73 @@ def run_ours(args):
     barrier()
     fused_ms = a.elapsed_time(b)
 
-    # ---- the UE8M0 (power-of-two scale) variant on the same inputs:
-    # activation quantization with ue8m0 scales + the GEMM on the tensor
-    # core's block-scaled MMA, same steps; then a per-kernel event pass
-    u8_items = []
-    ue8m0_ms = ue8m0_gemm_ms = None
+    # ---- the scale-format variants on the same inputs, each one step =
+    # its activation quantization + its GEMM per linear, timed like the
+    # headline step (graph replay), then a pass with events around the GEMMs:
+    #   ue8m0  -- power-of-two scales on the tensor core's block-scaled MMA
+    #   fp8r   -- one fp32 scale per activation row and weight row
+    variants = {}
     if not decode_workload(args.workload):
-        for it in items:
-            w = wl.to_torch_bf16(next(wb for lb, _, wb in lins if lb == it["label"])).to(dev)
-            q_w8, s_w8 = fp8.quant_weight_ue8m0(w)
-            del w
-            u8_items.append(dict(it=it, q_w=q_w8, s_w=s_w8,
-                                 q_a=torch.empty_like(it["q_a"]),
-                                 s_a=torch.empty((it["M"], it["K"] // 128), dtype=torch.float8_e8m0fnu,
-                                                 device=dev),
-                                 y=torch.empty_like(it["y"])))
+        wbits = {lb: wb for lb, _, wb in lins}
+        specs = {
+            "ue8m0": dict(wq=fp8.quant_weight_ue8m0, aq=fp8.quant_act_ue8m0,
+                          gemm=fp8.block_linear_ue8m0, kernel="gemm_ue8m0_kernel",
+                          s_a=lambda it: torch.empty((it["M"], it["K"] // 128),
+                                                     dtype=torch.float8_e8m0fnu, device=dev)),
+            "fp8r": dict(wq=fp8.quant_rowwise, aq=fp8.quant_rowwise,
+                         gemm=fp8.linear_rowwise, kernel="gemm_rowwise_kernel",
+                         s_a=lambda it: torch.empty((it["M"],), dtype=torch.float32, device=dev)),
+        }
+        for name, sp in specs.items():
+            v_items = []
+            for it in items:
+                w = wl.to_torch_bf16(wbits[it["label"]]).to(dev)
+                q_wv, s_wv = sp["wq"](w)
+                del w
+                v_items.append(dict(it=it, q_w=q_wv, s_w=s_wv, q_a=torch.empty_like(it["q_a"]),
+                                    s_a=sp["s_a"](it), y=torch.empty_like(it["y"])))
 
-        def ue8m0_step(ev=None):
-            for i, u in enumerate(u8_items):
-                fp8.quant_act_ue8m0(u["it"]["x"], u["q_a"], u["s_a"])
-                if ev is not None:
-                    ev[2 * i].record()
-                fp8.block_linear_ue8m0(u["q_a"], u["s_a"], u["q_w"], u["s_w"], u["y"])
-                if ev is not None:
-                    ev[2 * i + 1].record()
+            def v_step(ev=None, v_items=v_items, sp=sp):
+                for i, u in enumerate(v_items):
+                    sp["aq"](u["it"]["x"], u["q_a"], u["s_a"])
+                    if ev is not None:
+                        ev[2 * i].record()
+                    sp["gemm"](u["q_a"], u["s_a"], u["q_w"], u["s_w"], u["y"])
+                    if ev is not None:
+                        ev[2 * i + 1].record()
 
-        for _ in range(min(args.warmup, 3)):
-            ue8m0_step()
-        torch.cuda.synchronize()
-        u8_graph = None if args.eager else capture(ue8m0_step)
-        run_u8 = (lambda: u8_graph.replay()) if u8_graph is not None else ue8m0_step
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        barrier()
-        a.record()
-        for _ in range(args.steps):
-            run_u8()
-        b.record()
-        barrier()
-        ue8m0_ms = a.elapsed_time(b)
-        evs8 = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(args.steps)]
-        barrier()
-        for k in range(args.steps):
-            ue8m0_step(evs8[k])
-        barrier()
-        ue8m0_gemm_ms = sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs8 for i in range(n))
-        del u8_graph
+            for _ in range(min(args.warmup, 3)):
+                v_step()
+            torch.cuda.synchronize()
+            v_graph = None if args.eager else capture(v_step)
+            run_v = (lambda: v_graph.replay()) if v_graph is not None else v_step
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            barrier()
+            a.record()
+            for _ in range(args.steps):
+                run_v()
+            b.record()
+            barrier()
+            v_ms = a.elapsed_time(b)
+            evv = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(args.steps)]
+            barrier()
+            for k in range(args.steps):
+                v_step(evv[k])
+            barrier()
+            v_gemm_ms = sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evv for i in range(n))
+            del v_graph
+            variants[name] = dict(items=v_items, ms=v_ms, gemm_ms=v_gemm_ms, kernel=sp["kernel"])
     sampler.stop()
     fp8.check()
 
     # max over ranks
-    elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms, ue8m0_ms, ue8m0_gemm_ms = max_over_ranks(
-        [elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms, ue8m0_ms or 0.0, ue8m0_gemm_ms or 0.0],
-        dev, world)
+    vnames = sorted(variants)
+    maxed = max_over_ranks([elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms] +
+                           [variants[v][k] for v in vnames for k in ("ms", "gemm_ms")], dev, world)
+    elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms = maxed[:5]
+    for i, v in enumerate(vnames):
+        variants[v]["ms"], variants[v]["gemm_ms"] = maxed[5 + 2 * i], maxed[6 + 2 * i]
 
     ms_per_step = elapsed_ms / args.steps
     value = whole_job_rate(world, flops_step, args.steps, elapsed_ms) / 1e12
@@ -548,18 +571,19 @@ def run_ours(args):
                 worst = max(worst, within_tolerance(Y, R))
             parity = {"rows_per_linear": args.cpu_rows, "within_tolerance": worst <= 1.0,
                       "worst_bound_ratio": worst}
-        ue8m0 = None
-        if u8_items:
-            u8_gemm_tf = gemm_flops_step * args.steps / (ue8m0_gemm_ms * 1e-3) / 1e12
-            ue8m0 = {"value": whole_job_rate(world, flops_step, args.steps, ue8m0_ms) / 1e12,
-                     "unit": "TFLOP/s", "ms_per_step": ue8m0_ms / args.steps,
-                     "vs_fp32_scales": ms_per_step / (ue8m0_ms / args.steps),
-                     "gemm": {"kernel": "gemm_ue8m0_kernel", "achieved": u8_gemm_tf, "peak": fp8_peak,
-                              "unit": "TFLOP/s", "frac": u8_gemm_tf / fp8_peak,
-                              "ms_per_launch": ue8m0_gemm_ms / (args.steps * n),
-                              "traffic": recorded_traffic("gemm_ue8m0_kernel", args.workload)}}
+        variant_lines = {}
+        for v in vnames:
+            d = variants[v]
+            tf = gemm_flops_step * args.steps / (d["gemm_ms"] * 1e-3) / 1e12
+            variant_lines[v] = {
+                "value": whole_job_rate(world, flops_step, args.steps, d["ms"]) / 1e12,
+                "unit": "TFLOP/s", "ms_per_step": d["ms"] / args.steps,
+                "vs_fp32_block_scales": ms_per_step / (d["ms"] / args.steps),
+                "gemm": {"kernel": d["kernel"], "achieved": tf, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": tf / fp8_peak, "ms_per_launch": d["gemm_ms"] / (args.steps * n),
+                         "traffic": recorded_traffic(d["kernel"], args.workload)}}
             if world == 1 and not args.no_cpu:
-                ue8m0["parity"] = ue8m0_parity(u8_items, lins, args.ue8m0_rows, dev)
+                variant_lines[v]["parity"] = variant_parity(v, d["items"], lins, args.variant_rows, dev)
         traffic = recorded_traffic("gemm_prefill_kernel", args.workload)
         gemm_ms_per_launch = gemm_ms / (args.steps * n)
         line = {
@@ -591,7 +615,8 @@ def run_ours(args):
                       "vs_two_call": ms_per_step / (fused_ms / args.steps),
                       "kernel": "decode_kernel after act_quant (staged)" if decode else "gemm_fused_kernel",
                       "identical_to_two_call": fused_identical},
-            "ue8m0": ue8m0,
+            "ue8m0": variant_lines.get("ue8m0"),
+            "fp8r": variant_lines.get("fp8r"),
             "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary(),
             "cpu_baseline": cpu,
@@ -599,7 +624,7 @@ def run_ours(args):
         }
         print(json.dumps(line))
     del graph, fused_graph   # released before the process group goes away
-    u8_items.clear()
+    variants.clear()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -618,8 +643,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-rows", type=int, default=32)
     ap.add_argument("--ref-rows", type=int, default=4)
-    ap.add_argument("--ue8m0-rows", type=int, default=4,
-                    help="rows per linear of the UE8M0 leg checked against the oracle")
+    ap.add_argument("--variant-rows", type=int, default=4,
+                    help="rows per linear of the ue8m0 / fp8r legs checked against the oracle")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch every step's kernels one by one")
     args = ap.parse_args()

@@ -23,6 +23,7 @@ __all__ = [
     "Fp8blError", "BLOCK", "lib_path", "quant_act", "quant_weight", "block_linear",
     "block_linear_fused", "block_linear_noalloc", "workspace_bytes", "fused_workspace_bytes",
     "check", "version", "quant_act_ue8m0", "quant_weight_ue8m0", "block_linear_ue8m0",
+    "quant_rowwise", "linear_rowwise",
 ]
 
 BLOCK = 128
@@ -47,13 +48,16 @@ _lib.fp8_block_linear_fused_workspace_bytes.restype = _sz
 _lib.fp8_quant_act_ue8m0.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_quant_weight_ue8m0.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_block_linear_ue8m0.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
+_lib.fp8_quant_rowwise.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
+_lib.fp8_linear_rowwise.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
 _lib.fp8bl_check.argtypes = [_vp]
 _lib.fp8bl_status_string.argtypes = [ctypes.c_int]
 _lib.fp8bl_status_string.restype = ctypes.c_char_p
 _lib.fp8bl_version.restype = ctypes.c_int
 for _f in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
            "fp8_block_linear_noalloc", "fp8bl_check", "fp8_quant_act_ue8m0",
-           "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0"):
+           "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0", "fp8_quant_rowwise",
+           "fp8_linear_rowwise"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 STATUS = {0: "FP8BL_OK", 1: "FP8BL_ERR_NULL", 2: "FP8BL_ERR_SHAPE", 3: "FP8BL_ERR_ALIGN",
@@ -154,6 +158,34 @@ def block_linear_ue8m0(q_a, s_a, q_w, s_w, y=None) -> torch.Tensor:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
     _ok(_lib.fp8_block_linear_ue8m0(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
                                     _stream(q_a)), "fp8_block_linear_ue8m0")
+    return y
+
+
+# Row-wise variant ("BFL (fp8r / nvfp4)" page): one fp32 scale per row of
+# the activations and of the weight.
+
+
+def quant_rowwise(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None):
+    """bf16 [R, K] -> (e4m3 [R, K], fp32 [R]); K % 16 == 0."""
+    R, K = x.shape
+    if q is None:
+        q = torch.empty((R, K), dtype=torch.float8_e4m3fn, device=x.device)
+    if s is None:
+        s = torch.empty((R,), dtype=torch.float32, device=x.device)
+    _ok(_lib.fp8_quant_rowwise(_ptr(x), R, K, _ptr(q), _ptr(s), _stream(x)), "fp8_quant_rowwise")
+    return q, s
+
+
+def linear_rowwise(q_a, s_a, q_w, s_w, y=None) -> torch.Tensor:
+    """(e4m3 [M,K], fp32 [M], e4m3 [N,K], fp32 [N]) -> bf16 [M,N]."""
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    if q_w.shape[1] != K:
+        raise ValueError("q_a and q_w disagree on K")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
+    _ok(_lib.fp8_linear_rowwise(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
+                                _stream(q_a)), "fp8_linear_rowwise")
     return y
 
 

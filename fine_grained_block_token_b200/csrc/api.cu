@@ -253,6 +253,45 @@ fp8bl_status fp8_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const v
       launch_block_linear_ue8m0(q_a, s_a, q_w, s_w, y_bf16, M, N, K, *d, as_cuda(stream)));
 }
 
+fp8bl_status fp8_quant_rowwise(const void* x_bf16, int64_t R, int64_t K, void* q_e4m3, float* s,
+                               fp8bl_stream_t stream) {
+  if (!dim_ok(R, true) || !dim_ok(K, false) || K % 16) return FP8BL_ERR_SHAPE;
+  if (R == 0) return FP8BL_OK;
+  if (!x_bf16 || !q_e4m3 || !s) return FP8BL_ERR_NULL;
+  if (!aligned(x_bf16, 16) || !aligned(q_e4m3, 16) || !aligned(s, 4)) return FP8BL_ERR_ALIGN;
+  const size_t nx = static_cast<size_t>(R * K) * 2, nq = static_cast<size_t>(R * K),
+               ns = static_cast<size_t>(R) * 4;
+  if (overlap(x_bf16, nx, q_e4m3, nq) || overlap(x_bf16, nx, s, ns) || overlap(q_e4m3, nq, s, ns))
+    return FP8BL_ERR_OVERLAP;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  return from_cuda(launch_rowwise_quant(x_bf16, R, K, q_e4m3, s, as_cuda(stream)));
+}
+
+fp8bl_status fp8_linear_rowwise(const void* q_a, const float* s_a, const void* q_w,
+                                const float* s_w, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                                fp8bl_stream_t stream) {
+  if (!dim_ok(M, true) || !dim_ok(N, false) || !dim_ok(K, false) || N % 16 || K % 16)
+    return FP8BL_ERR_SHAPE;
+  if (M == 0) return FP8BL_OK;
+  if (!q_a || !s_a || !q_w || !s_w || !y_bf16) return FP8BL_ERR_NULL;
+  if (!aligned(q_a, 16) || !aligned(q_w, 16) || !aligned(y_bf16, 16) || !aligned(s_a, 4) ||
+      !aligned(s_w, 16))
+    return FP8BL_ERR_ALIGN;
+  const size_t ny = static_cast<size_t>(M * N) * 2;
+  if (overlap(y_bf16, ny, q_a, static_cast<size_t>(M * K)) ||
+      overlap(y_bf16, ny, q_w, static_cast<size_t>(N * K)) ||
+      overlap(y_bf16, ny, s_a, static_cast<size_t>(M) * 4) ||
+      overlap(y_bf16, ny, s_w, static_cast<size_t>(N) * 4))
+    return FP8BL_ERR_OVERLAP;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  return from_cuda(
+      launch_linear_rowwise(q_a, s_a, q_w, s_w, y_bf16, M, N, K, *d, as_cuda(stream)));
+}
+
 namespace fp8bl {
 namespace {
 // One thread waits on a freshly initialised mbarrier (phase 0 never

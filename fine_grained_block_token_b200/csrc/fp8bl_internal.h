@@ -43,6 +43,17 @@ cudaError_t launch_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const
                                       const uint8_t* s_w, void* y, int64_t M, int64_t N,
                                       int64_t K, const DeviceInfo& dev, cudaStream_t st);
 
+// Row-wise e4m3 quantization ("BFL (fp8r / nvfp4)"): bf16 [R, K] -> e4m3
+// [R, K] + one fp32 scale per row; K % 16 == 0.
+cudaError_t launch_rowwise_quant(const void* x, int64_t R, int64_t K, void* q, float* s,
+                                 cudaStream_t st);
+
+// Row-wise scaled linear: y = bf16(s_a[m] s_w[n] sum_k q_a[m,k] q_w[n,k]),
+// K and N multiples of 16; no workspace.
+cudaError_t launch_linear_rowwise(const void* q_a, const float* s_a, const void* q_w,
+                                  const float* s_w, void* y, int64_t M, int64_t N, int64_t K,
+                                  const DeviceInfo& dev, cudaStream_t st);
+
 // Largest M served by the decode (swap-AB, stream-K) schedule.
 constexpr int64_t kDecodeMaxM = 64;
 

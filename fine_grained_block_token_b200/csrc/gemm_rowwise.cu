@@ -1,0 +1,283 @@
+// Row-wise scaled FP8 linear for sm_100a:
+//   y[m,n] = bf16( s_a[m] * s_w[n] * sum_k e4m3(q_a[m,k]) e4m3(q_w[n,k]) )
+//
+// "BFL (fp8r / nvfp4)" page, first bullet of its list and its "Kernels"
+// table: an E4M3 weight with one fp32 scale per output row, activations
+// quantized per token row, multiplied as a scaled matmul with row-wise
+// scales.  With one scale per row and column the scales factor out of the
+// K sum, so the tensor core accumulates the whole K extent in fp32 in TMEM
+// and the epilogue applies s_a[m] * s_w[n] once.
+//
+// One CTA per SM (persistent), output tile 128 (M) x 256 (N), tiles visited
+// M-fastest.  12 warps:
+//   warp 0      TMA producer: A 128x128 and W 256x128 e4m3 tiles (128-byte
+//               swizzle; the tail of K past the matrix reads as zero) into a
+//               4-deep shared-memory ring.
+//   warp 1      MMA issuer (whole warp loops and waits, lane 0 issues): 4
+//               MMAs (M=128, N=256, K=32) per stage into the tile's
+//               accumulator, one of two 256-column TMEM buffers (tile t uses
+//               buffer t % 2, so a tile's epilogue overlaps the next tile's
+//               MMAs).
+//   warp 2      owns the TMEM allocation (512 columns).
+//   warps 4-11  epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 and
+//               columns 128 ((w - 4) / 4) .. +127 with two 64-column loads,
+//               releases the buffer, multiplies by s_a[row] * s_w[col] and
+//               stores bf16.
+// Every mbarrier wait is bounded in time; on expiry the kernel records an
+// error code in the error word, drains what it started and exits cleanly.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <mutex>
+
+#include "fp8bl_internal.h"
+#include "ptx_sm100.cuh"
+
+namespace fp8bl {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;
+constexpr int STAGES = 4;
+constexpr int UMMA_K = 32;
+constexpr int A_BYTES = BM * BK;
+constexpr int B_BYTES = BN * BK;
+constexpr int TMEM_COLS = 512;
+constexpr int NUM_THREADS = 384;
+constexpr int NUM_EPI_WARPS = 8;
+constexpr uint32_t IDESC = ptx::idesc_e4m3_f32(BM, BN);
+
+constexpr int SMEM_A_OFF = 0;
+constexpr int SMEM_B_OFF = SMEM_A_OFF + STAGES * A_BYTES;
+constexpr int SMEM_BAR_OFF = SMEM_B_OFF + STAGES * B_BYTES;
+constexpr int NUM_BARS = 2 * STAGES + 4 + 1;   // full, empty, tfull[2], tempty[2], drain
+constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NUM_BARS * 8;
+constexpr int SMEM_BYTES = SMEM_MISC_OFF + 16 + 1024;  // + slack for 1024-byte alignment
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+struct LinearArgs {
+  const float* s_a;   // [M]
+  const float* s_w;   // [N]
+  __nv_bfloat16* y;
+  int M, N, K;
+  int* err;
+};
+
+__device__ __forceinline__ void record_error(int* err, int code) { atomicCAS(err, 0, code); }
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_rowwise_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                    const __grid_constant__ CUtensorMap tmap_b, const LinearArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t smem_base = ptx::smem_u32(smem);
+  const uint32_t bar_base = smem_base + SMEM_BAR_OFF;
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SMEM_MISC_OFF);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int M = args.M, N = args.N, K = args.K;
+  const int num_m = (M + BM - 1) / BM;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_kb = (K + BK - 1) / BK;
+  const int num_tiles = num_m * num_n;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(tfull_bar(b), 1);
+      ptx::mbar_init(tempty_bar(b), NUM_EPI_WARPS);
+    }
+    ptx::mbar_init(drain_bar, 1);
+    ptx::fence_barrier_init();
+    ptx::prefetch_tmap(&tmap_a);
+    ptx::prefetch_tmap(&tmap_b);
+  }
+  if (warp == 2) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_holder), TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int last_phase[STAGES];
+      for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
+      uint32_t c = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m_blk = tile % num_m, n_blk = tile / num_m;
+        for (int kb = 0; kb < num_kb; ++kb, ++c) {
+          const int s = c % STAGES;
+          const uint32_t ph = (c / STAGES) & 1u;
+          if (!ptx::mbar_wait(empty_bar(s), ph ^ 1u)) {
+            record_error(args.err, kErrTimeoutProducer);
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
+          ptx::tma_load_2d(smem_base + SMEM_A_OFF + s * A_BYTES, &tmap_a, full_bar(s), kb * BK,
+                           m_blk * BM);
+          ptx::tma_load_2d(smem_base + SMEM_B_OFF + s * B_BYTES, &tmap_b, full_bar(s), kb * BK,
+                           n_blk * BN);
+          last_phase[s] = static_cast<int>(ph);
+        }
+      }
+      // Every load this thread issued lands before the CTA may exit.
+      for (int s = 0; s < STAGES; ++s)
+        if (last_phase[s] >= 0 && !ptx::mbar_wait(full_bar(s), static_cast<uint32_t>(last_phase[s])))
+          record_error(args.err, kErrTimeoutProducer);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    uint32_t c = 0, t_local = 0;
+    bool ok = true, issued = false;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t_local) {
+      const int buf = t_local & 1;
+      const uint32_t bph = (t_local >> 1) & 1u;
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait_spin(tempty_bar(buf), bph ^ 1u));
+      if (!ok) {
+        if (lane == 0) record_error(args.err, kErrTimeoutMma);
+        break;
+      }
+      const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+      for (int kb = 0; kb < num_kb; ++kb, ++c) {
+        const int s = c % STAGES;
+        const uint32_t sph = (c / STAGES) & 1u;
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait_spin(full_bar(s), sph));
+        if (!ok) {
+          if (lane == 0) record_error(args.err, kErrTimeoutMma);
+          break;
+        }
+        ptx::tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a_addr = smem_base + SMEM_A_OFF + s * A_BYTES;
+          const uint32_t b_addr = smem_base + SMEM_B_OFF + s * B_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k)
+            ptx::mma_f8f6f4(d, ptx::sdesc_kmajor_sw128(a_addr + k * UMMA_K),
+                            ptx::sdesc_kmajor_sw128(b_addr + k * UMMA_K), IDESC,
+                            (kb | k) != 0 ? 1u : 0u);
+          ptx::mma_commit(empty_bar(s));
+          if (kb == num_kb - 1) ptx::mma_commit(tfull_bar(buf));
+        }
+        __syncwarp();
+        issued = true;
+      }
+    }
+    if (issued && lane == 0) {
+      // All MMAs finish before the TMEM they write is released.
+      ptx::mma_commit(drain_bar);
+      if (!ptx::mbar_wait(drain_bar, 0)) record_error(args.err, kErrTimeoutMma);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    uint32_t t_local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t_local) {
+      const int m_blk = tile % num_m, n_blk = tile / num_m;
+      const int row = m_blk * BM + quarter * 32 + lane;
+      const int col0 = n_blk * BN + half * 128;
+      const int buf = t_local & 1;
+      const uint32_t bph = (t_local >> 1) & 1u;
+      const float sa = row < M ? __ldg(args.s_a + row) : 0.0f;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(tfull_bar(buf), bph))) {
+        if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
+        break;
+      }
+      ptx::tc_fence_after();
+      uint32_t v0[64], v1[64];
+      const uint32_t tb = tmem_base + lane_off + static_cast<uint32_t>(buf * BN + half * 128);
+      ptx::tmem_ld_32x32b_x64(tb, v0);
+      ptx::tmem_ld_32x32b_x64(tb + 64, v1);
+      ptx::tmem_ld_wait();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
+      if (row < M) {
+        __nv_bfloat16* yrow = args.y + static_cast<int64_t>(row) * N;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int col = col0 + 8 * j;
+          if (col < N) {     // N % 16 == 0: an 8-column chunk is all in or all out
+            const uint32_t* src = j < 8 ? v0 + 8 * j : v1 + 8 * (j - 8);
+            const float4 w0 = __ldg(reinterpret_cast<const float4*>(args.s_w + col));
+            const float4 w1 = __ldg(reinterpret_cast<const float4*>(args.s_w + col + 4));
+            const float sw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float lo = __uint_as_float(src[2 * i]) * (sa * sw[2 * i]);
+              const float hi = __uint_as_float(src[2 * i + 1]) * (sa * sw[2 * i + 1]);
+              __nv_bfloat162 p = __float22bfloat162_rn(make_float2(lo, hi));
+              o[i] = *reinterpret_cast<uint32_t*>(&p);
+            }
+            *reinterpret_cast<uint4*>(yrow + col) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+cudaError_t ensure_smem_attr() {
+  static cudaError_t st = cudaSuccess;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    st = cudaFuncSetAttribute(gemm_rowwise_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              SMEM_BYTES);
+  });
+  return st;
+}
+
+}  // namespace
+
+cudaError_t launch_linear_rowwise(const void* q_a, const float* s_a, const void* q_w,
+                                  const float* s_w, void* y, int64_t M, int64_t N, int64_t K,
+                                  const DeviceInfo& dev, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  cudaError_t e = ensure_smem_attr();
+  if (e != cudaSuccess) return e;
+  CUtensorMap ta, tb;
+  if (!make_tmap_u8(&ta, q_a, M, K, BM, BK) || !make_tmap_u8(&tb, q_w, N, K, BN, BK))
+    return cudaErrorInvalidValue;
+  LinearArgs a;
+  a.s_a = s_a;
+  a.s_w = s_w;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.err = dev.error_flag;
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  gemm_rowwise_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, a);
+  return cudaGetLastError();
+}
+
+}  // namespace fp8bl

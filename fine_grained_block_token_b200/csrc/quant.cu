@@ -236,7 +236,60 @@ cudaError_t weight_quant(const void* w, int64_t N, int64_t K, void* q, void* s, 
   return cudaGetLastError();
 }
 
+// Row-wise quantization ("BFL (fp8r / nvfp4)" page: one scale per row of
+// the weight, and per token row of the activations).  One CTA per row: the
+// row's 16-byte vectors are strided over the threads, the first kRowCache
+// per thread stay in registers between the abs-max pass and the quantizing
+// pass (rows up to 8192 elements are read once), the rest are read again
+// (from L2).  The scale and the division are those of the 1 x 128 groups.
+constexpr int kRowThreads = 256;
+constexpr int kRowCache = 4;
+
+__global__ void __launch_bounds__(kRowThreads)
+rowwise_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, float* __restrict__ s,
+                     int64_t nvec) {
+  __shared__ uint32_t warp_amax[kRowThreads / 32];
+  const int64_t row = blockIdx.x;
+  const uint4* xr = x + row * nvec;
+  uint2* qr = q + row * nvec;
+  uint4 cache[kRowCache];
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < kRowCache; ++i) {
+    const int64_t v = threadIdx.x + static_cast<int64_t>(i) * kRowThreads;
+    cache[i] = v < nvec ? ld_stream(xr + v) : make_uint4(0u, 0u, 0u, 0u);
+    m = absmax_bf16x2(m, absmax8_bf16x2(cache[i]));
+  }
+  for (int64_t v = threadIdx.x + kRowCache * kRowThreads; v < nvec; v += kRowThreads)
+    m = absmax_bf16x2(m, absmax8_bf16x2(__ldg(xr + v)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) warp_amax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = warp_amax[0];
+#pragma unroll
+  for (int i = 1; i < kRowThreads / 32; ++i) m = absmax_bf16x2(m, warp_amax[i]);
+  const GroupQuant<false> gq(absmax_halves_f32(m));
+#pragma unroll
+  for (int i = 0; i < kRowCache; ++i) {
+    const int64_t v = threadIdx.x + static_cast<int64_t>(i) * kRowThreads;
+    if (v < nvec) qr[v] = gq.quant(cache[i]);
+  }
+  for (int64_t v = threadIdx.x + kRowCache * kRowThreads; v < nvec; v += kRowThreads)
+    qr[v] = gq.quant(__ldg(xr + v));
+  if (threadIdx.x == 0) gq.store_scale(s, row);
+}
+
 }  // namespace
+
+cudaError_t launch_rowwise_quant(const void* x, int64_t R, int64_t K, void* q, float* s,
+                                 cudaStream_t st) {
+  if (R == 0) return cudaSuccess;
+  if (R > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
+  rowwise_quant_kernel<<<static_cast<unsigned>(R), kRowThreads, 0, st>>>(
+      static_cast<const uint4*>(x), static_cast<uint2*>(q), s, K / 8);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float* s,
                              int sm_count, cudaStream_t st) {

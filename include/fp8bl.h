@@ -210,6 +210,37 @@ fp8bl_status fp8_block_linear_ue8m0(const void *q_a, const uint8_t *s_a,
                                     void *y_bf16, int64_t M, int64_t N, int64_t K,
                                     fp8bl_stream_t stream);
 
+/*
+ * Row-wise FP8 variant (fp8r).
+ * Passage: "BFL (fp8r / nvfp4)" page of the diffusers docs, first bullet of
+ * its list (an E4M3 weight with one fp32 weight scale per row; activations
+ * quantized to E4M3 per row at run time) and its "Kernels" table (a scaled
+ * matmul with row-wise scales).  The page gives no formula; this library
+ * uses the rule of the calls above with one group per row:
+ *   s[r] = fp32(max(amax over row r, FP8BL_AMAX_EPS) / 448),
+ *   q = e4m3(fp32(x / s[r])),
+ *   y[m,n] = bf16(s_a[m] * s_w[n] * sum_k e4m3val(q_a[m,k]) * e4m3val(q_w[n,k])),
+ * the sum accumulated in fp32 on the tensor core, the scales applied once.
+ *
+ * fp8_quant_rowwise -- bf16 [R, K] -> e4m3 [R, K] + fp32 s [R]; serves both
+ *   the activations (R = M tokens) and the weights (R = N output channels).
+ *   R >= 0 (0 enqueues nothing), K > 0, K % 16 == 0, both <= FP8BL_MAX_DIM.
+ */
+fp8bl_status fp8_quant_rowwise(const void *x_bf16, int64_t R, int64_t K,
+                               void *q_e4m3, float *s, fp8bl_stream_t stream);
+/*
+ * fp8_linear_rowwise --
+ *   q_a in: e4m3 [M, K]   s_a in: fp32 [M]
+ *   q_w in: e4m3 [N, K]   s_w in: fp32 [N] (16-byte aligned)
+ *   y_bf16 out: bf16 [M, N]
+ *   M >= 0, N > 0, K > 0, N % 16 == 0, K % 16 == 0, all <= FP8BL_MAX_DIM.
+ *   No workspace.
+ */
+fp8bl_status fp8_linear_rowwise(const void *q_a, const float *s_a,
+                                const void *q_w, const float *s_w,
+                                void *y_bf16, int64_t M, int64_t N, int64_t K,
+                                fp8bl_stream_t stream);
+
 /* Workspace sizes (bytes) the two linear calls need for these sizes on the
  * current device; 0 when no scratch is needed.  Never fails: invalid sizes
  * return 0 (the linear call then reports the error). */

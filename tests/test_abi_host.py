@@ -32,7 +32,8 @@ def test_header_declares_expected_calls():
     names = _declared()
     for n in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
               "fp8_block_linear_workspace_bytes", "fp8bl_check", "fp8bl_status_string",
-              "fp8_quant_act_ue8m0", "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0"):
+              "fp8_quant_act_ue8m0", "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0",
+              "fp8_quant_rowwise", "fp8_linear_rowwise"):
         assert n in names
 
 
@@ -133,6 +134,26 @@ def test_ue8m0_argument_errors(lib):
     assert fl(a, sa, w, sw, _p(0x5000008), 4, 128, 128, None) == 3
     assert fl(a, sa, w, sw, a, 4, 128, 128, None) == 8
     assert fl(a, sa, w, sw, sw, 4, 128, 128, None) == 8           # y over the weight scales
+
+
+def test_rowwise_argument_errors(lib):
+    fq = lib.fp8_quant_rowwise
+    fq.argtypes = [V, ctypes.c_int64, ctypes.c_int64, V, V, V]
+    g = _p(0x10000)
+    assert fq(g, 4, 100, _p(0x20000), _p(0x30000), None) == 2      # K % 16
+    assert fq(g, 0, 16, None, None, None) == 0                     # empty
+    assert fq(g, 4, 16, None, _p(0x30000), None) == 1
+    assert fq(g, 4, 16, _p(0x20000), _p(0x30002), None) == 3       # scales need 4 bytes
+    assert fq(g, 4, 16, _p(0x10040), _p(0x30000), None) == 8       # q overlaps x
+    fl = lib.fp8_linear_rowwise
+    fl.argtypes = [V, V, V, V, V, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, V]
+    a, sa, w, sw, y = (_p(0x1000000 * (i + 1)) for i in range(5))
+    assert fl(a, sa, w, sw, y, 4, 24, 32, None) == 2               # N % 16
+    assert fl(a, sa, w, sw, y, 4, 32, 24, None) == 2               # K % 16
+    assert fl(a, sa, w, sw, y, 0, 32, 32, None) == 0
+    assert fl(a, sa, None, sw, y, 4, 32, 32, None) == 1
+    assert fl(a, sa, w, _p(0x4000004), y, 4, 32, 32, None) == 3    # s_w must be 16-byte aligned
+    assert fl(a, sa, w, sw, w, 4, 32, 32, None) == 8
 
 
 def test_valid_call_without_gpu_reports_cuda_error(lib):
