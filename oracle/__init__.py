@@ -209,7 +209,7 @@ def block_linear(q_a, s_a, q_w, s_w, rows=None, nthreads: int = 1) -> np.ndarray
 
 # ------------------------------------------------------------ UE8M0 scales
 # "Fine-grained FP8" page, "UE8M0 scale format" section: scales kept as
-# float8_e8m0fnu (scale_fmt="ue8m0").  Readings R6-R8 in fp8bl_oracle.c:
+# float8_e8m0fnu (scale_fmt="ue8m0").  Readings R11-R13 in fp8bl_oracle.c:
 # the scale is the fp32 scale rounded up to a power of two 2^e, stored as
 # the byte e + 127, and q = e4m3(x * 2^-e).
 
@@ -278,7 +278,7 @@ def block_linear_ue8m0(q_a, c_a, q_w, c_w, rows=None, nthreads: int = 1) -> np.n
 
 # ------------------------------------------------------ row-wise FP8 (fp8r)
 # "BFL (fp8r / nvfp4)" page: one fp32 scale per weight row and per
-# activation row.  Readings R9-R10 in fp8bl_oracle.c.
+# activation row.  Readings R14-R15 in fp8bl_oracle.c.
 
 
 def quant_rowwise(x_bf16, r0: int = 0, r1: int | None = None):

@@ -192,20 +192,20 @@ void oracle_quant_weight(const uint16_t *w, int64_t N, int64_t K,
  * instead of float32 (scale_fmt="ue8m0"), and on Blackwell the DeepGEMM
  * expert kernels accept only these.  The section gives neither how a scale
  * becomes a power of two nor a layout.  Readings used here:
- *   R6  a ue8m0 code c is an unsigned biased exponent: value 2^(c - 127),
+ *   R11  a ue8m0 code c is an unsigned biased exponent: value 2^(c - 127),
  *       c = 255 is NaN (the float8_e8m0fnu format); no sign, no zero.
- *   R7  the scale of a group or block is the smallest power of two
+ *   R12  the scale of a group or block is the smallest power of two
  *       s = 2^e with max(amax, EPS) <= 448 * s, i.e. the fp32 scale of R3
  *       rounded UP to a power of two, so the largest element still maps
  *       inside +-448 and nothing saturates; stored as c = e + 127, one byte
  *       per scale, in the same [M, K/128] and [N/128, K/128] grids.
- *   R8  q = encode(RN32(x * 2^-e)): the product is exact in fp64 and is
+ *   R13  q = encode(RN32(x * 2^-e)): the product is exact in fp64 and is
  *       rounded once to fp32 (the only rounding besides the e4m3 one; it
  *       matters only when x * 2^-e underflows fp32, where e4m3 gives 0).
  *   The GEMM is R5 with s = 2^(c - 127).
  */
 
-/* R6 */
+/* R11 */
 double oracle_ue8m0_decode(uint8_t c)
 {
     if (c == 255)
@@ -213,7 +213,7 @@ double oracle_ue8m0_decode(uint8_t c)
     return ldexp(1.0, (int)c - 127);
 }
 
-/* R7: the least e with a <= 448 * 2^e, found by exact comparisons
+/* R12: the least e with a <= 448 * 2^e, found by exact comparisons
  * (448 * 2^e is exact in fp64, and so is the fp32 amax). */
 uint8_t oracle_ue8m0_from_amax(float amax)
 {
@@ -227,7 +227,7 @@ uint8_t oracle_ue8m0_from_amax(float amax)
     return (uint8_t)(e + 127);
 }
 
-/* R8 for one value, given the group's code c. */
+/* R13 for one value, given the group's code c. */
 static uint8_t encode_pow2(float x, uint8_t c)
 {
     double v = (double)x * ldexp(1.0, 127 - (int)c);   /* exact */
@@ -293,14 +293,14 @@ void oracle_quant_weight_ue8m0(const uint16_t *w, int64_t N, int64_t K,
  * table runs the product as a scaled matmul with row-wise scales.  The page
  * gives no scale formula; the readings of R3/R4 carry over with one group
  * per row:
- *   R9   s[r] = RN32(max(amax over row r, EPS) / 448), q = encode(RN32(x / s[r]))
+ *   R14  s[r] = RN32(max(amax over row r, EPS) / 448), q = encode(RN32(x / s[r]))
  *        for activation rows (tokens) and weight rows (output channels);
- *   R10  y[m,n] = s_a[m] * s_w[n] * sum over all k of dec(q_a[m,k]) * dec(q_w[n,k]),
+ *   R15  y[m,n] = s_a[m] * s_w[n] * sum over all k of dec(q_a[m,k]) * dec(q_w[n,k]),
  *        in fp64 (the sum is exact: integer multiples of 2^-18 below 2^18,
  *        at most 2^17 terms, < 53 bits).
  */
 
-/* R9 for rows r0 .. r1-1 of a bf16 [R, K] matrix; s: fp32 [R]. */
+/* R14 for rows r0 .. r1-1 of a bf16 [R, K] matrix; s: fp32 [R]. */
 void oracle_quant_rowwise_rows(const uint16_t *x, int64_t K, uint8_t *q,
                                float *s, int64_t r0, int64_t r1)
 {
@@ -319,7 +319,7 @@ void oracle_quant_rowwise_rows(const uint16_t *x, int64_t K, uint8_t *q,
     }
 }
 
-/* R10 for the output rows listed in rows[0 .. nrows-1]; y fp64 [nrows, N]. */
+/* R15 for the output rows listed in rows[0 .. nrows-1]; y fp64 [nrows, N]. */
 int oracle_linear_rowwise_rows(const uint8_t *qa, const float *sa,
                                const uint8_t *qw, const float *sw,
                                int64_t N, int64_t K,
