@@ -14,7 +14,8 @@ Sources (transformers docs, "Fine-grained FP8" page):
   * "DeepGEMM fast path" section -- the dynamic activation scheme;
   * "UE8M0 scale format" section -- power-of-two scales stored as
     float8_e8m0fnu (the ``*_ue8m0`` functions).
-Row-wise FP8 (the ``*_rowwise`` functions): "BFL (fp8r / nvfp4)" page of the
+Static activation scale (``quant_act_static``): the "DeepGEMM fast path" section's
+static activation quantization.  Row-wise FP8 (the ``*_rowwise`` functions): "BFL (fp8r / nvfp4)" page of the
 diffusers docs, first bullet of its list and its "Kernels" table.
 The readings the pages leave open (scale formula, rounding, eps) are stated
 in the header comment of ``fp8bl_oracle.c``.
@@ -86,6 +87,8 @@ def bind(path: str):
     lib.oracle_quant_rowwise_rows.restype = None
     lib.oracle_linear_rowwise_rows.argtypes = [vp, vp, vp, vp, i64, i64, vp, i64, vp]
     lib.oracle_linear_rowwise_rows.restype = ctypes.c_int
+    lib.oracle_quant_act_static.argtypes = [vp, i64, i64, ctypes.c_float, vp, vp]
+    lib.oracle_quant_act_static.restype = None
     return lib
 
 
@@ -315,6 +318,20 @@ def linear_rowwise(q_a, s_a, q_w, s_w, rows=None) -> np.ndarray:
                                               _ptr(r), len(r), _ptr(y)) != 0:
             raise MemoryError("oracle allocation failed")
     return y
+
+
+def quant_act_static(x_bf16, s: float):
+    """Static activation quantization with one given fp32 scale (reading R16 in
+    fp8bl_oracle.c).  Returns (q uint8 [M, K], s_a float32 [M, K/128] all = s)."""
+    x = _as_bf16_bits(x_bf16)
+    M, K = x.shape
+    if K % BLOCK:
+        raise ValueError("K must be a multiple of 128")
+    q = np.empty((M, K), dtype=np.uint8)
+    sa = np.empty((M, K // BLOCK), dtype=np.float32)
+    if M:
+        _load().oracle_quant_act_static(_ptr(x), M, K, float(np.float32(s)), _ptr(q), _ptr(sa))
+    return q, sa
 
 
 def bf16_rne(y: np.ndarray) -> np.ndarray:

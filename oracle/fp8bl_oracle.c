@@ -347,6 +347,25 @@ int oracle_linear_rowwise_rows(const uint8_t *qa, const float *sa,
     return 0;
 }
 
+/* ------------------------------------------- static activation scale
+ *
+ * "Fine-grained FP8" page, "DeepGEMM fast path" section: next to the
+ * dynamic scheme there is static activation quantization (it always runs on
+ * the Triton path); the page says nothing more about it.  Reading:
+ *   R16  a static scheme has one given fp32 activation scale s per linear
+ *        (calibrated elsewhere): q = encode(RN32(x / s)), saturating by R2
+ *        for |x| > 448 s, and the linear is R5 with every s_a[m,j] = s.
+ */
+void oracle_quant_act_static(const uint16_t *x, int64_t M, int64_t K, float s,
+                             uint8_t *q, float *sa)
+{
+    int64_t G = K / OR_BLOCK;
+    for (int64_t i = 0; i < M * K; ++i)
+        q[i] = oracle_e4m3_encode(bf16_to_f32(x[i]) / s);
+    for (int64_t i = 0; i < M * G; ++i)
+        sa[i] = s;
+}
+
 /* ----------------------------------------------------------------- GEMM */
 
 /* R5 for the output rows listed in rows[0 .. nrows-1] (all N columns).

@@ -17,6 +17,7 @@ import workloads as wl
 from tests import test_oracle_gemm as tg
 from tests import test_oracle_quant as tq
 from tests import test_oracle_rowwise as trw
+from tests import test_oracle_static as tst
 from tests import test_oracle_ue8m0 as tu
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
@@ -150,4 +151,21 @@ def test_rowwise_pins_catch(tmp_path, monkeypatch, old, new):
         trw.test_unit_scales_reduce_to_integer_matmul,
         trw.test_scale_index_per_row_and_column,
     ]
+    assert any(_fails(c) for c in checks)
+
+
+STATIC_MUTANTS = [
+    # multiplies by the scale instead of dividing
+    ("q[i] = oracle_e4m3_encode(bf16_to_f32(x[i]) / s);", "q[i] = oracle_e4m3_encode(bf16_to_f32(x[i]) * s);"),
+    # scale grid not filled with the given scale
+    ("        sa[i] = s;", "        sa[i] = 1.0f;"),
+]
+
+
+@pytest.mark.parametrize("old,new", STATIC_MUTANTS)
+def test_static_pins_catch(tmp_path, monkeypatch, old, new):
+    lib = _build_mutant(tmp_path, old, new)
+    monkeypatch.setattr(oracle, "_lib", lib)
+    checks = [lambda: tst.test_vs_library_composition(0.01), tst.test_saturates_above_448_s,
+              tst.test_equals_dynamic_when_s_is_every_groups_scale]
     assert any(_fails(c) for c in checks)
