@@ -23,7 +23,7 @@ __all__ = [
     "Fp8blError", "BLOCK", "lib_path", "quant_act", "quant_weight", "block_linear",
     "block_linear_fused", "block_linear_noalloc", "workspace_bytes", "fused_workspace_bytes",
     "check", "version", "quant_act_ue8m0", "quant_weight_ue8m0", "block_linear_ue8m0",
-    "quant_rowwise", "linear_rowwise",
+    "quant_rowwise", "linear_rowwise", "quant_act_static",
 ]
 
 BLOCK = 128
@@ -49,6 +49,7 @@ _lib.fp8_quant_act_ue8m0.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_quant_weight_ue8m0.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_block_linear_ue8m0.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
 _lib.fp8_quant_rowwise.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
+_lib.fp8_quant_act_static.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp, _vp]
 _lib.fp8_linear_rowwise.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
 _lib.fp8bl_check.argtypes = [_vp]
 _lib.fp8bl_status_string.argtypes = [ctypes.c_int]
@@ -57,7 +58,7 @@ _lib.fp8bl_version.restype = ctypes.c_int
 for _f in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
            "fp8_block_linear_noalloc", "fp8bl_check", "fp8_quant_act_ue8m0",
            "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0", "fp8_quant_rowwise",
-           "fp8_linear_rowwise"):
+           "fp8_linear_rowwise", "fp8_quant_act_static"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 STATUS = {0: "FP8BL_OK", 1: "FP8BL_ERR_NULL", 2: "FP8BL_ERR_SHAPE", 3: "FP8BL_ERR_ALIGN",
@@ -101,6 +102,23 @@ def quant_act(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | 
     if s is None:
         s = torch.empty((M, K // BLOCK if K % BLOCK == 0 else 0), dtype=torch.float32, device=x.device)
     _ok(_lib.fp8_quant_act(_ptr(x), M, K, _ptr(q), _ptr(s), _stream(x)), "fp8_quant_act")
+    return q, s
+
+
+def quant_act_static(x: torch.Tensor, s_given: torch.Tensor, q: torch.Tensor | None = None,
+                     s: torch.Tensor | None = None):
+    """Static scheme: bf16 [M, K] with one given fp32 scale (a 1-element device
+    tensor) -> (e4m3 [M, K], fp32 [M, K/128] filled with that scale), ready
+    for block_linear."""
+    M, K = x.shape
+    if s_given.numel() != 1 or s_given.dtype != torch.float32:
+        raise ValueError("s_given must be one fp32 element")
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    if s is None:
+        s = torch.empty((M, K // BLOCK if K % BLOCK == 0 else 0), dtype=torch.float32, device=x.device)
+    _ok(_lib.fp8_quant_act_static(_ptr(x), M, K, _ptr(s_given), _ptr(q), _ptr(s), _stream(x)),
+        "fp8_quant_act_static")
     return q, s
 
 

@@ -108,6 +108,25 @@ fp8bl_status fp8_quant_act(const void* x_bf16, int64_t M, int64_t K, void* q_e4m
   return from_cuda(launch_act_quant(x_bf16, M, K, q_e4m3, s, d->sm_count, as_cuda(stream)));
 }
 
+fp8bl_status fp8_quant_act_static(const void* x_bf16, int64_t M, int64_t K, const float* s_given,
+                                  void* q_e4m3, float* s, fp8bl_stream_t stream) {
+  if (!dim_ok(M, true) || !dim_ok(K, false) || K % FP8BL_BLOCK) return FP8BL_ERR_SHAPE;
+  if (M == 0) return FP8BL_OK;
+  if (!x_bf16 || !s_given || !q_e4m3 || !s) return FP8BL_ERR_NULL;
+  if (!aligned(x_bf16, 16) || !aligned(q_e4m3, 16) || !aligned(s, 4) || !aligned(s_given, 4))
+    return FP8BL_ERR_ALIGN;
+  const size_t nx = static_cast<size_t>(M * K) * 2, nq = static_cast<size_t>(M * K),
+               ns = static_cast<size_t>(M * (K / 128)) * 4;
+  if (overlap(x_bf16, nx, q_e4m3, nq) || overlap(x_bf16, nx, s, ns) || overlap(q_e4m3, nq, s, ns) ||
+      overlap(s_given, 4, q_e4m3, nq) || overlap(s_given, 4, s, ns))
+    return FP8BL_ERR_OVERLAP;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  return from_cuda(
+      launch_act_quant_static(x_bf16, M, K, s_given, q_e4m3, s, d->sm_count, as_cuda(stream)));
+}
+
 fp8bl_status fp8_quant_weight(const void* w_bf16, int64_t N, int64_t K, void* q_e4m3, float* s,
                               fp8bl_stream_t stream) {
   if (!dim_ok(N, false) || !dim_ok(K, false) || N % FP8BL_BLOCK || K % FP8BL_BLOCK)

@@ -30,6 +30,11 @@ cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float
 cudaError_t launch_weight_quant(const void* w, int64_t N, int64_t K, void* q, float* s,
                                 cudaStream_t st);
 
+// Static activation scale ("DeepGEMM fast path" section): q = e4m3(x / s)
+// with the given fp32 scale *s_given (device), s[M, K/128] filled with it.
+cudaError_t launch_act_quant_static(const void* x, int64_t M, int64_t K, const float* s_given,
+                                    void* q, float* s, int sm_count, cudaStream_t st);
+
 // UE8M0 variants of both ("UE8M0 scale format"): one byte per scale, the
 // code e + 127 of the power-of-two scale 2^e.
 cudaError_t launch_act_quant_ue8m0(const void* x, int64_t M, int64_t K, void* q, uint8_t* s,

@@ -11,11 +11,13 @@
 // plus one scale.  Each warp keeps UNROLL pairs of groups in flight so the
 // SM has enough bytes outstanding to run at HBM bandwidth.
 //
-// Every kernel is instantiated twice: kPow2 = false writes fp32 scales
-// (s = amax / 448), kPow2 = true writes UE8M0 codes (the "UE8M0 scale
-// format" section of the same page: the scale rounded up to a power of two,
-// one byte each) and multiplies by the exact power of two instead of
-// dividing.
+// The kernels are instantiated per scale mode: kMode 0 writes fp32 scales
+// (s = amax / 448); kMode 1 writes UE8M0 codes (the "UE8M0 scale format"
+// section of the same page: the scale rounded up to a power of two, one byte
+// each) and multiplies by the exact power of two instead of dividing;
+// kMode 2 (activations only) is the static scheme of the page's "DeepGEMM
+// fast path" section: one given fp32 scale for the whole tensor, no abs-max,
+// written into every group's scale slot so the block GEMM applies it.
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -36,12 +38,17 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   return v;
 }
 
-// Per-group constants of either scale format, from the group's amax.
-template <bool kPow2>
+constexpr int kModeFp32 = 0;
+constexpr int kModeUe8m0 = 1;
+constexpr int kModeStatic = 2;
+
+// Per-group constants of each scale mode, from the group's amax (or, for
+// the static mode, from the given scale).
+template <int kMode>
 struct GroupQuant;
 
 template <>
-struct GroupQuant<false> {
+struct GroupQuant<kModeFp32> {
   float s;
   GroupScale g;
   __device__ __forceinline__ explicit GroupQuant(float amax)
@@ -53,7 +60,18 @@ struct GroupQuant<false> {
 };
 
 template <>
-struct GroupQuant<true> {
+struct GroupQuant<kModeStatic> {
+  float s;
+  GroupScale g;
+  __device__ __forceinline__ explicit GroupQuant(float given) : s(given), g(group_scale(given)) {}
+  __device__ __forceinline__ uint2 quant(uint4 v) const { return quant8(v, g); }
+  __device__ __forceinline__ void store_scale(void* out, int64_t i) const {
+    static_cast<float*>(out)[i] = s;
+  }
+};
+
+template <>
+struct GroupQuant<kModeUe8m0> {
   uint32_t code;
   float2 inv;
   __device__ __forceinline__ explicit GroupQuant(float amax)
@@ -65,10 +83,11 @@ struct GroupQuant<true> {
 };
 
 // num_groups = M * K / 128.  x: 16 uint4 per group; q: 16 uint2 per group.
-template <bool kPow2>
+template <int kMode>
 __global__ void __launch_bounds__(kAqThreads, 4)
 act_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, void* __restrict__ s,
-                 int64_t num_groups) {
+                 int64_t num_groups, const float* __restrict__ s_given) {
+  const float given = kMode == kModeStatic ? __ldg(s_given) : 0.0f;
   const int lane = threadIdx.x & 31;
   const int half = lane >> 4;
   const int l16 = lane & 15;
@@ -87,12 +106,16 @@ act_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, void* __res
 #pragma unroll
     for (int u = 0; u < kAqUnroll; ++u) {
       const int64_t g = (p0 + u * num_warps) * 2 + half;
-      uint32_t m = absmax8_bf16x2(v[u]);
-      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 8));
-      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      const GroupQuant<kPow2> gq(absmax_halves_f32(m));
+      float a = given;
+      if (kMode != kModeStatic) {
+        uint32_t m = absmax8_bf16x2(v[u]);
+        m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        a = absmax_halves_f32(m);
+      }
+      const GroupQuant<kMode> gq(a);
       const uint2 o = gq.quant(v[u]);
       if (g < num_groups) {
         q[g * 16 + l16] = o;
@@ -116,10 +139,11 @@ __device__ __forceinline__ void ld_stream32(const uint4* p, uint4& a, uint4& b) 
                : "l"(p));
 }
 
-template <bool kPow2>
+template <int kMode>
 __global__ void __launch_bounds__(kAqThreads, 4)
 act_quant32_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, void* __restrict__ s,
-                   int64_t num_groups) {
+                   int64_t num_groups, const float* __restrict__ s_given) {
+  const float given = kMode == kModeStatic ? __ldg(s_given) : 0.0f;
   const int lane = threadIdx.x & 31;
   const int sub = lane >> 3;      // group within the warp's 4
   const int l8 = lane & 7;        // 32-byte slice within the group
@@ -142,11 +166,15 @@ act_quant32_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, void* __r
 #pragma unroll
     for (int u = 0; u < kAq32Unroll; ++u) {
       const int64_t g = (p0 + u * num_warps) * 4 + sub;
-      uint32_t m = absmax_bf16x2(absmax8_bf16x2(va[u]), absmax8_bf16x2(vb[u]));
-      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      const GroupQuant<kPow2> gq(absmax_halves_f32(m));
+      float a = given;
+      if (kMode != kModeStatic) {
+        uint32_t m = absmax_bf16x2(absmax8_bf16x2(va[u]), absmax8_bf16x2(vb[u]));
+        m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        a = absmax_halves_f32(m);
+      }
+      const GroupQuant<kMode> gq(a);
       const uint2 lo = gq.quant(va[u]), hi = gq.quant(vb[u]);
       if (g < num_groups) {
         q[g * 8 + l8] = make_uint4(lo.x, lo.y, hi.x, hi.y);
@@ -161,7 +189,7 @@ act_quant32_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, void* __r
 // full 256-byte row segments.
 constexpr int kWqThreads = 256;
 
-template <bool kPow2>
+template <int kMode>
 __global__ void __launch_bounds__(kWqThreads)
 weight_quant_kernel(const uint4* __restrict__ w, uint2* __restrict__ q, void* __restrict__ s,
                     int64_t K, int64_t KB) {
@@ -186,7 +214,7 @@ weight_quant_kernel(const uint4* __restrict__ w, uint2* __restrict__ q, void* __
   a = warp_amax[0];
 #pragma unroll
   for (int i = 1; i < kWqThreads / 32; ++i) a = fmaxf(a, warp_amax[i]);
-  const GroupQuant<kPow2> gq(a);
+  const GroupQuant<kMode> gq(a);
   const int64_t qrow_stride = K / 8;  // uint2 per row
   const int64_t qbase = (bi * 128 + r0) * qrow_stride + bj * 16 + c;
 #pragma unroll
@@ -198,9 +226,9 @@ weight_quant_kernel(const uint4* __restrict__ w, uint2* __restrict__ q, void* __
 
 namespace {
 
-template <bool kPow2>
+template <int kMode>
 cudaError_t act_quant(const void* x, int64_t M, int64_t K, void* q, void* s, int sm_count,
-                      cudaStream_t st) {
+                      cudaStream_t st, const float* s_given = nullptr) {
   const int64_t groups = M * (K / 128);
   if (groups == 0) return cudaSuccess;
   if ((reinterpret_cast<uintptr_t>(x) & 31) == 0) {
@@ -209,8 +237,9 @@ cudaError_t act_quant(const void* x, int64_t M, int64_t K, void* q, void* s, int
     const int64_t blocks_needed = (warps_needed + (kAqThreads / 32) - 1) / (kAqThreads / 32);
     const int64_t max_blocks = static_cast<int64_t>(sm_count) * 4;
     const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
-    act_quant32_kernel<kPow2><<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
-                                                             static_cast<uint4*>(q), s, groups);
+    act_quant32_kernel<kMode><<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
+                                                             static_cast<uint4*>(q), s, groups,
+                                                             s_given);
     return cudaGetLastError();
   }
   const int64_t pairs = (groups + 1) / 2;
@@ -220,18 +249,18 @@ cudaError_t act_quant(const void* x, int64_t M, int64_t K, void* q, void* s, int
   // loop inside the kernel.
   const int64_t max_blocks = static_cast<int64_t>(sm_count) * 4;
   const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
-  act_quant_kernel<kPow2><<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
-                                                         static_cast<uint2*>(q), s, groups);
+  act_quant_kernel<kMode><<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
+                                                         static_cast<uint2*>(q), s, groups, s_given);
   return cudaGetLastError();
 }
 
-template <bool kPow2>
+template <int kMode>
 cudaError_t weight_quant(const void* w, int64_t N, int64_t K, void* q, void* s, cudaStream_t st) {
   const int64_t KB = K / 128;
   const int64_t blocks = (N / 128) * KB;
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
-  weight_quant_kernel<kPow2><<<static_cast<unsigned>(blocks), kWqThreads, 0, st>>>(
+  weight_quant_kernel<kMode><<<static_cast<unsigned>(blocks), kWqThreads, 0, st>>>(
       static_cast<const uint4*>(w), static_cast<uint2*>(q), s, K, KB);
   return cudaGetLastError();
 }
@@ -269,7 +298,7 @@ rowwise_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, float* 
   m = warp_amax[0];
 #pragma unroll
   for (int i = 1; i < kRowThreads / 32; ++i) m = absmax_bf16x2(m, warp_amax[i]);
-  const GroupQuant<false> gq(absmax_halves_f32(m));
+  const GroupQuant<kModeFp32> gq(absmax_halves_f32(m));
 #pragma unroll
   for (int i = 0; i < kRowCache; ++i) {
     const int64_t v = threadIdx.x + static_cast<int64_t>(i) * kRowThreads;
@@ -293,22 +322,27 @@ cudaError_t launch_rowwise_quant(const void* x, int64_t R, int64_t K, void* q, f
 
 cudaError_t launch_act_quant(const void* x, int64_t M, int64_t K, void* q, float* s,
                              int sm_count, cudaStream_t st) {
-  return act_quant<false>(x, M, K, q, s, sm_count, st);
+  return act_quant<kModeFp32>(x, M, K, q, s, sm_count, st);
 }
 
 cudaError_t launch_act_quant_ue8m0(const void* x, int64_t M, int64_t K, void* q, uint8_t* s,
                                    int sm_count, cudaStream_t st) {
-  return act_quant<true>(x, M, K, q, s, sm_count, st);
+  return act_quant<kModeUe8m0>(x, M, K, q, s, sm_count, st);
+}
+
+cudaError_t launch_act_quant_static(const void* x, int64_t M, int64_t K, const float* s_given,
+                                    void* q, float* s, int sm_count, cudaStream_t st) {
+  return act_quant<kModeStatic>(x, M, K, q, s, sm_count, st, s_given);
 }
 
 cudaError_t launch_weight_quant(const void* w, int64_t N, int64_t K, void* q, float* s,
                                 cudaStream_t st) {
-  return weight_quant<false>(w, N, K, q, s, st);
+  return weight_quant<kModeFp32>(w, N, K, q, s, st);
 }
 
 cudaError_t launch_weight_quant_ue8m0(const void* w, int64_t N, int64_t K, void* q, uint8_t* s,
                                       cudaStream_t st) {
-  return weight_quant<true>(w, N, K, q, s, st);
+  return weight_quant<kModeUe8m0>(w, N, K, q, s, st);
 }
 
 }  // namespace fp8bl

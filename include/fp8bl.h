@@ -87,6 +87,27 @@ fp8bl_status fp8_quant_act(const void *x_bf16, int64_t M, int64_t K,
                            void *q_e4m3, float *s, fp8bl_stream_t stream);
 
 /*
+ * fp8_quant_act_static -- activation quantization with one given scale
+ * (the static scheme).
+ * Passage: "Fine-grained FP8" page, "DeepGEMM fast path" section (static
+ * activation quantization, next to the dynamic scheme; the page says no more).
+ * This library reads it as: one fp32 activation scale per linear, supplied
+ * by the caller (calibrated elsewhere), q = e4m3(fp32(x / s)) rounded and
+ * saturated as above (|x| > 448 s gives +-448), and the product is the block
+ * linear with every activation group scale equal to s.  So the call writes
+ * s into every slot of the [M, K/128] scale array, and fp8_block_linear /
+ * fp8_block_linear_noalloc take the outputs unchanged.
+ *
+ *   x_bf16  in : bf16 [M, K]          s_given in : device pointer to one fp32,
+ *   q_e4m3  out: e4m3 [M, K]                       finite and > 0 (not checked)
+ *   s       out: fp32 [M, K/128], every element = *s_given
+ *   M >= 0 (M == 0 enqueues nothing), K > 0, K % 128 == 0, M, K <= FP8BL_MAX_DIM.
+ */
+fp8bl_status fp8_quant_act_static(const void *x_bf16, int64_t M, int64_t K,
+                                  const float *s_given, void *q_e4m3, float *s,
+                                  fp8bl_stream_t stream);
+
+/*
  * fp8_quant_weight -- 128 x 128 block weight quantization.
  * Passage: "Fine-grained FP8" page, first bullet of the opening list
  * (weight_block_size = (128, 128)).

@@ -33,7 +33,7 @@ def test_header_declares_expected_calls():
     for n in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
               "fp8_block_linear_workspace_bytes", "fp8bl_check", "fp8bl_status_string",
               "fp8_quant_act_ue8m0", "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0",
-              "fp8_quant_rowwise", "fp8_linear_rowwise"):
+              "fp8_quant_rowwise", "fp8_linear_rowwise", "fp8_quant_act_static"):
         assert n in names
 
 
@@ -154,6 +154,17 @@ def test_rowwise_argument_errors(lib):
     assert fl(a, sa, None, sw, y, 4, 32, 32, None) == 1
     assert fl(a, sa, w, _p(0x4000004), y, 4, 32, 32, None) == 3    # s_w must be 16-byte aligned
     assert fl(a, sa, w, sw, w, 4, 32, 32, None) == 8
+
+
+def test_static_argument_errors(lib):
+    f = lib.fp8_quant_act_static
+    f.argtypes = [V, ctypes.c_int64, ctypes.c_int64, V, V, V, V]
+    g, sg, q, s = _p(0x10000), _p(0x90000), _p(0x20000), _p(0x30000)
+    assert f(g, 4, 100, sg, q, s, None) == 2          # K % 128
+    assert f(g, 0, 128, None, None, None, None) == 0  # empty
+    assert f(g, 4, 128, None, q, s, None) == 1        # no given scale
+    assert f(g, 4, 128, _p(0x90002), q, s, None) == 3 # given scale misaligned
+    assert f(g, 4, 128, _p(0x20010), q, s, None) == 8 # given scale inside q
 
 
 def test_valid_call_without_gpu_reports_cuda_error(lib):

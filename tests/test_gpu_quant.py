@@ -109,3 +109,48 @@ def test_act_quant_16_byte_aligned_input(fp8):
     qo, so = oracle.quant_act(bits, nthreads=8)
     assert np.array_equal(f32(s).view(np.uint32), so.view(np.uint32))
     assert np.array_equal(u8(q), qo)
+
+
+# ------------------------------------------------ static activation scale
+
+
+@pytest.mark.parametrize("M,K,sc", [(32, 512, 0.01), (1, 128, 1.0), (129, 7168, 0.0037),
+                                    (64, 18432, 2.5e-4)])
+def test_act_quant_static(fp8, M, K, sc):
+    bits = wl.student_t_outliers(M, K, 3.0, 0.01, 100.0, M + K)
+    bits[0, :128] = 0x8000
+    s_given = torch.tensor([sc], dtype=torch.float32, device="cuda")
+    q, s = fp8.quant_act_static(to_dev(bits), s_given)
+    torch.cuda.synchronize()
+    qo, so = oracle.quant_act_static(bits, sc)
+    assert np.array_equal(f32(s), so)
+    assert np.count_nonzero(u8(q) != qo) == 0
+
+
+def test_act_quant_static_16_byte_aligned_input(fp8):
+    bits = wl.normal((9, 384), 3.0, 5)
+    buf = torch.empty(9 * 384 + 8, dtype=torch.bfloat16, device="cuda")
+    x = buf[8:].view(9, 384)
+    x.copy_(to_dev(bits))
+    s_given = torch.tensor([0.004], dtype=torch.float32, device="cuda")
+    q, s = fp8.quant_act_static(x, s_given)
+    torch.cuda.synchronize()
+    qo, so = oracle.quant_act_static(bits, 0.004)
+    assert np.array_equal(u8(q), qo) and np.array_equal(f32(s), so)
+
+
+def test_static_then_block_linear(fp8):
+    """The static outputs feed the block linear unchanged; parity with the
+    oracle's block linear from the same codes and scales."""
+    from tests.parity import check_gemm
+    xb = wl.normal((200, 1024), 1.0, 6)
+    wb = wl.normal((512, 1024), 0.02, 7)
+    sc = float(np.abs(wl.bf16_bits_to_f32(xb)).max() / 448.0 * 0.5)   # half the range: some saturation
+    q_a, s_a = fp8.quant_act_static(to_dev(xb), torch.tensor([sc], dtype=torch.float32, device="cuda"))
+    q_w, s_w = fp8.quant_weight(to_dev(wb))
+    y = fp8.block_linear(q_a, s_a, q_w, s_w)
+    fp8.check()
+    qo, so = oracle.quant_act_static(xb, sc)
+    assert np.array_equal(u8(q_a), qo)
+    R = oracle.block_linear(qo, so, u8(q_w), f32(s_w), nthreads=8)
+    check_gemm(f32(y), R, "static + block linear")
