@@ -9,7 +9,8 @@ variant of the page's "UE8M0 scale format" section (float8_e8m0fnu scales),
 whose GEMM runs on the tensor core's block-scaled MMA.  ``quant_rowwise`` /
 ``linear_rowwise`` are the row-wise FP8 scheme (fp8r) of the "BFL (fp8r /
 nvfp4)" page: one fp32 scale per activation row and per weight row.
-``quant_act_static`` is the static activation scheme (one given scale).
+``quant_act_static`` is the static activation scheme (one given scale), and
+``grouped_linear_ue8m0`` the grouped (MoE expert) form of the UE8M0 linear.
 
 The functions below come from ``_binding`` (a ctypes binding of
 ``libfp8bl.so``), loaded on first use so that the ``build`` submodule can be
@@ -20,7 +21,7 @@ __all__ = [
     "Fp8blError", "BLOCK", "STATUS", "lib_path", "quant_act", "quant_weight", "block_linear",
     "block_linear_fused", "block_linear_noalloc", "workspace_bytes", "fused_workspace_bytes",
     "check", "version", "quant_act_ue8m0", "quant_weight_ue8m0", "block_linear_ue8m0",
-    "quant_rowwise", "linear_rowwise", "quant_act_static",
+    "quant_rowwise", "linear_rowwise", "quant_act_static", "grouped_linear_ue8m0",
 ]
 
 

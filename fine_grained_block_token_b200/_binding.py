@@ -23,7 +23,7 @@ __all__ = [
     "Fp8blError", "BLOCK", "lib_path", "quant_act", "quant_weight", "block_linear",
     "block_linear_fused", "block_linear_noalloc", "workspace_bytes", "fused_workspace_bytes",
     "check", "version", "quant_act_ue8m0", "quant_weight_ue8m0", "block_linear_ue8m0",
-    "quant_rowwise", "linear_rowwise", "quant_act_static",
+    "quant_rowwise", "linear_rowwise", "quant_act_static", "grouped_linear_ue8m0",
 ]
 
 BLOCK = 128
@@ -50,6 +50,7 @@ _lib.fp8_quant_weight_ue8m0.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_block_linear_ue8m0.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
 _lib.fp8_quant_rowwise.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_quant_act_static.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp, _vp]
+_lib.fp8_grouped_linear_ue8m0.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]
 _lib.fp8_linear_rowwise.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
 _lib.fp8bl_check.argtypes = [_vp]
 _lib.fp8bl_status_string.argtypes = [ctypes.c_int]
@@ -58,7 +59,7 @@ _lib.fp8bl_version.restype = ctypes.c_int
 for _f in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
            "fp8_block_linear_noalloc", "fp8bl_check", "fp8_quant_act_ue8m0",
            "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0", "fp8_quant_rowwise",
-           "fp8_linear_rowwise", "fp8_quant_act_static"):
+           "fp8_linear_rowwise", "fp8_quant_act_static", "fp8_grouped_linear_ue8m0"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 STATUS = {0: "FP8BL_OK", 1: "FP8BL_ERR_NULL", 2: "FP8BL_ERR_SHAPE", 3: "FP8BL_ERR_ALIGN",
@@ -176,6 +177,24 @@ def block_linear_ue8m0(q_a, s_a, q_w, s_w, y=None) -> torch.Tensor:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
     _ok(_lib.fp8_block_linear_ue8m0(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
                                     _stream(q_a)), "fp8_block_linear_ue8m0")
+    return y
+
+
+def grouped_linear_ue8m0(q_a, s_a, q_w, s_w, expert_offsets, y=None) -> torch.Tensor:
+    """Grouped (MoE expert) UE8M0 linear: rows [off[e], off[e+1]) of
+    (e4m3 [M,K], e8m0 [M,K/128]) times expert e of (e4m3 [E,N,K],
+    e8m0 [E,N/128,K/128]); expert_offsets int32 [E+1] on the device."""
+    M, K = q_a.shape
+    E, N, Kw = q_w.shape
+    if Kw != K:
+        raise ValueError("q_a and q_w disagree on K")
+    if expert_offsets.dtype != torch.int32 or expert_offsets.numel() != E + 1:
+        raise ValueError("expert_offsets must be int32 [E + 1]")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
+    _ok(_lib.fp8_grouped_linear_ue8m0(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w),
+                                      _ptr(expert_offsets), _ptr(y), M, N, K, E, _stream(q_a)),
+        "fp8_grouped_linear_ue8m0")
     return y
 
 

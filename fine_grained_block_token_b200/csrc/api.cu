@@ -272,6 +272,30 @@ fp8bl_status fp8_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const v
       launch_block_linear_ue8m0(q_a, s_a, q_w, s_w, y_bf16, M, N, K, *d, as_cuda(stream)));
 }
 
+fp8bl_status fp8_grouped_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                      const uint8_t* s_w, const int32_t* expert_offsets,
+                                      void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t E,
+                                      fp8bl_stream_t stream) {
+  if (!linear_dims_ok(M, N, K) || E < 1 || E > kMaxExperts || N * E > FP8BL_MAX_DIM)
+    return FP8BL_ERR_SHAPE;
+  if (M == 0) return FP8BL_OK;
+  if (!q_a || !s_a || !q_w || !s_w || !expert_offsets || !y_bf16) return FP8BL_ERR_NULL;
+  if (!aligned(q_a, 16) || !aligned(q_w, 16) || !aligned(y_bf16, 16) || !aligned(expert_offsets, 4))
+    return FP8BL_ERR_ALIGN;
+  const size_t ny = static_cast<size_t>(M * N) * 2;
+  if (overlap(y_bf16, ny, q_a, static_cast<size_t>(M * K)) ||
+      overlap(y_bf16, ny, q_w, static_cast<size_t>(E * N * K)) ||
+      overlap(y_bf16, ny, s_a, static_cast<size_t>(M * (K / 128))) ||
+      overlap(y_bf16, ny, s_w, static_cast<size_t>(E * (N / 128) * (K / 128))) ||
+      overlap(y_bf16, ny, expert_offsets, static_cast<size_t>(E + 1) * 4))
+    return FP8BL_ERR_OVERLAP;
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  return from_cuda(launch_grouped_linear_ue8m0(q_a, s_a, q_w, s_w, expert_offsets, y_bf16, M, N,
+                                               K, E, *d, as_cuda(stream)));
+}
+
 fp8bl_status fp8_quant_rowwise(const void* x_bf16, int64_t R, int64_t K, void* q_e4m3, float* s,
                                fp8bl_stream_t stream) {
   if (!dim_ok(R, true) || !dim_ok(K, false) || K % 16) return FP8BL_ERR_SHAPE;

@@ -59,6 +59,14 @@ cudaError_t launch_linear_rowwise(const void* q_a, const float* s_a, const void*
                                   const float* s_w, void* y, int64_t M, int64_t N, int64_t K,
                                   const DeviceInfo& dev, cudaStream_t st);
 
+// Grouped (MoE expert) UE8M0 linear: row segments [off[e], off[e+1]) of
+// q_a times expert e's weights, q_w [E, N, K], s_w [E, N/128, K/128].
+constexpr int kMaxExperts = 1024;
+cudaError_t launch_grouped_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                        const uint8_t* s_w, const int32_t* offsets, void* y,
+                                        int64_t M, int64_t N, int64_t K, int64_t E,
+                                        const DeviceInfo& dev, cudaStream_t st);
+
 // Largest M served by the decode (swap-AB, stream-K) schedule.
 constexpr int64_t kDecodeMaxM = 64;
 

@@ -39,6 +39,16 @@
 // A single 256-column accumulator is what fits next to the scale-factor
 // columns, so the MMAs of the next tile wait for the epilogue's TMEM reads
 // (not for its stores).
+//
+// Grouped (MoE expert) form, same kernel: the rows of A are split into E
+// contiguous segments [off[e], off[e+1]) and segment e is multiplied by
+// expert e's weights W[e] ([E, N, K] stacked, scales [E, N/128, K/128]).
+// Warp 3 turns the offsets into a shared-memory table at start-up (clamped
+// to [0, M] and made non-decreasing, so any offsets stay in bounds) with
+// each expert's count of 128-row blocks; tiles run over all experts' blocks
+// (M-fastest) times the N tiles, and a tile's rows past its segment, like
+// its columns past N, are computed on whatever TMA loads but never stored.
+// The plain linear is the case E = 1, off = {0, M}.
 // Every mbarrier wait is bounded in time; on expiry the kernel records an
 // error code in the error word, drains what it started and exits cleanly.
 #include <cstdint>
@@ -76,15 +86,17 @@ constexpr int SMEM_B_OFF = SMEM_A_OFF + STAGES * A_BYTES;
 constexpr int SMEM_BAR_OFF = SMEM_B_OFF + STAGES * B_BYTES;
 constexpr int NUM_BARS = 2 * STAGES + 3;  // full, empty, tfull, tempty, drain
 constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NUM_BARS * 8;
-constexpr int SMEM_BYTES = SMEM_MISC_OFF + 16 + 1024;  // + slack for 1024-byte alignment
+constexpr int SMEM_TAB_OFF = SMEM_MISC_OFF + 16;   // expert table: offsets, block prefix
+constexpr int SMEM_BYTES = SMEM_TAB_OFF + 2 * (kMaxExperts + 1) * 4 + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(SF_COL0 >= ACC_COL + BN && SF_COL0 + 16 * STAGES <= TMEM_COLS, "TMEM columns");
 
 struct GemmArgs {
-  const uint8_t* s_a;   // ue8m0 [M, K/128]
-  const uint8_t* s_w;   // ue8m0 [N/128, K/128]
+  const uint8_t* s_a;      // ue8m0 [M, K/128]
+  const uint8_t* s_w;      // ue8m0 [E, N/128, K/128]
+  const int* offsets;      // [E + 1] segment starts (device), or null for one segment {0, M}
   __nv_bfloat16* y;
-  int M, N, K;
+  int M, N, K, E;
   int* err;
 };
 
@@ -110,11 +122,48 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int M = args.M, N = args.N, K = args.K;
-  const int num_m = (M + BM - 1) / BM;
+  const int M = args.M, N = args.N, K = args.K, E = args.E;
   const int num_n = (N + BN - 1) / BN;
   const int num_kb = K / BK;
-  const int num_tiles = num_m * num_n;
+  int* tab_off = reinterpret_cast<int*>(smem + SMEM_TAB_OFF);   // [E + 1]
+  int* tab_pre = tab_off + (kMaxExperts + 1);                    // [E + 1] blocks before e
+
+  if (warp == 3) {
+    // segment offsets: clamped to [0, M], running max (warp scans, 32 at a time)
+    int carry = 0;
+    for (int base = 0; base <= E; base += 32) {
+      const int i = base + lane;
+      int o = 0;
+      if (i <= E) {
+        o = args.offsets != nullptr ? __ldg(args.offsets + i) : (i == 0 ? 0 : M);
+        o = min(max(o, 0), M);
+      }
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, o, d);
+        if (lane >= d) o = max(o, t);
+      }
+      o = max(o, carry);
+      if (i <= E) tab_off[i] = o;
+      carry = __shfl_sync(0xffffffffu, o, 31);
+    }
+    __syncwarp();
+    // 128-row blocks before each expert
+    carry = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int b = e < E ? (tab_off[e + 1] - tab_off[e] + BM - 1) / BM : 0;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, b, d);
+        if (lane >= d) b += t;
+      }
+      b += carry;
+      if (e < E) tab_pre[e + 1] = b;
+      carry = __shfl_sync(0xffffffffu, b, 31);
+    }
+    if (lane == 0) tab_pre[0] = 0;
+  }
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -136,6 +185,21 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+  const int total_m = tab_pre[E];
+  const int num_tiles = total_m * num_n;
+  // tile -> (expert, first row, end of the expert's rows, N tile)
+  auto map_tile = [&](int tile, int& e, int& row0, int& row_end, int& n_blk) {
+    const int mb = tile % total_m;
+    n_blk = tile / total_m;
+    int lo = 0, hi = E - 1;          // the last expert whose first block is <= mb
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (tab_pre[mid] <= mb) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+    row0 = tab_off[e] + (mb - tab_pre[e]) * BM;
+    row_end = tab_off[e + 1];
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -145,7 +209,8 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
       uint32_t c = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m_blk = tile % num_m, n_blk = tile / num_m;
+        int e, row0, row_end, n_blk;
+        map_tile(tile, e, row0, row_end, n_blk);
         for (int kb = 0; kb < num_kb; ++kb, ++c) {
           const int s = c % STAGES;
           const uint32_t ph = (c / STAGES) & 1u;
@@ -156,9 +221,9 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
           }
           ptx::mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
           ptx::tma_load_2d(smem_base + SMEM_A_OFF + s * A_BYTES, &tmap_a, full_bar(s), kb * BK,
-                           m_blk * BM);
+                           row0);
           ptx::tma_load_2d(smem_base + SMEM_B_OFF + s * B_BYTES, &tmap_b, full_bar(s), kb * BK,
-                           n_blk * BN);
+                           e * N + n_blk * BN);
           last_phase[s] = static_cast<int>(ph);
         }
       }
@@ -229,19 +294,23 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
     auto write_sf = [&](uint32_t c) -> bool {
       const int tile = static_cast<int>(blockIdx.x + (c / num_kb) * gridDim.x);
       const int kb = static_cast<int>(c % num_kb);
-      const int m_blk = tile % num_m, n_blk = tile / num_m;
+      int e, row0, row_end, n_blk;
+      map_tile(tile, e, row0, row_end, n_blk);
       // loads first: they land while the slot is still in use
       uint32_t v[16];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int row = m_blk * BM + 32 * j + lane;
-        v[j] = row < M ? __ldg(args.s_a + static_cast<int64_t>(row) * num_kb + kb) : kUnitScale;
+        const int row = row0 + 32 * j + lane;
+        v[j] = row < row_end ? __ldg(args.s_a + static_cast<int64_t>(row) * num_kb + kb)
+                             : kUnitScale;
       }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int nb = n_blk * 2 + h;
-        v[4 + 4 * h] = nb < nblk_count ? __ldg(args.s_w + static_cast<int64_t>(nb) * num_kb + kb)
-                                       : kUnitScale;
+        v[4 + 4 * h] =
+            nb < nblk_count
+                ? __ldg(args.s_w + (static_cast<int64_t>(e) * nblk_count + nb) * num_kb + kb)
+                : kUnitScale;
       }
       const int s = c % STAGES;
       const uint32_t ph = (c / STAGES) & 1u;
@@ -277,8 +346,9 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
         if (!ok) break;
       }
-      const int m_blk = tile % num_m, n_blk = tile / num_m;
-      const int row = m_blk * BM + quarter * 32 + lane;
+      int e, row0, row_end, n_blk;
+      map_tile(tile, e, row0, row_end, n_blk);
+      const int row = row0 + quarter * 32 + lane;
       const int nb = n_blk * 2 + half;
       if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(tfull_bar, t_local & 1u))) {
         if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
@@ -293,7 +363,7 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(tempty_bar);
-      if (row < M && nb < nblk_count) {
+      if (row < row_end && nb < nblk_count) {
         uint4* dst = reinterpret_cast<uint4*>(args.y + static_cast<int64_t>(row) * N + nb * 128);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -331,27 +401,39 @@ cudaError_t ensure_smem_attr() {
 
 }  // namespace
 
-cudaError_t launch_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
-                                      const uint8_t* s_w, void* y, int64_t M, int64_t N,
-                                      int64_t K, const DeviceInfo& dev, cudaStream_t st) {
+cudaError_t launch_grouped_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                        const uint8_t* s_w, const int32_t* offsets, void* y,
+                                        int64_t M, int64_t N, int64_t K, int64_t E,
+                                        const DeviceInfo& dev, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
+  if (E < 1 || E > kMaxExperts) return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_attr();
   if (e != cudaSuccess) return e;
   CUtensorMap ta, tb;
-  if (!make_tmap_u8(&ta, q_a, M, K, BM, BK) || !make_tmap_u8(&tb, q_w, N, K, BN, BK))
+  if (!make_tmap_u8(&ta, q_a, M, K, BM, BK) || !make_tmap_u8(&tb, q_w, E * N, K, BN, BK))
     return cudaErrorInvalidValue;
   GemmArgs a;
   a.s_a = s_a;
   a.s_w = s_w;
+  a.offsets = offsets;
   a.y = static_cast<__nv_bfloat16*>(y);
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
+  a.E = static_cast<int>(E);
   a.err = dev.error_flag;
-  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  // tiles: at most ceil(M / 128) + E row blocks (one partial block per segment)
+  const int64_t row_blocks = (M + BM - 1) / BM + (offsets != nullptr ? E : 0);
+  const int64_t tiles = row_blocks * ((N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
   gemm_ue8m0_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                      const uint8_t* s_w, void* y, int64_t M, int64_t N,
+                                      int64_t K, const DeviceInfo& dev, cudaStream_t st) {
+  return launch_grouped_linear_ue8m0(q_a, s_a, q_w, s_w, nullptr, y, M, N, K, 1, dev, st);
 }
 
 }  // namespace fp8bl

@@ -232,6 +232,33 @@ fp8bl_status fp8_block_linear_ue8m0(const void *q_a, const uint8_t *s_a,
                                     fp8bl_stream_t stream);
 
 /*
+ * fp8_grouped_linear_ue8m0 -- grouped (MoE expert) form of
+ * fp8_block_linear_ue8m0.
+ * Passage: "Fine-grained FP8" page, "DeepGEMM fast path" section (MoE expert
+ * matmuls routed through DeepGEMM, experts_implementation="deepgemm" /
+ * "deepgemm_megamoe" on Blackwell) and its "UE8M0 scale format" section
+ * (on Blackwell the DeepGEMM expert kernels accept only UE8M0 scales).  The
+ * pages give no layout; this library takes the plainest one, a contiguous
+ * grouping: the M rows of q_a are sorted by expert, expert e owns rows
+ * [expert_offsets[e], expert_offsets[e+1]) and multiplies them by its own
+ * weights, y[rows of e] = that expert's fp8_block_linear_ue8m0.
+ *
+ *   q_a  in : e4m3 [M, K]           s_a in : ue8m0 codes [M, K/128]
+ *   q_w  in : e4m3 [E, N, K]        s_w in : ue8m0 codes [E, N/128, K/128]
+ *   expert_offsets in: DEVICE int32 [E + 1], 0 = off[0] <= off[1] <= ... <= off[E] = M.
+ *            The kernel clamps every value to [0, M] and takes a running maximum,
+ *            so malformed offsets cannot make it read or write out of bounds;
+ *            rows outside [off[0], off[E]) are not written.
+ *   y_bf16 out: bf16 [M, N]
+ *   1 <= E <= 1024, M >= 0, N, K > 0 and multiples of 128, E * N <= FP8BL_MAX_DIM.
+ */
+fp8bl_status fp8_grouped_linear_ue8m0(const void *q_a, const uint8_t *s_a,
+                                      const void *q_w, const uint8_t *s_w,
+                                      const int32_t *expert_offsets, void *y_bf16,
+                                      int64_t M, int64_t N, int64_t K, int64_t E,
+                                      fp8bl_stream_t stream);
+
+/*
  * Row-wise FP8 variant (fp8r).
  * Passage: "BFL (fp8r / nvfp4)" page of the diffusers docs, first bullet of
  * its list (an E4M3 weight with one fp32 weight scale per row; activations

@@ -334,6 +334,28 @@ def quant_act_static(x_bf16, s: float):
     return q, sa
 
 
+def grouped_linear_ue8m0(q_a, c_a, q_w, c_w, offsets, rows=None, nthreads: int = 1) -> np.ndarray:
+    """Grouped (MoE expert) UE8M0 linear, fp64 [M, N]: rows [off[e], off[e+1])
+    times expert e's weights q_w[e] / c_w[e] (a contiguous grouping of the
+    rows by expert, each segment the block linear of its expert).  Rows
+    outside [off[0], off[E]), and rows not listed in ``rows`` when it is
+    given, are NaN."""
+    q_a = np.ascontiguousarray(q_a, dtype=np.uint8)
+    q_w = np.ascontiguousarray(q_w, dtype=np.uint8)
+    M, K = q_a.shape
+    E, N, _ = q_w.shape
+    off = [int(v) for v in offsets]
+    if len(off) != E + 1 or off[0] < 0 or off[-1] > M or any(b < a for a, b in zip(off, off[1:])):
+        raise ValueError("offsets must be non-decreasing within [0, M]")
+    want = np.arange(M) if rows is None else np.unique(np.asarray(rows, dtype=np.int64))
+    y = np.full((M, N), np.nan, dtype=np.float64)
+    for e in range(E):
+        r = want[(want >= off[e]) & (want < off[e + 1])]
+        if len(r):
+            y[r] = block_linear_ue8m0(q_a, c_a, q_w[e], c_w[e], rows=r, nthreads=nthreads)
+    return y
+
+
 def bf16_rne(y: np.ndarray) -> np.ndarray:
     """Round fp64 values to bf16 (nearest, ties to even), returned as fp64.
 

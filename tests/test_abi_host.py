@@ -33,7 +33,8 @@ def test_header_declares_expected_calls():
     for n in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
               "fp8_block_linear_workspace_bytes", "fp8bl_check", "fp8bl_status_string",
               "fp8_quant_act_ue8m0", "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0",
-              "fp8_quant_rowwise", "fp8_linear_rowwise", "fp8_quant_act_static"):
+              "fp8_quant_rowwise", "fp8_linear_rowwise", "fp8_quant_act_static",
+              "fp8_grouped_linear_ue8m0"):
         assert n in names
 
 
@@ -165,6 +166,20 @@ def test_static_argument_errors(lib):
     assert f(g, 4, 128, None, q, s, None) == 1        # no given scale
     assert f(g, 4, 128, _p(0x90002), q, s, None) == 3 # given scale misaligned
     assert f(g, 4, 128, _p(0x20010), q, s, None) == 8 # given scale inside q
+
+
+def test_grouped_argument_errors(lib):
+    f = lib.fp8_grouped_linear_ue8m0
+    f.argtypes = [V, V, V, V, V, V] + [ctypes.c_int64] * 4 + [V]
+    a, sa, w, sw, off, y = (_p(0x1000000 * (i + 1)) for i in range(6))
+    assert f(a, sa, w, sw, off, y, 4, 128, 128, 0, None) == 2        # E < 1
+    assert f(a, sa, w, sw, off, y, 4, 128, 128, 1025, None) == 2     # E > 1024
+    assert f(a, sa, w, sw, off, y, 4, 1 << 24, 128, 128, None) == 2  # E * N too large
+    assert f(a, sa, w, sw, off, y, 4, 100, 128, 2, None) == 2        # N % 128
+    assert f(a, sa, w, sw, off, y, 0, 128, 128, 2, None) == 0        # empty
+    assert f(a, sa, w, sw, None, y, 4, 128, 128, 2, None) == 1       # no offsets
+    assert f(a, sa, w, sw, _p(0x5000002), y, 4, 128, 128, 2, None) == 3
+    assert f(a, sa, w, sw, off, off, 4, 128, 128, 2, None) == 8      # y over the offsets
 
 
 def test_valid_call_without_gpu_reports_cuda_error(lib):

@@ -1,0 +1,111 @@
+"""GPU parity of the grouped (MoE expert) UE8M0 linear against the oracle,
+through the C ABI.
+
+Method: "Fine-grained FP8" page ("DeepGEMM fast path": MoE expert matmuls;
+"UE8M0 scale format": Blackwell expert kernels take UE8M0 scales), read as a
+contiguous grouping of rows by expert.  Segment sizes cover empty experts,
+segments shorter than a 128-row tile, and segments that end inside a tile;
+malformed offsets are clamped by the kernel, and the test checks the clamped
+meaning.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from tests.parity import check_gemm, f32, to_dev, u8
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    import fine_grained_block_token_b200 as m
+    return m
+
+
+def _segments(g, M, E, p_empty=0.2):
+    """Random non-negative counts summing to M, some experts empty."""
+    w = g.exponential(1.0, E) * (g.random(E) > p_empty)
+    if w.sum() == 0:
+        w[0] = 1.0
+    c = np.floor(w / w.sum() * M).astype(np.int64)
+    c[np.argmax(w)] += M - c.sum()
+    return np.concatenate([[0], np.cumsum(c)]).astype(np.int32)
+
+
+def _quantized(fp8, M, N, K, E, seed):
+    xb = wl.normal((M, K), 1.0, seed)
+    wb = wl.normal((E * N, K), 0.02, seed + 1)
+    q_a, s_a = fp8.quant_act_ue8m0(to_dev(xb))
+    q_w, s_w = fp8.quant_weight_ue8m0(to_dev(wb))
+    return q_a, s_a, q_w.view(E, N, K), s_w.view(E, N // 128, K // 128)
+
+
+def _check(fp8, q_a, s_a, q_w, s_w, off, rows=None, label=""):
+    M = q_a.shape[0]
+    y = torch.full((M, q_w.shape[1]), 7.0, dtype=torch.bfloat16, device="cuda")
+    fp8.grouped_linear_ue8m0(q_a, s_a, q_w, s_w, torch.from_numpy(off).cuda(), y)
+    fp8.check()
+    R = oracle.grouped_linear_ue8m0(u8(q_a), u8(s_a), u8(q_w), u8(s_w), off, rows=rows, nthreads=8)
+    covered = np.zeros(M, bool)
+    covered[off[0]:off[-1]] = True
+    Y = f32(y)
+    assert np.all(Y[~covered] == 7.0), label + ": rows outside the segments were written"
+    idx = np.nonzero(covered)[0] if rows is None else np.intersect1d(rows, np.nonzero(covered)[0])
+    check_gemm(Y[idx], R[idx], label)
+
+
+@pytest.mark.parametrize("M,N,K,E,seed", [
+    (300, 256, 256, 3, 0), (1000, 384, 512, 8, 1), (77, 256, 384, 5, 2), (2048, 512, 1024, 64, 3),
+    (129, 128, 128, 1, 4),
+])
+def test_random_segments(fp8, M, N, K, E, seed):
+    g = np.random.default_rng(seed)
+    q_a, s_a, q_w, s_w = _quantized(fp8, M, N, K, E, 10 * seed)
+    _check(fp8, q_a, s_a, q_w, s_w, _segments(g, M, E), label=f"{M}x{N}x{K} E={E}")
+
+
+def test_segments_not_covering_all_rows(fp8):
+    q_a, s_a, q_w, s_w = _quantized(fp8, 400, 256, 256, 4, 7)
+    _check(fp8, q_a, s_a, q_w, s_w, np.array([37, 100, 100, 250, 333], np.int32), label="partial")
+
+
+def test_single_expert_equals_plain_call(fp8):
+    q_a, s_a, q_w, s_w = _quantized(fp8, 333, 384, 512, 1, 8)
+    y1 = fp8.block_linear_ue8m0(q_a, s_a, q_w[0], s_w[0])
+    y2 = fp8.grouped_linear_ue8m0(q_a, s_a, q_w, s_w, torch.tensor([0, 333], dtype=torch.int32,
+                                                                    device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_malformed_offsets_are_clamped(fp8):
+    """Out-of-range and decreasing offsets: the kernel clamps each to [0, M]
+    and takes a running maximum; the result is the grouping those define."""
+    M = 300
+    q_a, s_a, q_w, s_w = _quantized(fp8, M, 256, 256, 5, 9)
+    raw = np.array([-50, 120, 80, 400, 250, 1000], np.int32)
+    clamped = np.maximum.accumulate(np.clip(raw, 0, M)).astype(np.int32)
+    y = torch.full((M, 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    fp8.grouped_linear_ue8m0(q_a, s_a, q_w, s_w, torch.from_numpy(raw).cuda(), y)
+    fp8.check()
+    R = oracle.grouped_linear_ue8m0(u8(q_a), u8(s_a), u8(q_w), u8(s_w), clamped)
+    check_gemm(f32(y)[clamped[0]:clamped[-1]], R[clamped[0]:clamped[-1]], "clamped")
+
+
+def test_moe_sized(fp8):
+    """DeepSeek-V3-like expert MLP up-projection shape: 16 experts, K 7168,
+    N 2048, 8192 routed token rows; sampled rows against the oracle."""
+    g = np.random.default_rng(12)
+    M, N, K, E = 8192, 2048, 7168, 16
+    q_a, s_a, q_w, s_w = _quantized(fp8, M, N, K, E, 120)
+    off = _segments(g, M, E, p_empty=0.1)
+    rows = np.unique(np.concatenate([off[:-1], np.maximum(off[1:] - 1, 0), g.choice(M, 24, replace=False)]))
+    rows = rows[rows < M]
+    _check(fp8, q_a, s_a, q_w, s_w, off, rows=rows, label="moe")
+
+
+def test_no_timeout_recorded(fp8):
+    fp8.check()
