@@ -1,7 +1,7 @@
 """Benchmark of the fine-grained FP8 linear hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload llama3_prefill|deepseek_mlp|llama3_decode|sweep]
+                    [--workload llama3_prefill|deepseek_mlp|llama3_decode|sweep|deepseek_moe]
 
 One step (default workload, Llama-3-8B MLP prefill, M = 4096 tokens):
     quant_act(X1 [4096, 4096])   -> block_linear vs W_gate_up [28672, 4096]
@@ -276,6 +276,8 @@ def run_reference(args):
     _, rank, _ = rank_info()
     if rank != 0:
         return 0
+    if args.workload == "deepseek_moe":
+        return run_reference_moe(args)
     lins = workload_linears(args.workload)
     prepared = cpu_prepare(lins, args.ref_rows)
     for _ in range(args.warmup):
@@ -297,6 +299,242 @@ def run_reference(args):
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------ MoE experts
+
+def run_reference_moe(args):
+    """Reference arm on the MoE workload: the oracle on `ref_rows` routed rows
+    per expert linear, taken from the two largest experts (whose weights the
+    oracle quantizes before timing).  The weights are drawn by torch's CPU
+    generator (same distribution and seed as the GPU arm's, another stream)."""
+    import torch
+    import oracle
+    g = np.random.default_rng(0)
+    prepared = []
+    for name in ("up", "down"):
+        xb, off = wl.deepseek_moe(name)
+        N, K = wl.MOE_LINEARS[name]
+        E = wl.MOE_EXPERTS
+        big = np.argsort(np.diff(off))[-2:]
+        w = wl.deepseek_moe_weights(name, "cpu").view(torch.int16).numpy().view(np.uint16)
+        q_w = np.zeros((E, N, K), np.uint8)
+        s_w = np.full((E, N // 128, K // 128), 127, np.uint8)
+        for e in big:
+            q_w[e], s_w[e] = oracle.quant_weight_ue8m0(np.ascontiguousarray(w[e * N:(e + 1) * N]))
+        cand = np.concatenate([np.arange(off[e], off[e + 1]) for e in big])
+        rows = np.sort(g.choice(cand, min(args.ref_rows, len(cand)), replace=False))
+        prepared.append((name, xb, q_w, s_w, off, rows))
+    for _ in range(args.warmup):
+        for name, xb, q_w, s_w, off, rows in prepared:
+            moe_oracle_rows(xb, q_w, s_w, off, rows)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        for name, xb, q_w, s_w, off, rows in prepared:
+            t, f, _ = moe_oracle_rows(xb, q_w, s_w, off, rows)
+            tot_t += t
+            tot_f += f
+    value = tot_f / tot_t / 1e12
+    desc = (f"{args.ref_rows} routed rows of the two largest experts per expert linear (up, down): "
+            "ue8m0 activation quant + fp64 grouped GEMM of those rows; weights quantized before timing")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count() or 1,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def moe_oracle_rows(xb, q_w, s_w, off, rows):
+    """Oracle result of the sampled rows of one grouped linear: the oracle
+    quantizes those rows of X itself; the weights are the GPU's codes (held
+    bit-exact to the oracle by the tests).  Returns (seconds, flops, R)."""
+    import oracle
+    t0 = time.perf_counter()
+    per_row = [oracle.quant_act_ue8m0_rows(xb, int(r), int(r) + 1) for r in rows]
+    M = xb.shape[0]
+    qa = np.zeros((M, xb.shape[1]), np.uint8)
+    ca = np.full((M, xb.shape[1] // 128), 127, np.uint8)
+    for r, (q, c) in zip(rows, per_row):
+        qa[r], ca[r] = q[0], c[0]
+    R = oracle.grouped_linear_ue8m0(qa, ca, q_w, s_w, off, rows=rows, nthreads=os.cpu_count() or 1)
+    t = time.perf_counter() - t0
+    return t, 2.0 * len(rows) * q_w.shape[1] * q_w.shape[2], R[rows]
+
+
+def run_moe(args):
+    """Grouped (MoE expert) UE8M0 linears: one step = per expert linear (up,
+    down), ue8m0 activation quantization of the routed rows + the grouped
+    GEMM over the experts' segments."""
+    import torch
+    import torch.distributed as dist
+
+    import fine_grained_block_token_b200 as fp8
+
+    world, rank, local = rank_info()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    hbm_peak, bf16_peak, peak_src = peaks()
+    fp8_peak = bf16_peak * FP8_OVER_BF16
+    items = []
+    for name in ("up", "down"):
+        xb, off = wl.deepseek_moe(name)
+        N, K = wl.MOE_LINEARS[name]
+        E = wl.MOE_EXPERTS
+        w = wl.deepseek_moe_weights(name, dev)
+        q_w, s_w = fp8.quant_weight_ue8m0(w)
+        del w
+        M = xb.shape[0]
+        items.append(dict(label=name, xb=xb, x=wl.to_torch_bf16(xb).to(dev), off_np=off,
+                          off=torch.from_numpy(off).to(dev), q_w=q_w.view(E, N, K),
+                          s_w=s_w.view(E, N // 128, K // 128),
+                          q_a=torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev),
+                          s_a=torch.empty((M, K // 128), dtype=torch.float8_e8m0fnu, device=dev),
+                          y=torch.empty((M, N), dtype=torch.bfloat16, device=dev), M=M, N=N, K=K))
+    torch.cuda.synchronize()
+    flops_step = sum(2 * it["M"] * it["N"] * it["K"] for it in items)
+    n = len(items)
+
+    def step(ev=None):
+        for i, it in enumerate(items):
+            fp8.quant_act_ue8m0(it["x"], it["q_a"], it["s_a"])
+            if ev is not None:
+                ev[2 * i].record()
+            fp8.grouped_linear_ue8m0(it["q_a"], it["s_a"], it["q_w"], it["s_w"], it["off"], it["y"])
+            if ev is not None:
+                ev[2 * i + 1].record()
+
+    for _ in range(args.warmup):
+        step()
+    fp8.check()
+    graph = None
+    if not args.eager:
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize(dev)
+    run_step = (lambda: graph.replay()) if graph is not None else step
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    a.record()
+    for _ in range(args.steps):
+        run_step()
+    b.record()
+    barrier()
+    elapsed_ms = a.elapsed_time(b)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(args.steps)]
+    barrier()
+    for k in range(args.steps):
+        step(evs[k])
+    barrier()
+    gemm_ms = sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs for i in range(n))
+    fp8.check()
+    # end to end: X in from pinned host memory, Y back, every step
+    host_x = [wl.to_torch_bf16(it["xb"]).pin_memory() for it in items]
+    host_y = [torch.empty((it["M"], it["N"]), dtype=torch.bfloat16).pin_memory() for it in items]
+
+    def e2e_step():
+        for it, hx, hy in zip(items, host_x, host_y):
+            it["x"].copy_(hx, non_blocking=True)
+            fp8.quant_act_ue8m0(it["x"], it["q_a"], it["s_a"])
+            fp8.grouped_linear_ue8m0(it["q_a"], it["s_a"], it["q_w"], it["s_w"], it["off"], it["y"])
+            hy.copy_(it["y"], non_blocking=True)
+
+    for _ in range(min(args.warmup, 3)):
+        e2e_step()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    barrier()
+    a.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record()
+    barrier()
+    e2e_ms = a.elapsed_time(b)
+    sampler.stop()
+    fp8.check()
+    elapsed_ms, gemm_ms, e2e_ms = max_over_ranks([elapsed_ms, gemm_ms, e2e_ms], dev, world)
+    gemm_tf = flops_step * args.steps / (gemm_ms * 1e-3) / 1e12
+    if rank == 0:
+        cpu = parity = None
+        if world == 1 and not args.no_cpu:
+            t_tot, f_tot, worst = 0.0, 0.0, 0.0
+            g = np.random.default_rng(0)
+            for it in items:
+                rows = np.sort(g.choice(it["M"], args.cpu_rows, replace=False))
+                qw = it["q_w"].view(torch.uint8).cpu().numpy()
+                sw = it["s_w"].view(torch.uint8).cpu().numpy()
+                t, f, R = moe_oracle_rows(it["xb"], qw, sw, it["off_np"], rows)
+                t_tot += t
+                f_tot += f
+                Y = it["y"][torch.as_tensor(rows, device=dev)].float().cpu().numpy()
+                worst = max(worst, within_tolerance(Y, R))
+            cpu = {"value": f_tot / t_tot / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count() or 1,
+                   "kind": "oracle", "seconds": t_tot,
+                   "sample": f"{args.cpu_rows} random routed rows per expert linear (up, down): "
+                             "ue8m0 activation quant + fp64 grouped GEMM of those rows, all N columns"}
+            parity = {"rows_per_linear": args.cpu_rows, "within_tolerance": worst <= 1.0,
+                      "worst_bound_ratio": worst}
+        line = {
+            "metric": METRIC, "value": whole_job_rate(world, flops_step, args.steps, elapsed_ms) / 1e12,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3 (ue8m0 scales)", "data": "synthetic",
+            "config": {"workload": "deepseek_moe", "experts": wl.MOE_EXPERTS, "routed_rows": wl.MOE_ROWS,
+                       "linears": {it["label"]: [it["M"], it["N"], it["K"]] for it in items},
+                       "segment_rows": {it["label"]: np.diff(it["off_np"]).tolist() for it in items},
+                       "l2": "no flush: the step's expert weights (470 + 235 MB) exceed the 126 MB L2",
+                       "parallelism": f"replicas x{world} (no data-path collective)",
+                       "launch": "eager" if args.eager else "cuda_graph (one step captured, replayed)"},
+            "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": gemm_tf / fp8_peak,
+                         "traffic": recorded_traffic("gemm_ue8m0_kernel", "deepseek_moe"),
+                         "kernel": "gemm_ue8m0_kernel (grouped)",
+                         "peak_source": f"{peak_src} bf16 burst x {FP8_OVER_BF16} (nominal fp8/bf16)",
+                         "ms_per_launch": gemm_ms / (args.steps * n)},
+            "e2e": {"value": whole_job_rate(world, flops_step, e2e_steps, e2e_ms) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": sum(t.numel() * 2 for t in host_x),
+                    "d2h_bytes_per_step": sum(t.numel() * 2 for t in host_y), "steps": e2e_steps},
+            "gpu_launches": 2 * n * args.steps,
+            "clocks": sampler.summary(),
+            "cpu_baseline": cpu,
+            "parity": parity,
+        }
+        print(json.dumps(line))
+    del graph
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
     return 0
 
 
@@ -639,7 +877,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama3_prefill",
-                    choices=["llama3_prefill", "deepseek_mlp", "llama3_decode", "sweep"])
+                    choices=["llama3_prefill", "deepseek_mlp", "llama3_decode", "sweep", "deepseek_moe"])
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-rows", type=int, default=32)
     ap.add_argument("--ref-rows", type=int, default=4)
@@ -651,6 +889,8 @@ def main():
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "deepseek_moe":
+        return run_moe(args)
     return run_ours(args)
 
 

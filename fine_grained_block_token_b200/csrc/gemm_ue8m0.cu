@@ -45,9 +45,10 @@
 // expert e's weights W[e] ([E, N, K] stacked, scales [E, N/128, K/128]).
 // Warp 3 turns the offsets into a shared-memory table at start-up (clamped
 // to [0, M] and made non-decreasing, so any offsets stay in bounds) with
-// each expert's count of 128-row blocks; tiles run over all experts' blocks
-// (M-fastest) times the N tiles, and a tile's rows past its segment, like
-// its columns past N, are computed on whatever TMA loads but never stored.
+// each expert's count of 128-row blocks; tiles run expert by expert (each
+// expert's blocks times the N tiles, M-fastest), and a tile's rows past its
+// segment, like its columns past N, are computed on whatever TMA loads but
+// never stored.
 // The plain linear is the case E = 1, off = {0, M}.
 // Every mbarrier wait is bounded in time; on expiry the kernel records an
 // error code in the error word, drains what it started and exits cleanly.
@@ -187,17 +188,21 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
   const int total_m = tab_pre[E];
   const int num_tiles = total_m * num_n;
-  // tile -> (expert, first row, end of the expert's rows, N tile)
+  // tile -> (expert, first row, end of the expert's rows, N tile).  Tiles
+  // are expert-major (all of expert e's tiles, M-fastest, before expert
+  // e + 1), so an expert's rows of A and its weights are reused from L2
+  // while its tiles run; with one expert this is the plain M-fastest order.
   auto map_tile = [&](int tile, int& e, int& row0, int& row_end, int& n_blk) {
-    const int mb = tile % total_m;
-    n_blk = tile / total_m;
-    int lo = 0, hi = E - 1;          // the last expert whose first block is <= mb
+    int lo = 0, hi = E - 1;          // the last expert whose first tile is <= tile
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (tab_pre[mid] <= mb) lo = mid; else hi = mid - 1;
+      if (tab_pre[mid] * num_n <= tile) lo = mid; else hi = mid - 1;
     }
-    e = lo;
-    row0 = tab_off[e] + (mb - tab_pre[e]) * BM;
+    e = lo;                          // has at least one block (else e + 1 would match)
+    const int local = tile - tab_pre[e] * num_n;
+    const int blocks = tab_pre[e + 1] - tab_pre[e];
+    n_blk = local / blocks;
+    row0 = tab_off[e] + (local % blocks) * BM;
     row_end = tab_off[e + 1];
   };
 

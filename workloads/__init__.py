@@ -18,6 +18,13 @@ Workloads (shapes as N x K for weights, M x K for activations):
   sweep          X [M, 7168], M in {512, 1024, ..., 16384}, Student-t(df=3),
                  0.1% of channels scaled by 100, 1% of the 1x128 groups all
                  zero; W [2048, 7168] ~ N(0, 0.02).
+  deepseek_moe   16 experts of the DeepSeek-V3 expert MLP shape: up (gate
+                 and up fused) 4096x7168, down 7168x2048, stacked [E, N, K];
+                 8192 routed token rows sorted by expert, segment sizes a
+                 multinomial draw with Dirichlet(1) expert shares (uneven,
+                 some small); X ~ N(0,1) times a per-row LogNormal(0,1);
+                 W ~ N(0, 0.015), drawn on the GPU by torch's seeded
+                 generator (deepseek_moe_weights).
 
 Seeds: X draws use seed 0, W draws seed 1, the selection of outlier
 channels / zeroed blocks / zeroed groups seed 2 (one generator per role, so
@@ -45,15 +52,19 @@ DEEPSEEK_LINEARS = {"up": (18432, 7168), "down": (7168, 18432)}
 SWEEP_K = 7168
 SWEEP_N = 2048
 SWEEP_M = (512, 1024, 2048, 4096, 8192, 16384)
+MOE_EXPERTS = 16
+MOE_ROWS = 8192
+MOE_LINEARS = {"up": (4096, 7168), "down": (7168, 2048)}
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round fp32 to bf16 (nearest, ties to even) and return the bit patterns."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
+    u = x.view(np.uint32)
     nan = np.isnan(x)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    # u + 0x7FFF + lsb stays below 2^32 for every non-NaN pattern (at most
+    # 0xFF807FFF), so 32-bit arithmetic rounds exactly; NaNs are set below.
+    r = ((u + np.uint32(0x7FFF) + ((u >> 16) & np.uint32(1))) >> 16).astype(np.uint16)
     if nan.any():
         r[nan] = 0x7FC0
     return r
@@ -133,6 +144,39 @@ def deepseek_mlp(name: str, M: int = DEEPSEEK_M):
     x *= g.lognormal(0.0, 1.0, size=(M, 1)).astype(np.float32)
     w = normal((N, K), 0.015, SEED_W, salt)
     return f32_to_bf16_bits(x), zero_blocks(w, 0.01, salt)
+
+
+def moe_offsets(E: int = MOE_EXPERTS, M: int = MOE_ROWS) -> np.ndarray:
+    """int32 [E + 1] segment starts of M routed rows over E experts."""
+    g = _rng(SEED_SEL, 3001)
+    counts = g.multinomial(M, g.dirichlet(np.ones(E)))
+    return np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+
+
+def deepseek_moe(name: str, E: int = MOE_EXPERTS, M: int = MOE_ROWS):
+    """(X bits [M, K], offsets int32 [E + 1]) for the expert linear `name`;
+    the weights come from deepseek_moe_weights."""
+    N, K = MOE_LINEARS[name]
+    g = _rng(SEED_X, hash_name("moe_" + name))
+    x = g.standard_normal((M, K), dtype=np.float32)
+    x *= g.lognormal(0.0, 1.0, size=(M, 1)).astype(np.float32)
+    return f32_to_bf16_bits(x), moe_offsets(E, M)
+
+
+def deepseek_moe_weights(name: str, device, E: int = MOE_EXPERTS):
+    """Stacked expert weights [E * N, K] (expert e = rows e N .. e N + N - 1),
+    N(0, 0.015) in bf16, drawn on `device` by torch's generator seeded with
+    (SEED_W, salt): hundreds of millions of draws, which numpy on the host
+    would take tens of seconds for."""
+    import torch
+    N, K = MOE_LINEARS[name]
+    g = torch.Generator(device=device)
+    g.manual_seed(SEED_W * 1_000_003 + hash_name("moe_" + name))
+    w = torch.empty((E * N, K), dtype=torch.bfloat16, device=device)
+    for e in range(E):
+        w[e * N:(e + 1) * N] = (torch.randn((N, K), generator=g, device=device, dtype=torch.float32)
+                                * 0.015).to(torch.bfloat16)
+    return w
 
 
 def sweep_x(M: int, K: int = SWEEP_K):
