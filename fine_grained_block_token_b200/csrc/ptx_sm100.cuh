@@ -337,6 +337,116 @@ __device__ __forceinline__ void bulk_copy_s2s(uint32_t dst, uint32_t src, uint32
       : "memory");
 }
 
+// ------------------------------------------- CTA pairs (cta_group::2)
+//
+// Two CTAs of a cluster (ranks 2p, 2p + 1) act as one MMA unit: the even
+// one issues tcgen05.mma.cta_group::2 with M = 256, reading A rows
+// 0..127 and B rows 0..N/2-1 from its own shared memory and the rest from
+// its peer's at the same offsets, and writing accumulator rows 0..127 into
+// its own TMEM and 128..255 into the peer's.
+
+// Bounded waits with cluster-scope acquire, for barriers that another CTA
+// of the cluster arrives on.  Same bound and return value as mbar_wait.
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_spin_cluster(uint32_t bar, uint32_t parity,
+                                                       uint64_t limit_cycles = 1ull << 32) {
+  if (mbar_test_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_test_wait_cluster(bar, parity)) return true;
+    if ((i & 255u) == 0 && clock64() - t0 > limit_cycles) return false;
+  }
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_cycles = 1ull << 32) {
+#pragma unroll 1
+  for (int i = 0; i < 64; ++i)
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((i & 63u) == 0 && clock64() - t0 > limit_cycles) return false;
+  }
+}
+
+// Arrive once, with cluster-scope release, on the mbarrier at the
+// shared::cluster address `remote_bar` (from map_to_cta).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
+               : "memory");
+}
+
+// TMEM allocation for a CTA pair: the same warp of both CTAs executes it,
+// with the same destination offset.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// D (+)= A * B^T for the CTA pair, e4m3 x e4m3 -> fp32, issued by the even
+// CTA; no output lanes disabled.
+__device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z)
+      : "memory");
+}
+
+// Arrive once on the mbarrier at shared offset `bar` of every CTA in
+// `cta_mask` when all previously issued pair MMAs of this thread completed.
+__device__ __forceinline__ void mma_commit_pair_multicast(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(cta_mask)
+      : "memory");
+}
+
+// 2-D tiled load into this CTA's shared memory whose completion (in bytes)
+// is counted on the pair's even CTA's mbarrier (`bar` = shared::cluster
+// address of that barrier).  Not a multicast load.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m, uint32_t bar,
+                                                 int32_t c0, int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
 // Arrive (once) on the mbarrier at shared offset `bar` in every CTA of
 // `cta_mask` when all previously issued MMAs of this thread have completed.
 __device__ __forceinline__ void mma_commit_multicast(uint32_t bar, uint16_t cta_mask) {
