@@ -84,6 +84,7 @@ KERNEL_SOURCES = {
     "gemm_prefill_kernel": ("gemm.cu", "ptx_sm100.cuh", "quant_math.cuh"),
     "gemm_ue8m0_kernel": ("gemm_ue8m0.cu", "ptx_sm100.cuh"),
     "gemm_rowwise_kernel": ("gemm_rowwise.cu", "ptx_sm100.cuh"),
+    "gemm_rowwise_pair_kernel": ("gemm_rowwise.cu", "ptx_sm100.cuh"),
 }
 
 
@@ -722,7 +723,9 @@ def run_ours(args):
                           s_a=lambda it: torch.empty((it["M"], it["K"] // 128),
                                                      dtype=torch.float8_e8m0fnu, device=dev)),
             "fp8r": dict(wq=fp8.quant_rowwise, aq=fp8.quant_rowwise,
-                         gemm=fp8.linear_rowwise, kernel="gemm_rowwise_kernel",
+                         gemm=fp8.linear_rowwise,
+                         # CTA pairs above one 128-row tile (the prefill workloads)
+                         kernel="gemm_rowwise_pair_kernel",
                          s_a=lambda it: torch.empty((it["M"],), dtype=torch.float32, device=dev)),
         }
         for name, sp in specs.items():
