@@ -118,3 +118,21 @@ def test_full_size_prefill(fp8, which):
 
 def test_no_timeout_recorded(fp8):
     fp8.check()
+
+
+@pytest.mark.parametrize("M,N,K", [(129, 512, 1024), (255, 256, 2048), (256, 768, 512), (257, 256, 384),
+                                   (4096, 2048, 4096)])
+def test_pair_boundaries_and_repeated_runs(fp8, M, N, K):
+    """M around the CTA-pair tile (256 rows: the odd CTA with no rows, a
+    partial tile, several tiles): parity, then five more runs bit-identical
+    (a hand-off race between the two CTAs would show up as differing runs)."""
+    xb = wl.normal((M, K), 1.0, 0, 7 * M + N + K)
+    wb = wl.normal((N, K), 0.02, 1, 7 * M + N + K)
+    rows = None if M <= 300 else np.array([0, 1, 127, 128, 255, 256, 2047, 4095])
+    y, R, (q_a, s_a, q_w, s_w, y0) = _run(fp8, xb, wb, rows=rows)
+    check_gemm(y, R, f"{M}x{N}x{K}")
+    for _ in range(5):
+        y1 = fp8.linear_rowwise(q_a, s_a, q_w, s_w)
+        torch.cuda.synchronize()
+        assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+    fp8.check()
