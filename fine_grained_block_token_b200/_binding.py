@@ -91,17 +91,74 @@ def _u8(t: torch.Tensor) -> torch.Tensor:
     return t.view(torch.uint8) if t.dtype != torch.uint8 else t
 
 
+# The C ABI takes raw pointers and sizes and cannot see strides, devices or
+# dtypes, so every tensor is checked here before its pointer is passed: on
+# the CUDA device of the call's first input, dense (contiguous), of the
+# expected dtype and shape.  Violations raise before anything is enqueued.
+_CODES = (torch.float8_e4m3fn, torch.uint8)          # e4m3 codes, or their bytes
+_E8M0 = (torch.float8_e8m0fnu, torch.uint8)          # ue8m0 scale codes, or their bytes
+_F32 = (torch.float32,)
+_BF16 = (torch.bfloat16,)
+
+
+def _device_of(t, name: str):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device (got {t.device})")
+    return t.device
+
+
+def _need(t, name: str, dtypes, shape, device) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {' or '.join(map(str, dtypes))}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check_linear(q_a, s_a, q_w, s_w, y):
+    """Checks the operands of the fp32-scale linear; returns (M, N, K)."""
+    dev = _device_of(q_a, "q_a")
+    M, K = _dims2(q_a, "q_a")
+    N = _dims2(q_w, "q_w")[0]
+    _need(q_a, "q_a", _CODES, (M, K), dev)
+    _need(s_a, "s_a", _F32, (M, K // BLOCK), dev)
+    _need(q_w, "q_w", _CODES, (N, K), dev)
+    _need(s_w, "s_w", _F32, (N // BLOCK, K // BLOCK), dev)
+    if y is not None:
+        _need(y, "y", _BF16, (M, N), dev)
+    return M, N, K
+
+
+def _dims2(t, name: str):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
+    return t.shape
+
+
 def version() -> int:
     return _lib.fp8bl_version()
 
 
 def quant_act(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None):
     """bf16 [M, K] -> (e4m3 [M, K], fp32 [M, K/128]).  Outputs may be given."""
-    M, K = x.shape
+    dev = _device_of(x, "x")
+    M, K = _dims2(x, "x")
+    _need(x, "x", _BF16, (M, K), dev)
     if q is None:
         q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
     if s is None:
-        s = torch.empty((M, K // BLOCK if K % BLOCK == 0 else 0), dtype=torch.float32, device=x.device)
+        s = torch.empty((M, K // BLOCK), dtype=torch.float32, device=x.device)
+    _need(q, "q", _CODES, (M, K), dev)
+    _need(s, "s", _F32, (M, K // BLOCK), dev)
     _ok(_lib.fp8_quant_act(_ptr(x), M, K, _ptr(q), _ptr(s), _stream(x)), "fp8_quant_act")
     return q, s
 
@@ -111,13 +168,18 @@ def quant_act_static(x: torch.Tensor, s_given: torch.Tensor, q: torch.Tensor | N
     """Static scheme: bf16 [M, K] with one given fp32 scale (a 1-element device
     tensor) -> (e4m3 [M, K], fp32 [M, K/128] filled with that scale), ready
     for block_linear."""
-    M, K = x.shape
-    if s_given.numel() != 1 or s_given.dtype != torch.float32:
-        raise ValueError("s_given must be one fp32 element")
+    dev = _device_of(x, "x")
+    M, K = _dims2(x, "x")
+    _need(x, "x", _BF16, (M, K), dev)
+    if not isinstance(s_given, torch.Tensor) or s_given.numel() != 1:
+        raise ValueError("s_given must be a one-element fp32 tensor")
+    _need(s_given, "s_given", _F32, None, dev)
     if q is None:
         q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
     if s is None:
-        s = torch.empty((M, K // BLOCK if K % BLOCK == 0 else 0), dtype=torch.float32, device=x.device)
+        s = torch.empty((M, K // BLOCK), dtype=torch.float32, device=x.device)
+    _need(q, "q", _CODES, (M, K), dev)
+    _need(s, "s", _F32, (M, K // BLOCK), dev)
     _ok(_lib.fp8_quant_act_static(_ptr(x), M, K, _ptr(s_given), _ptr(q), _ptr(s), _stream(x)),
         "fp8_quant_act_static")
     return q, s
@@ -125,11 +187,15 @@ def quant_act_static(x: torch.Tensor, s_given: torch.Tensor, q: torch.Tensor | N
 
 def quant_weight(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None):
     """bf16 [N, K] -> (e4m3 [N, K], fp32 [N/128, K/128])."""
-    N, K = w.shape
+    dev = _device_of(w, "w")
+    N, K = _dims2(w, "w")
+    _need(w, "w", _BF16, (N, K), dev)
     if q is None:
         q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
     if s is None:
         s = torch.empty((N // BLOCK, K // BLOCK), dtype=torch.float32, device=w.device)
+    _need(q, "q", _CODES, (N, K), dev)
+    _need(s, "s", _F32, (N // BLOCK, K // BLOCK), dev)
     _ok(_lib.fp8_quant_weight(_ptr(w), N, K, _ptr(q), _ptr(s), _stream(w)), "fp8_quant_weight")
     return q, s
 
@@ -142,12 +208,15 @@ def quant_weight(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor
 def quant_act_ue8m0(x: torch.Tensor, q: torch.Tensor | None = None,
                     s: torch.Tensor | None = None):
     """bf16 [M, K] -> (e4m3 [M, K], float8_e8m0fnu [M, K/128])."""
-    M, K = x.shape
+    dev = _device_of(x, "x")
+    M, K = _dims2(x, "x")
+    _need(x, "x", _BF16, (M, K), dev)
     if q is None:
         q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
     if s is None:
-        s = torch.empty((M, K // BLOCK if K % BLOCK == 0 else 0), dtype=torch.float8_e8m0fnu,
-                        device=x.device)
+        s = torch.empty((M, K // BLOCK), dtype=torch.float8_e8m0fnu, device=x.device)
+    _need(q, "q", _CODES, (M, K), dev)
+    _need(s, "s", _E8M0, (M, K // BLOCK), dev)
     _ok(_lib.fp8_quant_act_ue8m0(_ptr(x), M, K, _ptr(q), _ptr(s), _stream(x)),
         "fp8_quant_act_ue8m0")
     return q, s
@@ -156,11 +225,15 @@ def quant_act_ue8m0(x: torch.Tensor, q: torch.Tensor | None = None,
 def quant_weight_ue8m0(w: torch.Tensor, q: torch.Tensor | None = None,
                        s: torch.Tensor | None = None):
     """bf16 [N, K] -> (e4m3 [N, K], float8_e8m0fnu [N/128, K/128])."""
-    N, K = w.shape
+    dev = _device_of(w, "w")
+    N, K = _dims2(w, "w")
+    _need(w, "w", _BF16, (N, K), dev)
     if q is None:
         q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
     if s is None:
         s = torch.empty((N // BLOCK, K // BLOCK), dtype=torch.float8_e8m0fnu, device=w.device)
+    _need(q, "q", _CODES, (N, K), dev)
+    _need(s, "s", _E8M0, (N // BLOCK, K // BLOCK), dev)
     _ok(_lib.fp8_quant_weight_ue8m0(_ptr(w), N, K, _ptr(q), _ptr(s), _stream(w)),
         "fp8_quant_weight_ue8m0")
     return q, s
@@ -169,12 +242,16 @@ def quant_weight_ue8m0(w: torch.Tensor, q: torch.Tensor | None = None,
 def block_linear_ue8m0(q_a, s_a, q_w, s_w, y=None) -> torch.Tensor:
     """(e4m3 [M,K], e8m0 [M,K/128], e4m3 [N,K], e8m0 [N/128,K/128]) -> bf16 [M,N],
     on the tensor core's block-scaled MMA."""
-    M, K = q_a.shape
-    N = q_w.shape[0]
-    if q_w.shape[1] != K:
-        raise ValueError("q_a and q_w disagree on K")
+    dev = _device_of(q_a, "q_a")
+    M, K = _dims2(q_a, "q_a")
+    N = _dims2(q_w, "q_w")[0]
+    _need(q_a, "q_a", _CODES, (M, K), dev)
+    _need(s_a, "s_a", _E8M0, (M, K // BLOCK), dev)
+    _need(q_w, "q_w", _CODES, (N, K), dev)
+    _need(s_w, "s_w", _E8M0, (N // BLOCK, K // BLOCK), dev)
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
+    _need(y, "y", _BF16, (M, N), dev)
     _ok(_lib.fp8_block_linear_ue8m0(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
                                     _stream(q_a)), "fp8_block_linear_ue8m0")
     return y
@@ -184,14 +261,19 @@ def grouped_linear_ue8m0(q_a, s_a, q_w, s_w, expert_offsets, y=None) -> torch.Te
     """Grouped (MoE expert) UE8M0 linear: rows [off[e], off[e+1]) of
     (e4m3 [M,K], e8m0 [M,K/128]) times expert e of (e4m3 [E,N,K],
     e8m0 [E,N/128,K/128]); expert_offsets int32 [E+1] on the device."""
-    M, K = q_a.shape
-    E, N, Kw = q_w.shape
-    if Kw != K:
-        raise ValueError("q_a and q_w disagree on K")
-    if expert_offsets.dtype != torch.int32 or expert_offsets.numel() != E + 1:
-        raise ValueError("expert_offsets must be int32 [E + 1]")
+    dev = _device_of(q_a, "q_a")
+    M, K = _dims2(q_a, "q_a")
+    if q_w.dim() != 3:
+        raise ValueError(f"q_w must be 3-D [E, N, K], got shape {tuple(q_w.shape)}")
+    E, N, _ = q_w.shape
+    _need(q_a, "q_a", _CODES, (M, K), dev)
+    _need(s_a, "s_a", _E8M0, (M, K // BLOCK), dev)
+    _need(q_w, "q_w", _CODES, (E, N, K), dev)
+    _need(s_w, "s_w", _E8M0, (E, N // BLOCK, K // BLOCK), dev)
+    _need(expert_offsets, "expert_offsets", (torch.int32,), (E + 1,), dev)
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
+    _need(y, "y", _BF16, (M, N), dev)
     _ok(_lib.fp8_grouped_linear_ue8m0(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w),
                                       _ptr(expert_offsets), _ptr(y), M, N, K, E, _stream(q_a)),
         "fp8_grouped_linear_ue8m0")
@@ -204,23 +286,31 @@ def grouped_linear_ue8m0(q_a, s_a, q_w, s_w, expert_offsets, y=None) -> torch.Te
 
 def quant_rowwise(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None):
     """bf16 [R, K] -> (e4m3 [R, K], fp32 [R]); K % 16 == 0."""
-    R, K = x.shape
+    dev = _device_of(x, "x")
+    R, K = _dims2(x, "x")
+    _need(x, "x", _BF16, (R, K), dev)
     if q is None:
         q = torch.empty((R, K), dtype=torch.float8_e4m3fn, device=x.device)
     if s is None:
         s = torch.empty((R,), dtype=torch.float32, device=x.device)
+    _need(q, "q", _CODES, (R, K), dev)
+    _need(s, "s", _F32, (R,), dev)
     _ok(_lib.fp8_quant_rowwise(_ptr(x), R, K, _ptr(q), _ptr(s), _stream(x)), "fp8_quant_rowwise")
     return q, s
 
 
 def linear_rowwise(q_a, s_a, q_w, s_w, y=None) -> torch.Tensor:
     """(e4m3 [M,K], fp32 [M], e4m3 [N,K], fp32 [N]) -> bf16 [M,N]."""
-    M, K = q_a.shape
-    N = q_w.shape[0]
-    if q_w.shape[1] != K:
-        raise ValueError("q_a and q_w disagree on K")
+    dev = _device_of(q_a, "q_a")
+    M, K = _dims2(q_a, "q_a")
+    N = _dims2(q_w, "q_w")[0]
+    _need(q_a, "q_a", _CODES, (M, K), dev)
+    _need(s_a, "s_a", _F32, (M,), dev)
+    _need(q_w, "q_w", _CODES, (N, K), dev)
+    _need(s_w, "s_w", _F32, (N,), dev)
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
+    _need(y, "y", _BF16, (M, N), dev)
     _ok(_lib.fp8_linear_rowwise(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
                                 _stream(q_a)), "fp8_linear_rowwise")
     return y
@@ -235,6 +325,8 @@ def fused_workspace_bytes(M: int, N: int, K: int) -> int:
 
 
 def _workspace(nbytes: int, device, given):
+    if given is not None:
+        _need(given, "workspace", (torch.uint8,), None, device)
     if nbytes == 0:
         return given, 0 if given is None else given.numel() * given.element_size()
     if given is None:
@@ -244,10 +336,7 @@ def _workspace(nbytes: int, device, given):
 
 def block_linear(q_a, s_a, q_w, s_w, y=None, workspace=None) -> torch.Tensor:
     """(e4m3 [M,K], fp32 [M,K/128], e4m3 [N,K], fp32 [N/128,K/128]) -> bf16 [M,N]."""
-    M, K = q_a.shape
-    N = q_w.shape[0]
-    if q_w.shape[1] != K:
-        raise ValueError("q_a and q_w disagree on K")
+    M, N, K = _check_linear(q_a, s_a, q_w, s_w, y)
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
     ws, wsb = _workspace(workspace_bytes(M, N, K), q_a.device, workspace)
@@ -259,10 +348,14 @@ def block_linear(q_a, s_a, q_w, s_w, y=None, workspace=None) -> torch.Tensor:
 def block_linear_fused(x, q_w, s_w, y=None, workspace=None) -> torch.Tensor:
     """bf16 x [M,K] with quantized weights -> bf16 [M,N]; the activation
     quantization happens inside the GEMM, bit-identical to quant_act."""
-    M, K = x.shape
-    N = q_w.shape[0]
-    if q_w.shape[1] != K:
-        raise ValueError("x and q_w disagree on K")
+    dev = _device_of(x, "x")
+    M, K = _dims2(x, "x")
+    N = _dims2(q_w, "q_w")[0]
+    _need(x, "x", _BF16, (M, K), dev)
+    _need(q_w, "q_w", _CODES, (N, K), dev)
+    _need(s_w, "s_w", _F32, (N // BLOCK, K // BLOCK), dev)
+    if y is not None:
+        _need(y, "y", _BF16, (M, N), dev)
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     ws, wsb = _workspace(fused_workspace_bytes(M, N, K), x.device, workspace)
@@ -276,10 +369,9 @@ def block_linear_noalloc(q_a, s_a, q_w, s_w, y) -> torch.Tensor:
     no workspace, and nothing is allocated here or in the library, so the
     output tensor ``y`` (bf16 [M, N]) must be given.  For callers that cannot
     allocate device memory where they run the layer."""
-    M, K = q_a.shape
-    N = q_w.shape[0]
-    if q_w.shape[1] != K:
-        raise ValueError("q_a and q_w disagree on K")
+    if y is None:
+        raise ValueError("block_linear_noalloc needs the output tensor y")
+    M, N, K = _check_linear(q_a, s_a, q_w, s_w, y)
     _ok(_lib.fp8_block_linear_noalloc(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
                                       _stream(q_a)), "fp8_block_linear_noalloc")
     return y
