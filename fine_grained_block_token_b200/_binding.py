@@ -93,8 +93,9 @@ def _u8(t: torch.Tensor) -> torch.Tensor:
 
 # The C ABI takes raw pointers and sizes and cannot see strides, devices or
 # dtypes, so every tensor is checked here before its pointer is passed: on
-# the CUDA device of the call's first input, dense (contiguous), of the
-# expected dtype and shape.  Violations raise before anything is enqueued.
+# the current CUDA device (that of the call's first input), dense
+# (contiguous), of the expected dtype and shape.  Violations raise before
+# anything is enqueued.
 _CODES = (torch.float8_e4m3fn, torch.uint8)          # e4m3 codes, or their bytes
 _E8M0 = (torch.float8_e8m0fnu, torch.uint8)          # ue8m0 scale codes, or their bytes
 _F32 = (torch.float32,)
@@ -106,6 +107,12 @@ def _device_of(t, name: str):
         raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise ValueError(f"{name} must be on a CUDA device (got {t.device})")
+    # the library launches on the current device: a tensor elsewhere would
+    # hand another device's pointers to its kernels
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{name} is on {t.device} but the current device is cuda:{cur}; "
+                         f"call under `with torch.cuda.device({t.device.index}):`")
     return t.device
 
 
