@@ -210,3 +210,47 @@ def test_selftest_wait_timeout_rejects_bad_arguments(lib):
     assert f((1 << 32) + 1, 0, None) == 2
     assert f(1000, 2, None) == 2
     assert f(1000, -1, None) == 2
+
+
+def _decode_slots_needed(N, K, G):
+    """Brute force over the stream-K partition of the decode schedule: CTA g
+    streams units [g*U/G, (g+1)*U/G) of the flattened (weight block, K chunk)
+    space (U = N/128 * K/128) and stores one partial per block it touches,
+    in slot (block - first block of its range).  Returns the largest number
+    of slots any CTA uses."""
+    KB = K // 128
+    U = (N // 128) * KB
+    most = 0
+    for g in range(G):
+        lo, hi = g * U // G, (g + 1) * U // G
+        if hi > lo:
+            most = max(most, (hi - 1) // KB - lo // KB + 1)
+    return most
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_decode_workspace_covers_every_partial_slot(lib, seed):
+    """The workspace the library asks for must hold the per-block counters
+    plus, for each of the G CTAs, a partial [Mpad, 128] fp32 for every block
+    its range touches; a smaller stride would let a CTA write past its
+    slots (and the last CTA past the buffer).  Without a GPU the library
+    plans for 148 SMs; G = min(148, U / ceil(KB / 8)) CTAs."""
+    import numpy as np
+    f = lib.fp8_block_linear_workspace_bytes
+    f.argtypes = [ctypes.c_int64] * 3
+    f.restype = ctypes.c_size_t
+    g = np.random.default_rng(seed)
+    shapes = [(1, 128, 128), (64, 128, 128), (1, 256, 32768), (17, 28672, 4096), (64, 4096, 14336),
+              (8, 1024, 4096), (33, 128, 1024 * 128)]
+    shapes += [(int(g.integers(1, 65)), 128 * int(g.integers(1, 300)), 128 * int(g.integers(1, 200)))
+               for _ in range(40)]
+    for M, N, K in shapes:
+        KB, U = K // 128, (N // 128) * (K // 128)
+        G = max(1, min(148, U // ((KB + 7) // 8)))
+        mpad = (M + 15) // 16 * 16
+        counters = ((N // 128) * 4 + 255) // 256 * 256
+        ws = f(M, N, K)
+        per_slot = G * mpad * 128 * 4
+        assert ws > counters and (ws - counters) % per_slot == 0, (M, N, K, ws)
+        assert (ws - counters) // per_slot >= _decode_slots_needed(N, K, G), (M, N, K)
+    assert f(65, 4096, 4096) == 0          # prefill sizes need no workspace
