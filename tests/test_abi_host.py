@@ -254,3 +254,20 @@ def test_decode_workspace_covers_every_partial_slot(lib, seed):
         assert ws > counters and (ws - counters) % per_slot == 0, (M, N, K, ws)
         assert (ws - counters) // per_slot >= _decode_slots_needed(N, K, G), (M, N, K)
     assert f(65, 4096, 4096) == 0          # prefill sizes need no workspace
+
+
+def test_fused_workspace_holds_the_staged_activations(lib):
+    """At decode sizes the fused entry point quantizes into its workspace
+    (codes M*K bytes, then scales M*K/128 fp32, each 256-byte aligned) after
+    the decode schedule's own scratch; at prefill sizes it needs none."""
+    ws = lib.fp8_block_linear_workspace_bytes
+    fw = lib.fp8_block_linear_fused_workspace_bytes
+    for f in (ws, fw):
+        f.argtypes = [ctypes.c_int64] * 3
+        f.restype = ctypes.c_size_t
+    up = lambda v: (v + 255) // 256 * 256
+    for M, N, K in [(1, 128, 128), (7, 4096, 4096), (64, 28672, 4096), (33, 4096, 14336),
+                    (64, 128, 1024 * 128)]:
+        assert fw(M, N, K) >= up(ws(M, N, K)) + up(M * K) + up(M * (K // 128) * 4), (M, N, K)
+    for M, N, K in [(65, 4096, 4096), (8192, 7168, 18432)]:
+        assert fw(M, N, K) == 0 and ws(M, N, K) == 0
