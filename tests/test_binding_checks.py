@@ -6,6 +6,8 @@ The CPU cases need no GPU: a tensor that is not on a CUDA device is refused
 before the library is called.  The GPU cases build wrong operands on the
 device and check that each is refused by the binding, and that the library
 then still runs a correct call (nothing was enqueued by the refused ones).
+A last CPU case checks that every ctypes signature in the binding has as
+many arguments as its declaration in include/fp8bl.h.
 """
 import pytest
 import torch
@@ -96,3 +98,31 @@ def test_wrong_operands_refused_on_device():
     ref = (x.float() @ w.float().t())
     err = (y.float() - ref).norm() / ref.norm()
     assert float(err) < 0.1
+
+
+def _header_param_counts():
+    import os
+    import re
+    hdr = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fp8bl.h")
+    txt = re.sub(r"/\*.*?\*/", "", open(hdr).read(), flags=re.S)
+    out = {}
+    for name, params in re.findall(r"\b(fp8\w*)\s*\(([^;{]*?)\)\s*;", txt, flags=re.S):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argtypes_match_the_header():
+    """Every function the binding declares to ctypes takes as many arguments
+    as its C declaration (a missing or extra one would shift every pointer
+    after it)."""
+    from fine_grained_block_token_b200 import _binding as b
+    counts = _header_param_counts()
+    checked = 0
+    for name, n in counts.items():
+        f = getattr(b._lib, name)
+        if f.argtypes is None:
+            continue
+        assert len(f.argtypes) == n, (name, len(f.argtypes), n)
+        checked += 1
+    assert checked >= 15
