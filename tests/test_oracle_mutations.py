@@ -4,7 +4,9 @@ Each case compiles a mutated copy of oracle/fp8bl_oracle.c into a temporary
 library, swaps it in for the real one, and checks that at least one pin of
 the relevant kind fails.  This shows the pins are sensitive to the plausible
 errors they are meant to catch (a dropped term, a transposed index, the
-reciprocal instead of the division, a wrong rounding).
+reciprocal instead of the division, a wrong rounding).  The grouped (MoE)
+oracle is a Python composition, so its mutants are planted in a copy of that
+Python function instead.
 """
 import os
 import subprocess
@@ -169,3 +171,49 @@ def test_static_pins_catch(tmp_path, monkeypatch, old, new):
     checks = [lambda: tst.test_vs_library_composition(0.01), tst.test_saturates_above_448_s,
               tst.test_equals_dynamic_when_s_is_every_groups_scale]
     assert any(_fails(c) for c in checks)
+
+
+GROUPED_MUTANTS = [
+    # segment end taken as inclusive
+    ("(want < off[e + 1])", "(want <= off[e + 1])"),
+    # segment start taken as exclusive
+    ("(want >= off[e])", "(want > off[e])"),
+    # the next expert's weights and scales
+    ("q_w[e], c_w[e]", "q_w[min(e + 1, E - 1)], c_w[min(e + 1, E - 1)]"),
+    # expert 0's weight scales for every expert
+    ("q_w[e], c_w[e]", "q_w[e], c_w[0]"),
+    # offsets no longer validated
+    ('raise ValueError("offsets must be non-decreasing within [0, M]")', "pass"),
+]
+
+
+@pytest.mark.parametrize("old,new", GROUPED_MUTANTS)
+def test_grouped_pins_catch(monkeypatch, old, new):
+    """The grouped oracle is a Python composition of the pinned UE8M0 block
+    linear, so its mutants are planted in a copy of that Python function."""
+    import inspect
+    from tests import test_oracle_grouped as tgr
+    src = inspect.getsource(oracle.grouped_linear_ue8m0)
+    assert old in src, old
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new, 1), "<grouped mutant>", "exec"), ns)
+    monkeypatch.setattr(oracle, "grouped_linear_ue8m0", ns["grouped_linear_ue8m0"])
+    checks = [tgr.test_vs_exact_rationals_with_an_empty_expert, tgr.test_one_expert_is_the_block_linear,
+              tgr.test_rows_depend_only_on_their_expert, tgr.test_rows_outside_the_segments_are_not_produced,
+              tgr.test_bad_offsets_raise, tgr.test_row_subset_matches_full]
+
+    def fails(fn):
+        try:
+            fn()
+        except (Exception, pytest.fail.Exception):   # a failed assertion, pytest.raises, or a crash
+            return True
+        return False
+    assert any(fails(c) for c in checks)
+
+
+def test_real_grouped_oracle_passes_the_same_checks():
+    from tests import test_oracle_grouped as tgr
+    for c in (tgr.test_vs_exact_rationals_with_an_empty_expert, tgr.test_one_expert_is_the_block_linear,
+              tgr.test_rows_depend_only_on_their_expert, tgr.test_rows_outside_the_segments_are_not_produced,
+              tgr.test_bad_offsets_raise, tgr.test_row_subset_matches_full):
+        c()
