@@ -136,3 +136,41 @@ def test_bf16_rne_view():
     import torch
     ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
     assert np.array_equal(oracle.bf16_rne(v.astype(np.float64)), ref)
+
+
+def _bf16_value(bits):
+    """fp64 value of bf16 bit patterns (exact)."""
+    b = np.asarray(bits, dtype=np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def test_bf16_rne_view_fp64_ties_and_near_ties():
+    """fp64 inputs (the oracle's GEMM results are fp64): brute force over the
+    bf16 grid around each value picks the nearest, ties to the even code.
+    Cases include exact midpoints between neighbouring bf16 values and
+    midpoints moved by a few fp64 ulps -- the values a detour through fp32
+    would round twice (midpoint + 2^-40 relative becomes the midpoint in
+    fp32, then rounds to even instead of up)."""
+    rng = np.random.default_rng(7)
+    lo_bits = rng.integers(0x0080, 0x7F00, 4000).astype(np.uint32)      # normal positive bf16
+    lo, hi = _bf16_value(lo_bits), _bf16_value(lo_bits + 1)
+    mid = (lo + hi) / 2                                                   # exact in fp64
+    eps = np.abs(mid) * 2.0 ** -40
+    vals = np.concatenate([mid, mid + eps, mid - eps, lo + (hi - lo) * rng.random(4000)])
+    vals = np.concatenate([vals, -vals])
+    got = oracle.bf16_rne(vals)
+    a = np.abs(vals)
+    base = (a.astype(np.float32).view(np.uint32) >> 16).astype(np.int64)  # within one code of the answer
+    best = np.empty_like(a)
+    for i in range(len(a)):
+        cands = _bf16_value(np.arange(max(base[i] - 2, 0), base[i] + 3))
+        d = np.abs(cands - a[i])
+        k = np.flatnonzero(d == d.min())
+        if len(k) > 1:                                                    # a tie: the even code
+            codes = np.arange(max(base[i] - 2, 0), base[i] + 3)[k]
+            k = k[codes % 2 == 0]
+        best[i] = cands[k[0]]
+    assert np.array_equal(got, np.sign(vals) * best)
+    # the double-rounding trap is really exercised: fp32 first would differ
+    via32 = np.asarray(oracle.bf16_rne(vals.astype(np.float32).astype(np.float64)))
+    assert np.count_nonzero(via32 != got) > 1000
