@@ -539,7 +539,426 @@ def run_moe(args):
     return 0
 
 
+# ----------------------------------------------------- per-config legs
+#
+# The default run reports every workload of the build on the same JSON line:
+# besides the headline prefill step, `decode` (the 16 Llama-3-8B decode
+# linears and a whole layer per token count), `deepseek_mlp`, `sweep` and
+# `tiny`.  Each leg times on the device (CUDA events around CUDA-graph
+# replays, max over ranks) and carries its roofline fraction, an oracle check
+# of sampled outputs and an oracle CPU baseline.
+L2_BYTES = 126e6
+
+
+def capture_graph(fn, dev):
+    """CUDA graph of fn() (one warm-up run on a side stream first)."""
+    import torch
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize(dev)
+    return g
+
+
+def timed_replays(run, reps, barrier, warm=2):
+    """Device ms of `reps` calls of run() between two events (after `warm`
+    untimed calls), with a barrier + synchronize on both sides."""
+    import torch
+    for _ in range(warm):
+        run()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    a.record()
+    for _ in range(reps):
+        run()
+    b.record()
+    barrier()
+    return a.elapsed_time(b)
+
+
+def copies_for(bytes_per_launch: float) -> int:
+    """Distinct buffer copies a rotation needs so that every launch reads
+    operands that left the L2 (the rotation moves >= 2.5 x L2)."""
+    return max(2, int(np.ceil(2.5 * L2_BYTES / bytes_per_launch)))
+
+
+def decode_bytes(M, N, K):
+    """Algorithmic bytes of one decode linear: W codes + block scales, X codes
+    + group scales, bf16 Y."""
+    return N * K + (N // 128) * (K // 128) * 4 + M * K + M * (K // 128) * 4 + 2 * M * N
+
+
+def leg_decode(fp8, dev, barrier, args, hbm_peak):
+    """Llama-3-8B decode linears (M in {1, 8, 32, 64}).  Every linear is timed
+    as a graph of back-to-back launches, each on another copy of the
+    quantized weights (distinct addresses, >= 2.5 x L2 per rotation), so each
+    launch streams its weights from HBM as in a model whose layers all
+    differ.  `layer` times one whole decoder layer per token count (4
+    activation quantizations + q, k, v, o, gate+up, down) over 4 layers'
+    weight copies."""
+    import torch
+    names = list(wl.LLAMA3_8B_LINEARS)
+    wsets = {}
+    for name in names:
+        N, K = wl.LLAMA3_8B_LINEARS[name]
+        w = wl.to_torch_bf16(wl.llama3_decode_w(name)).to(dev)
+        q_w, s_w = fp8.quant_weight(w)
+        del w
+        R = copies_for(N * K)
+        wsets[name] = [(q_w, s_w)] + [(q_w.clone(), s_w.clone()) for _ in range(R - 1)]
+    torch.cuda.synchronize(dev)
+    out, acts = {}, {}
+    tot_bytes, tot_ms = 0.0, 0.0
+    for M in wl.DECODE_M:
+        for name in names:
+            N, K = wl.LLAMA3_8B_LINEARS[name]
+            xb = wl.llama3_decode_x(M, name)
+            x = wl.to_torch_bf16(xb).to(dev)
+            q_a, s_a = fp8.quant_act(x)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(max(fp8.workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
+            cps = wsets[name]
+
+            def run(q_a=q_a, s_a=s_a, y=y, ws=ws, cps=cps):
+                for q_w, s_w in cps:
+                    fp8.block_linear(q_a, s_a, q_w, s_w, y, ws)
+
+            g = capture_graph(run, dev)
+            reps = max(2, int(np.ceil(args.decode_launches / len(cps))))
+            ms = timed_replays(g.replay, reps, barrier)
+            del g
+            launches = reps * len(cps)
+            out[f"{name}_M{M}"] = dict(ms=ms, launches=launches, bytes=decode_bytes(M, N, K))
+            acts[(name, M)] = dict(xb=xb, x=x, q_a=q_a, s_a=s_a, y=y, ws=ws)
+    # whole layers: q, k, v share the attention input; o, gate+up and down
+    # each quantize their own input
+    layers = 4
+    layer_out = {}
+    for M in wl.DECODE_M:
+        qa_bufs = {n: (torch.empty_like(acts[(n, M)]["q_a"]), torch.empty_like(acts[(n, M)]["s_a"]))
+                   for n in names}
+        # the layer writes its own outputs (the per-linear outputs above are
+        # checked against the oracle afterwards)
+        y_bufs = {n: torch.empty_like(acts[(n, M)]["y"]) for n in names}
+
+        def layer_run(M=M, qa_bufs=qa_bufs, y_bufs=y_bufs):
+            for l in range(layers):
+                def lin(name, idx, xname):
+                    cp = wsets[name][idx % len(wsets[name])]
+                    fp8.block_linear(qa_bufs[xname][0], qa_bufs[xname][1], cp[0], cp[1], y_bufs[name],
+                                     acts[(name, M)]["ws"])
+                fp8.quant_act(acts[("qo", M)]["x"], *qa_bufs["qo"])
+                lin("qo", 2 * l, "qo")
+                lin("kv", 2 * l, "qo")
+                lin("kv", 2 * l + 1, "qo")
+                fp8.quant_act(acts[("kv", M)]["x"], *qa_bufs["kv"])
+                lin("qo", 2 * l + 1, "kv")
+                fp8.quant_act(acts[("gate_up", M)]["x"], *qa_bufs["gate_up"])
+                lin("gate_up", l, "gate_up")
+                fp8.quant_act(acts[("down", M)]["x"], *qa_bufs["down"])
+                lin("down", l, "down")
+
+        g = capture_graph(layer_run, dev)
+        reps = max(2, args.decode_launches // 24)
+        ms = timed_replays(g.replay, reps, barrier)
+        del g
+        wbytes = sum(decode_bytes(M, *wl.LLAMA3_8B_LINEARS[n]) for n in ("qo", "kv", "kv", "qo", "gate_up", "down"))
+        qbytes = sum(M * K * 3 + M * (K // 128) * 4 for K in (4096, 4096, 4096, 14336))
+        layer_out[f"M{M}"] = dict(ms=ms, reps=reps * layers, bytes=wbytes + qbytes)
+    return out, layer_out, acts, wsets
+
+
+def decode_oracle(acts, wsets, rows_per_linear=1):
+    """The oracle on the decode linears: every M = 1 linear complete (the CPU
+    baseline: activation quant + fp64 GEMM, weights' codes from the GPU) and
+    `rows_per_linear` sampled rows of the M = 8, 32, 64 linears.  Returns
+    (cpu_baseline dict, parity dict)."""
+    import torch
+    import oracle
+    threads = os.cpu_count() or 1
+    t_tot, b_tot, worst = 0.0, 0.0, 0.0
+    g = np.random.default_rng(5)
+    for (name, M), a in acts.items():
+        q_w, s_w = wsets[name][0]
+        qw = q_w.view(torch.uint8).cpu().numpy()
+        sw = s_w.cpu().numpy()
+        N, K = qw.shape
+        rows = np.arange(M) if M == 1 else np.sort(g.choice(M, rows_per_linear, replace=False))
+        xs = np.ascontiguousarray(a["xb"][rows])
+        t0 = time.perf_counter()
+        qa, sa = oracle.quant_act(xs, nthreads=threads)
+        R = oracle.block_linear(qa, sa, qw, sw, nthreads=threads)
+        dt = time.perf_counter() - t0
+        if M == 1:
+            t_tot += dt
+            b_tot += decode_bytes(1, N, K)
+        Y = a["y"][torch.as_tensor(rows, device=a["y"].device)].float().cpu().numpy()
+        worst = max(worst, within_tolerance(Y, R))
+    cpu = {"value": b_tot / t_tot / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+           "seconds": t_tot,
+           "sample": "the four Llama-3-8B decode linears at M = 1, complete (activation quant + "
+                     "fp64 block-scaled GEMM; weights quantized before timing); GB/s of the same "
+                     "algorithmic bytes as the GPU figure"}
+    par = {"rows": f"all rows at M = 1, {rows_per_linear} sampled row(s) at M = 8, 32, 64, all N",
+           "within_tolerance": worst <= 1.0, "worst_bound_ratio": worst}
+    return cpu, par
+
+
+def leg_gemm_workload(fp8, dev, barrier, args, lins):
+    """One large-M workload (e.g. the DeepSeek-V3 MLP): the step = per linear
+    quant_act + block_linear, graph-replayed; the GEMMs' own rate from a pass
+    with events around them; the fused entry point on the same inputs, with
+    a bit-identity check against the two-call output."""
+    import torch
+    items = []
+    for label, xb, wb in lins:
+        M, K = xb.shape
+        N = wb.shape[0]
+        x = wl.to_torch_bf16(xb).to(dev)
+        w = wl.to_torch_bf16(wb).to(dev)
+        q_w, s_w = fp8.quant_weight(w)
+        del w
+        items.append(dict(label=label, xb=xb, x=x, q_w=q_w, s_w=s_w,
+                          q_a=torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev),
+                          s_a=torch.empty((M, K // 128), dtype=torch.float32, device=dev),
+                          y=torch.empty((M, N), dtype=torch.bfloat16, device=dev), M=M, N=N, K=K))
+
+    def step(ev=None):
+        for i, it in enumerate(items):
+            fp8.quant_act(it["x"], it["q_a"], it["s_a"])
+            if ev is not None:
+                ev[2 * i].record()
+            fp8.block_linear(it["q_a"], it["s_a"], it["q_w"], it["s_w"], it["y"])
+            if ev is not None:
+                ev[2 * i + 1].record()
+
+    g = capture_graph(step, dev)
+    ms = timed_replays(g.replay, args.steps, barrier)
+    del g
+    n = len(items)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(args.steps)]
+    barrier()
+    for k in range(args.steps):
+        step(evs[k])
+    barrier()
+    gemm_ms = sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs for i in range(n))
+    y_ref = [it["y"].clone() for it in items]
+
+    def fused():
+        for it in items:
+            fp8.block_linear_fused(it["x"], it["q_w"], it["s_w"], it["y"])
+
+    g = capture_graph(fused, dev)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    same = all(torch.equal(r.view(torch.int16), it["y"].view(torch.int16)) for r, it in zip(y_ref, items))
+    fused_ms = timed_replays(g.replay, args.steps, barrier)
+    del g
+    flops = sum(2 * it["M"] * it["N"] * it["K"] for it in items)
+    return items, dict(ms=ms, gemm_ms=gemm_ms, fused_ms=fused_ms, flops=flops, identical=same)
+
+
+def rows_oracle_check(items, rows_per_linear, seed=0):
+    """Oracle on `rows_per_linear` random rows of every linear (it quantizes
+    those rows of the same input bits itself; weights: the GPU's codes, held
+    bit-exact to the oracle by the tests).  Returns (cpu_baseline, parity)."""
+    import torch
+    import oracle
+    threads = os.cpu_count() or 1
+    t_tot, f_tot, worst = 0.0, 0.0, 0.0
+    for i, it in enumerate(items):
+        g = np.random.default_rng([seed, i])
+        rows = np.sort(g.choice(it["M"], min(rows_per_linear, it["M"]), replace=False))
+        qw = it["q_w"].view(torch.uint8).cpu().numpy()
+        sw = it["s_w"].cpu().numpy()
+        xs = np.ascontiguousarray(it["xb"][rows])
+        t0 = time.perf_counter()
+        qa, sa = oracle.quant_act(xs, nthreads=threads)
+        R = oracle.block_linear(qa, sa, qw, sw, nthreads=threads)
+        t_tot += time.perf_counter() - t0
+        f_tot += 2.0 * len(rows) * it["N"] * it["K"]
+        Y = it["y"][torch.as_tensor(rows, device=it["y"].device)].float().cpu().numpy()
+        worst = max(worst, within_tolerance(Y, R))
+    desc = (f"{rows_per_linear} random rows per linear ({', '.join(it['label'] for it in items)}), "
+            "all N columns; activation quant + fp64 GEMM of those rows; weights quantized before timing")
+    return ({"value": f_tot / t_tot / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+             "sample": desc, "seconds": t_tot},
+            {"rows_per_linear": rows_per_linear, "within_tolerance": worst <= 1.0,
+             "worst_bound_ratio": worst})
+
+
+def leg_sweep(fp8, dev, barrier, args):
+    """Sweep X [M, 7168], M = 512 .. 16384, against W [2048, 7168]: per M the
+    activation quantizer's GB/s, the unfused GEMM's and the fused entry
+    point's TFLOP/s.  Every launch reads another copy of its operands
+    (>= 2.5 x L2 per rotation), so small M is not served from the L2."""
+    import torch
+    wb = wl.sweep_w()
+    w = wl.to_torch_bf16(wb).to(dev)
+    q_w0, s_w0 = fp8.quant_weight(w)
+    del w
+    K, N = wl.SWEEP_K, wl.SWEEP_N
+    res, items = {}, []
+    for M in wl.SWEEP_M:
+        xb = wl.sweep_x(M)
+        x0 = wl.to_torch_bf16(xb).to(dev)
+        qbytes = M * K * 3 + M * (K // 128) * 4
+        gbytes = M * K + N * K + 2 * M * N
+        R = copies_for(min(qbytes, gbytes))
+        xs = [x0] + [x0.clone() for _ in range(R - 1)]
+        qs = [(torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev),
+               torch.empty((M, K // 128), dtype=torch.float32, device=dev)) for _ in range(R)]
+        ws = [(q_w0, s_w0)] + [(q_w0.clone(), s_w0.clone()) for _ in range(R - 1)]
+        ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+        reps = max(2, int(np.ceil(args.sweep_launches / R)))
+
+        def quant():
+            for x, (q, s) in zip(xs, qs):
+                fp8.quant_act(x, q, s)
+
+        def gemm():
+            for (q, s), (qw, sw), y in zip(qs, ws, ys):
+                fp8.block_linear(q, s, qw, sw, y)
+
+        yf = [torch.empty_like(y) for y in ys]
+
+        def fused():
+            for x, (qw, sw), y in zip(xs, ws, yf):
+                fp8.block_linear_fused(x, qw, sw, y)
+
+        r = {}
+        for key, fn in (("quant", quant), ("gemm", gemm), ("fused", fused)):
+            g = capture_graph(fn, dev)
+            r[key] = timed_replays(g.replay, reps, barrier) / (reps * R)
+            del g
+        torch.cuda.synchronize(dev)
+        same = all(torch.equal(a.view(torch.int16), b.view(torch.int16)) for a, b in zip(ys, yf))
+        res[f"M{M}"] = dict(quant_ms=r["quant"], gemm_ms=r["gemm"], fused_ms=r["fused"], identical=same,
+                            qbytes=qbytes, flops=2.0 * M * N * K, copies=R)
+        items.append(dict(label=f"M{M}", xb=xb, q_w=q_w0, s_w=s_w0, y=ys[0], M=M, N=N, K=K))
+        del xs, qs, ws, yf
+    return res, items
+
+
+def leg_tiny(fp8, dev, barrier, args):
+    """The tiny linear (X [32, 512], W [256, 512]): latency of one
+    quant_act + block_linear, from a graph of back-to-back calls; the output
+    is compared with the oracle element by element."""
+    import torch
+    import oracle
+    xb, wb = wl.tiny()
+    x = wl.to_torch_bf16(xb).to(dev)
+    q_w, s_w = fp8.quant_weight(wl.to_torch_bf16(wb).to(dev))
+    M, K = xb.shape
+    N = wb.shape[0]
+    q_a = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev)
+    s_a = torch.empty((M, K // 128), dtype=torch.float32, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(fp8.workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
+    calls = 50
+
+    def run():
+        for _ in range(calls):
+            fp8.quant_act(x, q_a, s_a)
+            fp8.block_linear(q_a, s_a, q_w, s_w, y, ws)
+
+    g = capture_graph(run, dev)
+    ms = timed_replays(g.replay, 4, barrier) / (4 * calls)
+    del g
+    t0 = time.perf_counter()
+    qa, sa = oracle.quant_act(xb)
+    R = oracle.block_linear(qa, sa, q_w.view(torch.uint8).cpu().numpy(), s_w.cpu().numpy())
+    cpu_s = time.perf_counter() - t0
+    worst = within_tolerance(y.float().cpu().numpy(), R)
+    codes_same = bool(np.array_equal(q_a.view(torch.uint8).cpu().numpy(), qa) and
+                      np.array_equal(s_a.cpu().numpy().view(np.uint32), sa.view(np.uint32)))
+    return dict(ms=ms, flops=2.0 * M * N * K, worst=worst, codes_same=codes_same, cpu_s=cpu_s)
+
+
 # ----------------------------------------------------------------- GPU side
+
+def legs_json(legs, world, args, hbm_peak, fp8_peak, peak_src):
+    """JSON keys of the per-config legs (rank 0, after the max over ranks).
+    The oracle checks and CPU baselines run only at N = 1 (replicas compute
+    the same thing)."""
+    out = {}
+    cpu_ok = world == 1 and not args.no_cpu
+    dec, lay, acts, wsets = legs["decode"]
+    lin = {}
+    tb, tm = 0.0, 0.0
+    for k, d in dec.items():
+        us = d["ms"] * 1e3 / d["launches"]
+        gbs = d["bytes"] / (us * 1e-6) / 1e9
+        lin[k] = {"us": us, "GBps": gbs, "frac": gbs / hbm_peak, "bytes": d["bytes"]}
+        tb += d["bytes"] * d["launches"]
+        tm += d["ms"]
+    agg = tb / (tm * 1e-3) / 1e9
+    layer = {}
+    for k, d in lay.items():
+        us = d["ms"] * 1e3 / d["reps"]
+        gbs = d["bytes"] / (us * 1e-6) / 1e9
+        layer[k] = {"us_per_layer": us, "GBps": gbs, "frac": gbs / hbm_peak}
+    dcpu, dpar = decode_oracle(acts, wsets) if cpu_ok else (None, None)
+    out["decode"] = {
+        "metric": "decode linear GB/s (algorithmic bytes: W codes + block scales, X codes + scales, Y)",
+        "value": agg, "unit": "GB/s", "peak": hbm_peak, "frac": agg / hbm_peak,
+        "peak_source": f"{peak_src} copy", "kernel": "decode_kernel",
+        "linears": lin, "layer": layer,
+        "config": {"workload": "llama3_decode", "M": list(wl.DECODE_M),
+                   "linears": {n: list(v) for n, v in wl.LLAMA3_8B_LINEARS.items()},
+                   "l2": "each launch reads another copy of the weights (a rotation moves >= 2.5 x L2)",
+                   "launch": "CUDA graph of back-to-back launches (programmatic dependent launch)",
+                   "layer": "one decoder layer = 4 activation quantizations + q, k, v, o, gate+up, down; "
+                            "4 layers' weight copies per replay"},
+        "cpu_baseline": dcpu, "parity": dpar}
+    items, ds = legs["deepseek_mlp"]
+    tf = ds["flops"] * args.steps / (ds["gemm_ms"] * 1e-3) / 1e12
+    step_tf = whole_job_rate(world, ds["flops"], args.steps, ds["ms"]) / 1e12
+    dcpu, dpar = rows_oracle_check(items, 4) if cpu_ok else (None, None)
+    out["deepseek_mlp"] = {
+        "value": step_tf, "unit": "TFLOP/s", "ms_per_step": ds["ms"] / args.steps,
+        "config": {"workload": "deepseek_mlp",
+                   "linears": {it["label"]: [it["M"], it["N"], it["K"]] for it in items},
+                   "l2": "no flush: a step's inputs exceed the 126 MB L2"},
+        "gemm": {"kernel": "gemm_prefill_kernel", "achieved": tf, "peak": fp8_peak, "unit": "TFLOP/s",
+                 "frac": tf / fp8_peak, "ms_per_launch": ds["gemm_ms"] / (args.steps * len(items)),
+                 "traffic": recorded_traffic("gemm_prefill_kernel", "deepseek_mlp")},
+        "fused": {"value": whole_job_rate(world, ds["flops"], args.steps, ds["fused_ms"]) / 1e12,
+                  "vs_two_call": ds["ms"] / ds["fused_ms"], "identical_to_two_call": ds["identical"]},
+        "cpu_baseline": dcpu, "parity": dpar}
+    sw, sitems = legs["sweep"]
+    per = {}
+    for k, d in sw.items():
+        q_gbs = d["qbytes"] / (d["quant_ms"] * 1e-3) / 1e9
+        g_tf = d["flops"] / (d["gemm_ms"] * 1e-3) / 1e12
+        f_tf = d["flops"] / (d["fused_ms"] * 1e-3) / 1e12
+        per[k] = {"act_quant_GBps": q_gbs, "act_quant_frac": q_gbs / hbm_peak,
+                  "gemm_TFLOPs": g_tf, "gemm_frac": g_tf / fp8_peak,
+                  "fused_TFLOPs": f_tf, "fused_vs_two_call": (d["quant_ms"] + d["gemm_ms"]) / d["fused_ms"],
+                  "identical_to_two_call": d["identical"], "copies": d["copies"]}
+    scpu, spar = rows_oracle_check(sitems, 4, seed=1) if cpu_ok else (None, None)
+    out["sweep"] = {
+        "unit": {"act_quant": "GB/s", "gemm": "TFLOP/s"}, "hbm_peak": hbm_peak, "fp8_peak": fp8_peak,
+        "config": {"workload": "sweep", "M": list(wl.SWEEP_M), "N": wl.SWEEP_N, "K": wl.SWEEP_K,
+                   "l2": "each launch reads another copy of its operands (a rotation moves >= 2.5 x L2)"},
+        "per_M": per, "cpu_baseline": scpu, "parity": spar}
+    t = legs["tiny"]
+    out["tiny"] = {"us_per_linear": t["ms"] * 1e3, "unit": "us (quant_act + block_linear)",
+                   "TFLOPs": t["flops"] / (t["ms"] * 1e-3) / 1e12,
+                   "config": {"workload": "tiny", "M": 32, "N": 256, "K": 512,
+                              "launch": "CUDA graph of 50 back-to-back calls"},
+                   "parity": {"all_elements": True, "within_tolerance": t["worst"] <= 1.0,
+                              "worst_bound_ratio": t["worst"], "codes_and_scales_bit_exact": t["codes_same"]},
+                   "cpu_baseline": {"value": t["cpu_s"] * 1e6, "unit": "us", "kind": "oracle",
+                                    "cores": 1, "sample": "the whole tiny linear"} if cpu_ok else None}
+    return out
+
 
 def run_ours(args):
     import torch
@@ -649,9 +1068,24 @@ def run_ours(args):
     for k in range(args.steps):
         step(evs[k])
     barrier()
-    act_ms = sum(e[4 * i].elapsed_time(e[4 * i + 1]) for e in evs for i in range(n))
     gemm_ms = sum(e[4 * i + 2].elapsed_time(e[4 * i + 3]) for e in evs for i in range(n))
     fp8.check()
+
+    # ---- the activation quantizer's own rate: a graph of back-to-back
+    # quantizations of the step's inputs (no events between kernels; the
+    # step's inputs exceed the L2, so every launch reads X from HBM)
+    aq_per_graph = 10
+
+    def quant_only():
+        for _ in range(aq_per_graph):
+            for it in items:
+                fp8.quant_act(it["x"], it["q_a"], it["s_a"])
+
+    aq_graph = capture_graph(quant_only, dev)
+    aq_reps = max(2, args.steps // 5)
+    act_ms = timed_replays(aq_graph.replay, aq_reps, barrier)
+    del aq_graph
+    act_steps = aq_per_graph * aq_reps
 
     # ---- end to end: pinned host inputs in, outputs back, every step
     host_x = [wl.to_torch_bf16(it["xb"]).pin_memory() for it in items]
@@ -768,22 +1202,47 @@ def run_ours(args):
             v_gemm_ms = sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evv for i in range(n))
             del v_graph
             variants[name] = dict(items=v_items, ms=v_ms, gemm_ms=v_gemm_ms, kernel=sp["kernel"])
+    # ---- the other workloads of the build, on the same line
+    legs = {}
+    run_legs = args.workload == "llama3_prefill" and not args.no_legs
+    if run_legs:
+        legs["decode"] = leg_decode(fp8, dev, barrier, args, hbm_peak)
+        legs["deepseek_mlp"] = leg_gemm_workload(fp8, dev, barrier, args,
+                                                 workload_linears("deepseek_mlp"))
+        legs["sweep"] = leg_sweep(fp8, dev, barrier, args)
+        legs["tiny"] = leg_tiny(fp8, dev, barrier, args)
     sampler.stop()
     fp8.check()
 
-    # max over ranks
+    # max over ranks (every device time below is the slowest rank's)
     vnames = sorted(variants)
-    maxed = max_over_ranks([elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms] +
-                           [variants[v][k] for v in vnames for k in ("ms", "gemm_ms")], dev, world)
+    times = [elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms] + \
+        [variants[v][k] for v in vnames for k in ("ms", "gemm_ms")]
+    leg_slots = []
+    if run_legs:
+        dec, lay, _, _ = legs["decode"]
+        for k in sorted(dec):
+            leg_slots.append((dec[k], "ms"))
+        for k in sorted(lay):
+            leg_slots.append((lay[k], "ms"))
+        _, ds = legs["deepseek_mlp"]
+        leg_slots += [(ds, "ms"), (ds, "gemm_ms"), (ds, "fused_ms")]
+        sw, _ = legs["sweep"]
+        for k in sorted(sw):
+            leg_slots += [(sw[k], "quant_ms"), (sw[k], "gemm_ms"), (sw[k], "fused_ms")]
+        leg_slots.append((legs["tiny"], "ms"))
+    maxed = max_over_ranks(times + [d[k] for d, k in leg_slots], dev, world)
     elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms = maxed[:5]
     for i, v in enumerate(vnames):
         variants[v]["ms"], variants[v]["gemm_ms"] = maxed[5 + 2 * i], maxed[6 + 2 * i]
+    for (d, k), v in zip(leg_slots, maxed[len(times):]):
+        d[k] = v
 
     ms_per_step = elapsed_ms / args.steps
     value = whole_job_rate(world, flops_step, args.steps, elapsed_ms) / 1e12
     e2e_value = whole_job_rate(world, flops_step, e2e_steps, e2e_ms) / 1e12
     gemm_tflops = gemm_flops_step * args.steps / (gemm_ms * 1e-3) / 1e12
-    act_gbs = act_bytes_step * args.steps / (act_ms * 1e-3) / 1e9
+    act_gbs = act_bytes_step * act_steps / (act_ms * 1e-3) / 1e9
     launches_per_step = 2 * n
     fused_value = whole_job_rate(world, flops_step, args.steps, fused_ms) / 1e12
     decode = args.workload == "llama3_decode"
@@ -849,7 +1308,10 @@ def run_ours(args):
                           "peak_source": f"{peak_src} bf16 burst x {FP8_OVER_BF16} (nominal fp8/bf16)",
                           "ms_per_launch": gemm_ms_per_launch}),
             "act_quant": {"achieved": act_gbs, "peak": hbm_peak, "unit": "GB/s",
-                          "frac": act_gbs / hbm_peak, "peak_source": f"{peak_src} copy"},
+                          "frac": act_gbs / hbm_peak, "peak_source": f"{peak_src} copy",
+                          "kernel": "act_quant32_kernel",
+                          "timing": f"CUDA graph of {aq_per_graph} x the step's quantizations back to back, "
+                                    f"{aq_reps} replays"},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "fused": {"value": fused_value, "unit": "TFLOP/s", "ms_per_step": fused_ms / args.steps,
@@ -858,6 +1320,7 @@ def run_ours(args):
                       "identical_to_two_call": fused_identical},
             "ue8m0": variant_lines.get("ue8m0"),
             "fp8r": variant_lines.get("fp8r"),
+            **(legs_json(legs, world, args, hbm_peak, fp8_peak, peak_src) if run_legs else {}),
             "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary(),
             "cpu_baseline": cpu,
@@ -888,6 +1351,12 @@ def main():
                     help="rows per linear of the ue8m0 / fp8r legs checked against the oracle")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch every step's kernels one by one")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="headline prefill step only (skip the decode, deepseek_mlp, sweep, tiny keys)")
+    ap.add_argument("--decode-launches", type=int, default=96,
+                    help="timed launches per decode linear (rounded up to whole weight rotations)")
+    ap.add_argument("--sweep-launches", type=int, default=12,
+                    help="timed launches per sweep size and kernel (whole rotations)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps
     if args.impl == "reference":

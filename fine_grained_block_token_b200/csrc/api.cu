@@ -17,7 +17,6 @@ namespace {
 // device image of this library; read and cleared by fp8bl_check().
 __device__ int g_kernel_error;
 
-constexpr int kMaxDevices = 64;
 DeviceInfo g_info[kMaxDevices];
 std::once_flag g_once[kMaxDevices];
 

@@ -16,16 +16,26 @@
 //     caller's workspace.
 //   - reduce: a block that one CTA covers alone is written as bf16 directly.
 //     For a shared block, every contributing CTA writes its partial and
-//     bumps the block's counter; the last one to arrive sums the block's
-//     partials in increasing CTA order (a fixed order: results are
-//     bit-identical run to run) and writes bf16 Y[m, n].  The counters live
-//     at the head of the workspace and are zeroed (cudaMemsetAsync) before
-//     every launch.
+//     counts itself in on the block's counter; the last one to arrive sums
+//     the block's partials in increasing CTA order (a fixed order: results
+//     are bit-identical run to run), writes bf16 Y[m, n] and puts the
+//     counter back to zero.  A counter holds a 48-bit call tag next to the
+//     count, and a count whose tag differs from the launch's tag reads as
+//     zero, so the workspace needs no clearing before a launch (a cleared or
+//     reset counter is the zero word; a stale one carries another tag).
 // Warps: 0 TMA producer (W tile 128x128 + X tile Mpad x 128 per stage,
-// 8 stages), 1 MMA issuer, 2 TMEM owner, 3 idle, 4-7 promotion (one weight
-// row per thread, Mpad fp32 accumulators, scale s_w[blk, j] * s_a[m, j]).
+// 8 stages), 1 MMA issuer, 2 TMEM owner, 3 scale products (for every chunk
+// the Mpad factors s_w[blk, j] * s_a[m, j], once per CTA, into a shared
+// ring), 4-11 promotion: two warps per TMEM lane quarter, one weight row
+// per thread, each warp a contiguous part of the token columns.
+// The kernel is launched with programmatic stream serialization: its set-up
+// (barriers, TMEM, tensor-map prefetch, an L2 prefetch of its first weight
+// tiles) overlaps the previous kernel, and it waits for that kernel to
+// finish before its first access to anything another kernel can write.
 // Every mbarrier wait is bounded; on expiry the kernel records an error
 // code, drains what it started and exits cleanly.
+#include <atomic>
+#include <chrono>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -45,28 +55,31 @@ constexpr int MAX_MPAD = 64;
 constexpr int DSTAGES = 8;
 constexpr int DTBUFS = 4;
 constexpr int DUMMA_K = 32;
+constexpr int CSLOTS = 16;                   // ring of per-chunk scale products
 constexpr int W_BYTES = DBM * DBK;           // 16 KB
 constexpr int X_BYTES = MAX_MPAD * DBK;      // 8 KB (box rows = Mpad <= 64)
 constexpr int DTMEM_COLS = 256;              // DTBUFS * MAX_MPAD
-constexpr int DNUM_THREADS = 256;
+constexpr int DNUM_THREADS = 384;
+constexpr int PROMO_THREADS = 256;           // warps 4-11
 
 constexpr int DSMEM_W_OFF = 0;
 constexpr int DSMEM_X_OFF = DSMEM_W_OFF + DSTAGES * W_BYTES;
-constexpr int DSMEM_BAR_OFF = DSMEM_X_OFF + DSTAGES * X_BYTES;
-constexpr int DNUM_BARS = 2 * DSTAGES + 2 * DTBUFS + 1;
+constexpr int DSMEM_C_OFF = DSMEM_X_OFF + DSTAGES * X_BYTES;
+constexpr int DSMEM_BAR_OFF = DSMEM_C_OFF + CSLOTS * MAX_MPAD * 4;
+constexpr int DNUM_BARS = 2 * DSTAGES + 2 * DTBUFS + 2 * CSLOTS + 1;
 constexpr int DSMEM_MISC_OFF = DSMEM_BAR_OFF + DNUM_BARS * 8;
-constexpr int DSMEM_BYTES = DSMEM_MISC_OFF + 16 + 1024;
+constexpr int DSMEM_BYTES = DSMEM_MISC_OFF + 16 + 1024;   // + slack for 1024-byte alignment
 
 struct DecodeArgs {
-  const float* s_a;       // [M, KB]
-  const float* s_w;       // [NB, KB]
-  __nv_bfloat16* y;       // [M, N]
-  int* counters;          // [NB], zero on entry
-  float* partial;         // [G * maxseg, Mpad, 128]
-  int N;
-  int M, Mpad, KB;
-  int64_t units;          // NB * KB
-  int G;                  // CTAs
+  const float* s_a;                 // [M, KB]
+  const float* s_w;                 // [NB, KB]
+  __nv_bfloat16* y;                 // [M, N]
+  unsigned long long* counters;     // [NB] tagged arrival counters
+  float* partial;                   // [G * maxseg, Mpad, 128]
+  unsigned long long tag;           // this launch's tag, 1 .. 2^48 - 1
+  int64_t units;                    // NB * KB
+  int N, M, KB;
+  int G;                            // CTAs
   int maxseg;
   int* err;
 };
@@ -77,6 +90,186 @@ __device__ __forceinline__ int64_t range_start(int g, int64_t units, int G) {
 
 __device__ __forceinline__ void record_error(int* err, int code) { atomicCAS(err, 0, code); }
 
+// Counts one contributor in on a block counter and says whether it was the
+// last of `contributors`.  Word = tag << 16 | count; a word carrying another
+// tag (a zero word included) counts as zero.
+__device__ __forceinline__ bool arrive_last(unsigned long long* ctr, unsigned long long tag,
+                                            int contributors) {
+  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(ctr);
+  unsigned long long assumed, next;
+  do {
+    assumed = old;
+    const unsigned long long base = (assumed >> 16) == tag ? (assumed & 0xFFFFull) : 0ull;
+    next = (tag << 16) | (base + 1ull);
+    old = atomicCAS(ctr, assumed, next);
+  } while (old != assumed);
+  return (next & 0xFFFFull) == static_cast<unsigned long long>(contributors);
+}
+
+struct PromoCtx {
+  uint32_t smem_base, tmem_base;
+  const float* prods;       // shared ring [CSLOTS][MAX_MPAD]
+  volatile int* last_flag;  // shared
+  int64_t u_begin, u_end;
+  int g, quarter, lane;
+};
+
+__device__ __forceinline__ uint32_t dbar(uint32_t smem_base, int i) {
+  return smem_base + DSMEM_BAR_OFF + 8u * i;
+}
+// barrier indices
+__device__ __forceinline__ int bi_full(int s) { return s; }
+__device__ __forceinline__ int bi_empty(int s) { return DSTAGES + s; }
+__device__ __forceinline__ int bi_tfull(int b) { return 2 * DSTAGES + b; }
+__device__ __forceinline__ int bi_tempty(int b) { return 2 * DSTAGES + DTBUFS + b; }
+__device__ __forceinline__ int bi_cfull(int i) { return 2 * DSTAGES + 2 * DTBUFS + i; }
+__device__ __forceinline__ int bi_cempty(int i) { return 2 * DSTAGES + 2 * DTBUFS + CSLOTS + i; }
+__device__ __forceinline__ int bi_drain() { return 2 * DSTAGES + 2 * DTBUFS + 2 * CSLOTS; }
+
+// Promotion by one warp: token columns COL0 .. COL0 + NC - 1 of its lane
+// quarter's 32 weight rows (NC = 0: the warp only takes part in the
+// block-end barriers and reductions).  acc[m] += partial[m] * (s_w * s_a[m])
+// with the product read from the shared ring.  All eight promotion warps
+// walk the same chunks and reach the same named barriers in the same order;
+// after a timed-out wait a warp stops touching TMEM and the ring but keeps
+// walking.
+template <int MPAD, int NC, int COL0>
+__device__ __forceinline__ void decode_promote(const DecodeArgs& args, const PromoCtx& cx) {
+  const int lane = cx.lane;
+  const int n_local = cx.quarter * 32 + lane;   // weight row within the block
+  const uint32_t lane_off = static_cast<uint32_t>(cx.quarter * 32) << 16;
+  const int KB = args.KB;
+  const int first_blk = static_cast<int>(cx.u_begin / KB);
+  constexpr int NA = NC > 0 ? NC : 1;
+  float acc[NA];
+#pragma unroll
+  for (int m = 0; m < NA; ++m) acc[m] = 0.0f;
+  uint32_t c = 0;
+  bool ok = true;
+  int blk = first_blk;
+  int kb = static_cast<int>(cx.u_begin - static_cast<int64_t>(first_blk) * KB) - 1;
+  for (int64_t u = cx.u_begin; u < cx.u_end; ++u) {
+    if (++kb == KB) {
+      kb = 0;
+      ++blk;
+    }
+    const int buf = c % DTBUFS;
+    const uint32_t bph = (c / DTBUFS) & 1u;
+    const int slot = c % CSLOTS;
+    const uint32_t cph = (c / CSLOTS) & 1u;
+    ++c;
+    if (NC > 0 && ok) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(dbar(cx.smem_base, bi_tfull(buf)), bph))) {
+        if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
+        ok = false;
+      } else {
+        ptx::tc_fence_after();
+        uint32_t v[NA];
+#pragma unroll
+        for (int j = 0; j < NC / 16; ++j)
+          ptx::tmem_ld_32x32b_x16(
+              cx.tmem_base + lane_off + static_cast<uint32_t>(buf * MAX_MPAD + COL0 + j * 16),
+              *reinterpret_cast<uint32_t(*)[16]>(&v[j * 16]));
+        ptx::tmem_ld_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(dbar(cx.smem_base, bi_tempty(buf)));
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(dbar(cx.smem_base, bi_cfull(slot)), cph))) {
+          if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
+          ok = false;
+        } else {
+          const float4* cr = reinterpret_cast<const float4*>(cx.prods + slot * MAX_MPAD + COL0);
+#pragma unroll
+          for (int j = 0; j < NC / 4; ++j) {
+            const float4 p = cr[j];
+            acc[4 * j + 0] = __fmaf_rn(__uint_as_float(v[4 * j + 0]), p.x, acc[4 * j + 0]);
+            acc[4 * j + 1] = __fmaf_rn(__uint_as_float(v[4 * j + 1]), p.y, acc[4 * j + 1]);
+            acc[4 * j + 2] = __fmaf_rn(__uint_as_float(v[4 * j + 2]), p.z, acc[4 * j + 2]);
+            acc[4 * j + 3] = __fmaf_rn(__uint_as_float(v[4 * j + 3]), p.w, acc[4 * j + 3]);
+          }
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(dbar(cx.smem_base, bi_cempty(slot)));
+        }
+      }
+    }
+    if (kb == KB - 1 || u + 1 == cx.u_end) {
+      // end of this block's segment
+      const int64_t blk_u0 = static_cast<int64_t>(blk) * KB;
+      const int64_t y_off = static_cast<int64_t>(blk) * 128 + n_local;
+      if (blk_u0 >= cx.u_begin && kb == KB - 1) {
+        // the whole block was accumulated by this CTA: write bf16 directly
+#pragma unroll
+        for (int m = 0; m < NC; ++m)
+          if (COL0 + m < args.M)
+            args.y[static_cast<int64_t>(COL0 + m) * args.N + y_off] = __float2bfloat16_rn(acc[m]);
+      } else {
+        float* dst = args.partial +
+                     (static_cast<int64_t>(cx.g) * args.maxseg + (blk - first_blk)) * (MPAD * 128);
+#pragma unroll
+        for (int m = 0; m < NC; ++m) dst[(COL0 + m) * 128 + n_local] = acc[m];
+        // Publish the partial and count this CTA in; the last one reduces.
+        // The barrier orders every thread's stores before one thread's
+        // fence + atomic (the fence is cumulative), as a grid-wide barrier
+        // does; the last CTA fences again before reading.
+        ptx::named_barrier_sync(1, PROMO_THREADS);
+        const int g_lo = static_cast<int>(((blk_u0 + 1) * args.G - 1) / args.units);
+        const int g_hi = static_cast<int>(((blk_u0 + KB) * args.G - 1) / args.units);
+        if (threadIdx.x == 128) {
+          __threadfence();
+          const bool last = arrive_last(args.counters + blk, args.tag, g_hi - g_lo + 1);
+          if (last) {
+            // every contributor has counted in: the counter is free again
+            atomicExch(args.counters + blk, 0ull);
+            __threadfence();
+          }
+          *cx.last_flag = last ? 1 : 0;
+        }
+        ptx::named_barrier_sync(1, PROMO_THREADS);
+        if (*cx.last_flag) {
+          // Sum the block's partials in increasing CTA order.  All 256
+          // promotion threads take part: thread t sums row t % 128, token
+          // columns (t / 128) * MPAD / 2 .. + MPAD / 2 - 1; UR partials'
+          // loads are in flight together.
+          constexpr int HALF = MPAD / 2;
+          constexpr int UR = HALF <= 8 ? 4 : (HALF <= 16 ? 2 : 1);
+          const int t = threadIdx.x - 128;
+          const int rn = t & 127;
+          const int m0 = (t >> 7) * HALF;
+          float sum[HALF];
+#pragma unroll
+          for (int m = 0; m < HALF; ++m) sum[m] = 0.0f;
+          for (int gg = g_lo; gg <= g_hi; gg += UR) {
+            float tv[UR][HALF];
+#pragma unroll
+            for (int r = 0; r < UR; ++r) {
+              const int gi = gg + r <= g_hi ? gg + r : g_hi;
+              const int fb = static_cast<int>(range_start(gi, args.units, args.G) / KB);
+              const float* src = args.partial +
+                                 (static_cast<int64_t>(gi) * args.maxseg + (blk - fb)) * (MPAD * 128) +
+                                 m0 * 128 + rn;
+#pragma unroll
+              for (int m = 0; m < HALF; ++m) tv[r][m] = __ldcg(src + m * 128);
+            }
+#pragma unroll
+            for (int r = 0; r < UR; ++r)
+              if (gg + r <= g_hi) {
+#pragma unroll
+                for (int m = 0; m < HALF; ++m) sum[m] += tv[r][m];
+              }
+          }
+          const int64_t yo = static_cast<int64_t>(blk) * 128 + rn;
+#pragma unroll
+          for (int m = 0; m < HALF; ++m)
+            if (m0 + m < args.M)
+              args.y[static_cast<int64_t>(m0 + m) * args.N + yo] = __float2bfloat16_rn(sum[m]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < NA; ++m) acc[m] = 0.0f;
+    }
+  }
+}
+
 template <int MPAD>
 __global__ void __launch_bounds__(DNUM_THREADS, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
@@ -85,15 +278,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t smem_base = ptx::smem_u32(smem);
-  const uint32_t bar_base = smem_base + DSMEM_BAR_OFF;
-  auto full_bar = [&](int s) { return bar_base + 8u * s; };
-  auto empty_bar = [&](int s) { return bar_base + 8u * (DSTAGES + s); };
-  auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * DSTAGES + b); };
-  auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * DSTAGES + DTBUFS + b); };
-  const uint32_t drain_bar = bar_base + 8u * (2 * DSTAGES + 2 * DTBUFS);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + DSMEM_MISC_OFF);
+  auto bar = [&](int i) { return dbar(smem_base, i); };
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + DSMEM_MISC_OFF);
+  float* prods = reinterpret_cast<float*>(smem + DSMEM_C_OFF);
   constexpr uint32_t IDESC = ptx::idesc_e4m3_f32(DBM, MPAD);
   constexpr uint32_t STAGE_TX = W_BYTES + MPAD * DBK;
+  // token columns per promotion half: half 0 takes NC0, half 1 the rest
+  constexpr int NC0 = MPAD <= 32 ? 16 : 32;
+  constexpr int NC1 = MPAD - NC0;
+  constexpr int LOADERS = NC1 > 0 ? 8 : 4;     // promotion warps that read TMEM
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -104,236 +297,169 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < DSTAGES; ++s) {
-      ptx::mbar_init(full_bar(s), 1);
-      ptx::mbar_init(empty_bar(s), 1);
+      ptx::mbar_init(bar(bi_full(s)), 1);
+      ptx::mbar_init(bar(bi_empty(s)), 1);
     }
     for (int b = 0; b < DTBUFS; ++b) {
-      ptx::mbar_init(tfull_bar(b), 1);
-      ptx::mbar_init(tempty_bar(b), 4);
+      ptx::mbar_init(bar(bi_tfull(b)), 1);
+      ptx::mbar_init(bar(bi_tempty(b)), LOADERS);
     }
-    ptx::mbar_init(drain_bar, 1);
+    for (int i = 0; i < CSLOTS; ++i) {
+      ptx::mbar_init(bar(bi_cfull(i)), 32);
+      ptx::mbar_init(bar(bi_cempty(i)), LOADERS);
+    }
+    ptx::mbar_init(bar(bi_drain()), 1);
     ptx::fence_barrier_init();
     ptx::prefetch_tmap(&tmap_w);
     ptx::prefetch_tmap(&tmap_x);
+    // Warm the L2 with the first weight tiles while the previous kernel may
+    // still run (a prefetch only; the loads below come after the wait).
+    int blk = static_cast<int>(u_begin / KB);
+    int kb = static_cast<int>(u_begin - static_cast<int64_t>(blk) * KB);
+    for (int64_t u = u_begin; u < u_end && u < u_begin + DSTAGES;
+         ++u, (++kb == KB ? (kb = 0, ++blk) : 0))
+      ptx::tma_prefetch_2d(&tmap_w, kb * DBK, blk * DBM);
   }
   if (warp == 2) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_holder), DTMEM_COLS);
+    ptx::tmem_alloc(ptx::smem_u32(misc), DTMEM_COLS);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(misc);
+  // From here on the kernel reads what earlier kernels wrote (activation
+  // codes and scales) and writes what they may read (Y, the workspace).
+  ptx::grid_dep_wait();
+  if (threadIdx.x == 0) ptx::grid_dep_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    {
-      uint32_t issued_mask = 0, phase_mask = 0;
-      uint32_t c = 0;
-      int blk = static_cast<int>(u_begin / KB);
-      int kb = static_cast<int>(u_begin - static_cast<int64_t>(blk) * KB);
-      for (int64_t u = u_begin; u < u_end; ++u, ++c, (++kb == KB ? (kb = 0, ++blk) : 0)) {
-        const int s = c % DSTAGES;
-        const uint32_t ph = (c / DSTAGES) & 1u;
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(empty_bar(s), ph ^ 1u))) {
-          if (lane == 0) record_error(args.err, kErrTimeoutProducer);
-          break;
-        }
-        if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(full_bar(s), STAGE_TX);
-          ptx::tma_load_2d(smem_base + DSMEM_W_OFF + s * W_BYTES, &tmap_w, full_bar(s), kb * DBK,
-                           blk * DBM);
-          ptx::tma_load_2d(smem_base + DSMEM_X_OFF + s * X_BYTES, &tmap_x, full_bar(s), kb * DBK, 0);
-        }
-        __syncwarp();
-        issued_mask |= 1u << s;
-        phase_mask = (phase_mask & ~(1u << s)) | (ph << s);
+    uint32_t issued_mask = 0, phase_mask = 0;
+    uint32_t c = 0;
+    int blk = static_cast<int>(u_begin / KB);
+    int kb = static_cast<int>(u_begin - static_cast<int64_t>(blk) * KB);
+    for (int64_t u = u_begin; u < u_end; ++u, ++c, (++kb == KB ? (kb = 0, ++blk) : 0)) {
+      const int s = c % DSTAGES;
+      const uint32_t ph = (c / DSTAGES) & 1u;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(bar(bi_empty(s)), ph ^ 1u))) {
+        if (lane == 0) record_error(args.err, kErrTimeoutProducer);
+        break;
       }
-      if (lane == 0)
-        for (int s = 0; s < DSTAGES; ++s)
-          if (((issued_mask >> s) & 1u) && !ptx::mbar_wait(full_bar(s), (phase_mask >> s) & 1u))
-            record_error(args.err, kErrTimeoutProducer);
+      if (lane == 0) {
+        ptx::mbar_arrive_expect_tx(bar(bi_full(s)), STAGE_TX);
+        ptx::tma_load_2d(smem_base + DSMEM_W_OFF + s * W_BYTES, &tmap_w, bar(bi_full(s)), kb * DBK,
+                         blk * DBM);
+        ptx::tma_load_2d(smem_base + DSMEM_X_OFF + s * X_BYTES, &tmap_x, bar(bi_full(s)), kb * DBK, 0);
+      }
       __syncwarp();
+      issued_mask |= 1u << s;
+      phase_mask = (phase_mask & ~(1u << s)) | (ph << s);
     }
+    // every load issued lands before the CTA may exit
+    if (lane == 0)
+      for (int s = 0; s < DSTAGES; ++s)
+        if (((issued_mask >> s) & 1u) && !ptx::mbar_wait(bar(bi_full(s)), (phase_mask >> s) & 1u))
+          record_error(args.err, kErrTimeoutProducer);
+    __syncwarp();
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     // The whole warp runs the loop (the wait results are made warp-uniform
     // with a vote) and lane 0 issues: measured on B200, a loop run by lane 0
     // alone with a data-dependent exit costs ~600 cycles per chunk.
-    {
-      uint32_t c = 0;
-      bool issued = false;
-      for (int64_t u = u_begin; u < u_end; ++u, ++c) {
-        const int s = c % DSTAGES;
-        const uint32_t sph = (c / DSTAGES) & 1u;
-        const int buf = c % DTBUFS;
-        const uint32_t bph = (c / DTBUFS) & 1u;
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(tempty_bar(buf), bph ^ 1u) &&
-                                         ptx::mbar_wait_spin(full_bar(s), sph))) {
-          if (lane == 0) record_error(args.err, kErrTimeoutMma);
-          break;
-        }
-        ptx::tc_fence_after();
-        if (lane == 0) {
-          const uint32_t w_addr = smem_base + DSMEM_W_OFF + s * W_BYTES;
-          const uint32_t x_addr = smem_base + DSMEM_X_OFF + s * X_BYTES;
-          const uint32_t d = tmem_base + static_cast<uint32_t>(buf * MAX_MPAD);
-#pragma unroll
-          for (int k = 0; k < DBK / DUMMA_K; ++k)
-            ptx::mma_f8f6f4(d, ptx::sdesc_kmajor_sw128(w_addr + k * DUMMA_K),
-                            ptx::sdesc_kmajor_sw128(x_addr + k * DUMMA_K), IDESC, k > 0 ? 1u : 0u);
-          ptx::mma_commit(tfull_bar(buf));
-          ptx::mma_commit(empty_bar(s));
-        }
-        __syncwarp();
-        issued = true;
+    uint32_t c = 0;
+    bool issued = false;
+    for (int64_t u = u_begin; u < u_end; ++u, ++c) {
+      const int s = c % DSTAGES;
+      const uint32_t sph = (c / DSTAGES) & 1u;
+      const int buf = c % DTBUFS;
+      const uint32_t bph = (c / DTBUFS) & 1u;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(bar(bi_tempty(buf)), bph ^ 1u) &&
+                                       ptx::mbar_wait_spin(bar(bi_full(s)), sph))) {
+        if (lane == 0) record_error(args.err, kErrTimeoutMma);
+        break;
       }
-      if (issued && lane == 0) {
-        ptx::mma_commit(drain_bar);
-        if (!ptx::mbar_wait(drain_bar, 0)) record_error(args.err, kErrTimeoutMma);
+      ptx::tc_fence_after();
+      if (lane == 0) {
+        const uint32_t w_addr = smem_base + DSMEM_W_OFF + s * W_BYTES;
+        const uint32_t x_addr = smem_base + DSMEM_X_OFF + s * X_BYTES;
+        const uint32_t d = tmem_base + static_cast<uint32_t>(buf * MAX_MPAD);
+#pragma unroll
+        for (int k = 0; k < DBK / DUMMA_K; ++k)
+          ptx::mma_f8f6f4(d, ptx::sdesc_kmajor_sw128(w_addr + k * DUMMA_K),
+                          ptx::sdesc_kmajor_sw128(x_addr + k * DUMMA_K), IDESC, k > 0 ? 1u : 0u);
+        ptx::mma_commit(bar(bi_tfull(buf)));
+        ptx::mma_commit(bar(bi_empty(s)));
       }
       __syncwarp();
+      issued = true;
     }
-  } else if (warp >= 4) {
-    // ----------------------------------------------------------- promotion
-    const int quarter = warp & 3;
-    const int n_local = quarter * 32 + lane;          // weight row within the block
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int first_blk = static_cast<int>(u_begin / KB);
-    float acc[MPAD];
-#pragma unroll
-    for (int m = 0; m < MPAD; ++m) acc[m] = 0.0f;
-    uint32_t c = 0;
-    bool ok = true;
-
-    // Scales of chunk u: s_w[blk, kb] and the activation scales of tokens
-    // `lane` and `lane + 32`.  They are loaded PF chunks ahead into slot
-    // (u - u_begin) % PF; the loop is unrolled PF times so every slot index
-    // is a compile-time constant and a slot is refilled right after its use
-    // (no register shuffling that would stall on the loads).
+    if (issued && lane == 0) {
+      ptx::mma_commit(bar(bi_drain()));
+      if (!ptx::mbar_wait(bar(bi_drain()), 0)) record_error(args.err, kErrTimeoutMma);
+    }
+    __syncwarp();
+  } else if (warp == 3) {
+    // ------------------------------------------------------ scale products
+    // prods[slot][m] = s_w[blk, kb] * s_a[m, kb] for every chunk of the
+    // range, up to CSLOTS chunks ahead of the promotion warps.  Lane l
+    // covers tokens l and l + 32.  The scales of a chunk are loaded PF
+    // chunks ahead (L2 path: another kernel wrote them) into a register slot
+    // that is refilled right after its use.
     constexpr int PF = 4;
     float pw[PF], plo[PF], phi[PF];
     auto load_scales = [&](int64_t uu, float& w, float& lo, float& hi) {
+      w = lo = hi = 0.0f;
       if (uu < u_end) {
         const int b = static_cast<int>(uu / KB);
         const int k = static_cast<int>(uu - static_cast<int64_t>(b) * KB);
-        w = __ldg(args.s_w + static_cast<int64_t>(b) * KB + k);
-        lo = lane < args.M ? __ldg(args.s_a + static_cast<int64_t>(lane) * KB + k) : 0.0f;
-        hi = (MPAD > 32 && lane + 32 < args.M)
-                 ? __ldg(args.s_a + static_cast<int64_t>(lane + 32) * KB + k)
-                 : 0.0f;
+        w = __ldcg(args.s_w + static_cast<int64_t>(b) * KB + k);
+        if (lane < args.M) lo = __ldcg(args.s_a + static_cast<int64_t>(lane) * KB + k);
+        if (MPAD > 32 && lane + 32 < args.M)
+          hi = __ldcg(args.s_a + static_cast<int64_t>(lane + 32) * KB + k);
       }
     };
 #pragma unroll
-    for (int i = 0; i < PF; ++i) {
-      pw[i] = plo[i] = phi[i] = 0.0f;
-      load_scales(u_begin + i, pw[i], plo[i], phi[i]);
-    }
-
-    int blk = first_blk;
-    int kb = static_cast<int>(u_begin - static_cast<int64_t>(first_blk) * KB) - 1;
-    for (int64_t u0 = u_begin; u0 < u_end; u0 += PF) {
+    for (int i = 0; i < PF; ++i) load_scales(u_begin + i, pw[i], plo[i], phi[i]);
+    uint32_t c = 0;
+    bool ok = true;
+    for (int64_t u0 = u_begin; u0 < u_end && ok; u0 += PF) {
 #pragma unroll
       for (int i = 0; i < PF; ++i) {
         const int64_t u = u0 + i;
         if (u >= u_end) break;
-        if (++kb == KB) {
-          kb = 0;
-          ++blk;
-        }
-        const float sw = pw[i], sa_lo = plo[i], sa_hi = phi[i];
+        const float cw = pw[i], clo = plo[i], chi = phi[i];
         load_scales(u + PF, pw[i], plo[i], phi[i]);
-        const int buf = c % DTBUFS;
-        const uint32_t bph = (c / DTBUFS) & 1u;
+        const int slot = c % CSLOTS;
+        const uint32_t ph = (c / CSLOTS) & 1u;
         ++c;
-        // After a timed-out wait this warp stops touching TMEM but keeps
-        // walking its range, so that every named barrier below is reached
-        // by all four promotion warps.
-        if (ok && !ptx::mbar_wait_spin(tfull_bar(buf), bph)) {
-          record_error(args.err, kErrTimeoutEpilogue);
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(bar(bi_cempty(slot)), ph ^ 1u))) {
+          if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
           ok = false;
+          break;
         }
-        if (ok) {
-          ptx::tc_fence_after();
-          uint32_t v[MPAD];
-#pragma unroll
-          for (int j = 0; j < MPAD / 16; ++j)
-            ptx::tmem_ld_32x32b_x16(
-                tmem_base + lane_off + static_cast<uint32_t>(buf * MAX_MPAD + j * 16),
-                *reinterpret_cast<uint32_t(*)[16]>(&v[j * 16]));
-          ptx::tmem_ld_wait();
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
-#pragma unroll
-          for (int m = 0; m < MPAD; ++m) {
-            const float sa = __shfl_sync(0xffffffffu, m < 32 ? sa_lo : sa_hi, m & 31);
-            acc[m] = __fmaf_rn(__uint_as_float(v[m]), sw * sa, acc[m]);
-          }
-        }
-        if (kb == KB - 1 || u + 1 == u_end) {
-          // end of this block's segment
-          const int64_t blk_u0 = static_cast<int64_t>(blk) * KB;
-          const int64_t y_off = static_cast<int64_t>(blk) * 128 + n_local;
-          if (blk_u0 >= u_begin && kb == KB - 1) {
-            // the whole block was accumulated by this CTA: write bf16 directly
-#pragma unroll
-            for (int m = 0; m < MPAD; ++m)
-              if (m < args.M) args.y[static_cast<int64_t>(m) * args.N + y_off] = __float2bfloat16_rn(acc[m]);
-          } else {
-            float* dst = args.partial +
-                         (static_cast<int64_t>(g) * args.maxseg + (blk - first_blk)) * (MPAD * 128);
-#pragma unroll
-            for (int m = 0; m < MPAD; ++m) dst[m * 128 + n_local] = acc[m];
-            // publish the partial and count this CTA in; the last one reduces.
-            // The barrier orders every thread's stores before one thread's
-            // fence + atomic (the fence is cumulative), as a grid-wide
-            // barrier does; the last CTA fences again before reading.
-            ptx::named_barrier_sync(1, 128);
-            __shared__ int last_flag;
-            const int g_lo = static_cast<int>(((blk_u0 + 1) * args.G - 1) / args.units);
-            const int g_hi = static_cast<int>(((blk_u0 + KB) * args.G - 1) / args.units);
-            if (threadIdx.x == 128) {
-              __threadfence();
-              last_flag = atomicAdd(args.counters + blk, 1) == g_hi - g_lo;
-              if (last_flag) __threadfence();
-            }
-            ptx::named_barrier_sync(1, 128);
-            if (last_flag) {
-              // sum the block's partials in increasing CTA order; the loads
-              // of UR partials are in flight together
-              constexpr int UR = MPAD <= 16 ? 4 : (MPAD <= 32 ? 2 : 1);
-#pragma unroll
-              for (int m = 0; m < MPAD; ++m) acc[m] = 0.0f;
-              for (int gg = g_lo; gg <= g_hi; gg += UR) {
-                float t[UR][MPAD];
-#pragma unroll
-                for (int r = 0; r < UR; ++r) {
-                  const int gi = gg + r <= g_hi ? gg + r : g_hi;
-                  const int fb = static_cast<int>(range_start(gi, args.units, args.G) / KB);
-                  const float* src = args.partial +
-                                     (static_cast<int64_t>(gi) * args.maxseg + (blk - fb)) * (MPAD * 128) +
-                                     n_local;
-#pragma unroll
-                  for (int m = 0; m < MPAD; ++m) t[r][m] = __ldcg(src + m * 128);
-                }
-#pragma unroll
-                for (int r = 0; r < UR; ++r)
-                  if (gg + r <= g_hi) {
-#pragma unroll
-                    for (int m = 0; m < MPAD; ++m) acc[m] += t[r][m];
-                  }
-              }
-#pragma unroll
-              for (int m = 0; m < MPAD; ++m)
-                if (m < args.M) args.y[static_cast<int64_t>(m) * args.N + y_off] = __float2bfloat16_rn(acc[m]);
-            }
-          }
-#pragma unroll
-          for (int m = 0; m < MPAD; ++m) acc[m] = 0.0f;
-        }
+        float* cr = prods + slot * MAX_MPAD;
+        cr[lane] = cw * clo;
+        if (MPAD > 32) cr[32 + lane] = cw * chi;
+        ptx::mbar_arrive(bar(bi_cfull(slot)));
       }
     }
+  } else if (warp >= 4) {
+    // ----------------------------------------------------------- promotion
+    PromoCtx cx;
+    cx.smem_base = smem_base;
+    cx.tmem_base = tmem_base;
+    cx.prods = prods;
+    cx.last_flag = reinterpret_cast<volatile int*>(misc + 1);
+    cx.u_begin = u_begin;
+    cx.u_end = u_end;
+    cx.g = g;
+    cx.quarter = warp & 3;
+    cx.lane = lane;
+    if (warp < 8)
+      decode_promote<MPAD, NC0, 0>(args, cx);
+    else
+      decode_promote<MPAD, NC1, NC0>(args, cx);
   }
 
   ptx::tc_fence_before();
@@ -365,20 +491,56 @@ DecodeGeometry decode_geometry(int64_t M, int64_t N, int64_t K, int sm_count) {
   return d;
 }
 
+// Tag of one launch: a per-process random start advanced by an odd constant
+// per launch, kept to 48 bits and never zero.  A graph replays its launches
+// with their tags; that is sound because every launch that completes leaves
+// its counters at zero.
+unsigned long long next_launch_tag() {
+  static std::atomic<unsigned long long> seq{0};
+  static const unsigned long long salt = [] {
+    unsigned long long x = static_cast<unsigned long long>(
+        std::chrono::high_resolution_clock::now().time_since_epoch().count());
+    x ^= reinterpret_cast<uintptr_t>(&seq) * 0x9E3779B97F4A7C15ull;
+    x ^= x >> 29;
+    x *= 0xBF58476D1CE4E5B9ull;
+    x ^= x >> 32;
+    return x;
+  }();
+  const unsigned long long t =
+      (salt + 0x9E3779B97F4A7C15ull * (seq.fetch_add(1, std::memory_order_relaxed) + 1)) &
+      ((1ull << 48) - 1);
+  return t ? t : 1ull;
+}
+
 template <int MPAD>
 cudaError_t launch_decode_t(const CUtensorMap& tw, const CUtensorMap& tx, const DecodeArgs& a,
                             cudaStream_t st) {
-  static cudaError_t attr = cudaFuncSetAttribute(
-      decode_kernel<MPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, DSMEM_BYTES);
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t status[kMaxDevices];
+  const cudaError_t attr = once_per_device(once, status, [](int) {
+    return cudaFuncSetAttribute(decode_kernel<MPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                DSMEM_BYTES);
+  });
   if (attr != cudaSuccess) return attr;
-  decode_kernel<MPAD><<<a.G, DNUM_THREADS, DSMEM_BYTES, st>>>(tw, tx, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.G), 1, 1);
+  cfg.blockDim = dim3(DNUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = DSMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  set_programmatic_serialization(at[0]);
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<MPAD>, tw, tx, a);
 }
 
 }  // namespace
 
-// Workspace: NB block counters (rounded up to 256 bytes), then the partials.
-size_t decode_counter_bytes(int64_t N) { return static_cast<size_t>(((N / 128) * 4 + 255) / 256 * 256); }
+// Workspace: NB 64-bit block counters (rounded up to 256 bytes), then the
+// partials.
+size_t decode_counter_bytes(int64_t N) {
+  return static_cast<size_t>(((N / 128) * 8 + 255) / 256 * 256);
+}
 
 size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count) {
   const DecodeGeometry d = decode_geometry(M, N, K, sm_count);
@@ -397,18 +559,16 @@ cudaError_t launch_block_linear_decode(const void* q_a, const float* s_a, const 
   a.s_a = s_a;
   a.s_w = s_w;
   a.y = static_cast<__nv_bfloat16*>(y);
-  a.counters = static_cast<int*>(workspace);
+  a.counters = static_cast<unsigned long long*>(workspace);
   a.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + decode_counter_bytes(N));
+  a.tag = next_launch_tag();
+  a.units = d.units;
   a.N = static_cast<int>(N);
   a.M = static_cast<int>(M);
-  a.Mpad = d.Mpad;
   a.KB = static_cast<int>(K / 128);
-  a.units = d.units;
   a.G = d.G;
   a.maxseg = d.maxseg;
   a.err = dev.error_flag;
-  cudaError_t e = cudaMemsetAsync(workspace, 0, decode_counter_bytes(N), st);
-  if (e != cudaSuccess) return e;
   switch (d.Mpad) {
     case 16: return launch_decode_t<16>(tw, tx, a, st);
     case 32: return launch_decode_t<32>(tw, tx, a, st);

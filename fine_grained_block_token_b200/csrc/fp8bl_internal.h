@@ -7,8 +7,37 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <mutex>
 
 namespace fp8bl {
+
+// Per-device state is kept in arrays indexed by the device ordinal.
+constexpr int kMaxDevices = 64;
+
+// Runs `init(dev)` once for each device -- the current device at the call --
+// and returns the status it recorded for that device (kernel attributes such
+// as the shared-memory opt-in belong to one device).  *dev_out receives the
+// ordinal when given.
+template <class Init>
+cudaError_t once_per_device(std::once_flag* flags, cudaError_t* status, Init init,
+                            int* dev_out = nullptr) {
+  int dev = -1;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(flags[dev], [&] { status[dev] = init(dev); });
+  if (dev_out) *dev_out = dev;
+  return status[dev];
+}
+
+// Launch attribute for programmatic dependent launch: the kernel may begin
+// while the previous kernel on the stream finishes; every kernel launched
+// this way calls ptx::grid_dep_wait() before touching global memory that
+// another kernel writes or reads.
+inline void set_programmatic_serialization(cudaLaunchAttribute& a) {
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+}
 
 struct DeviceInfo {
   int device = -1;

@@ -496,13 +496,15 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
 // One-time set-up: opt in to the dynamic shared memory and find how many
 // clusters of CL CTAs fit on the device at once.
 cudaError_t ensure_fused_ready(int* max_clusters) {
-  static cudaError_t st = cudaSuccess;
-  static int clusters = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    st = cudaFuncSetAttribute(gemm_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              SMEM_BYTES);
-    if (st != cudaSuccess) return;
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t status[kMaxDevices];
+  static int clusters_of[kMaxDevices];
+  int dev = 0;
+  const cudaError_t r = once_per_device(once, status, [](int d) {
+    int& clusters = clusters_of[d];
+    cudaError_t st = cudaFuncSetAttribute(gemm_fused_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (st != cudaSuccess) return st;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(CL, 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -516,9 +518,10 @@ cudaError_t ensure_fused_ready(int* max_clusters) {
     cfg.numAttrs = 1;
     st = cudaOccupancyMaxActiveClusters(&clusters, gemm_fused_kernel, &cfg);
     if (st == cudaSuccess && clusters < 1) st = cudaErrorInvalidConfiguration;
-  });
-  *max_clusters = clusters;
-  return st;
+    return st;
+  }, &dev);
+  *max_clusters = r == cudaSuccess ? clusters_of[dev] : 0;
+  return r;
 }
 
 }  // namespace

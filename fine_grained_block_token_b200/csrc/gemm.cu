@@ -283,13 +283,12 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
 }
 
 cudaError_t ensure_smem_attr() {
-  static cudaError_t st = cudaSuccess;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    st = cudaFuncSetAttribute(gemm_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              SMEM_BYTES);
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t st[kMaxDevices];
+  return once_per_device(once, st, [](int) {
+    return cudaFuncSetAttribute(gemm_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES);
   });
-  return st;
 }
 
 }  // namespace

@@ -471,13 +471,15 @@ gemm_rowwise_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
 }
 
 cudaError_t ensure_pair_ready(int* max_clusters) {
-  static cudaError_t st = cudaSuccess;
-  static int clusters = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    st = cudaFuncSetAttribute(gemm_rowwise_pair_kernel,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, PSMEM_BYTES);
-    if (st != cudaSuccess) return;
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t status[kMaxDevices];
+  static int clusters_of[kMaxDevices];
+  int dev = 0;
+  const cudaError_t r = once_per_device(once, status, [](int d) {
+    int& clusters = clusters_of[d];
+    cudaError_t st = cudaFuncSetAttribute(gemm_rowwise_pair_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, PSMEM_BYTES);
+    if (st != cudaSuccess) return st;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -491,19 +493,19 @@ cudaError_t ensure_pair_ready(int* max_clusters) {
     cfg.numAttrs = 1;
     st = cudaOccupancyMaxActiveClusters(&clusters, gemm_rowwise_pair_kernel, &cfg);
     if (st == cudaSuccess && clusters < 1) st = cudaErrorInvalidConfiguration;
-  });
-  *max_clusters = clusters;
-  return st;
+    return st;
+  }, &dev);
+  *max_clusters = r == cudaSuccess ? clusters_of[dev] : 0;
+  return r;
 }
 
 cudaError_t ensure_smem_attr() {
-  static cudaError_t st = cudaSuccess;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    st = cudaFuncSetAttribute(gemm_rowwise_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              SMEM_BYTES);
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t st[kMaxDevices];
+  return once_per_device(once, st, [](int) {
+    return cudaFuncSetAttribute(gemm_rowwise_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES);
   });
-  return st;
 }
 
 }  // namespace

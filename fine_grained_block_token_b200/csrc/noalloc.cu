@@ -11,17 +11,18 @@
 // load until the process exits.
 //
 // Host code must not use the array's name as a device address (on the host
-// it names a stand-in object): the device address is fetched once per
-// device with cudaGetSymbolAddress, on the first call made while that
-// device is current, and cached.  Because that set-up runs a CUDA runtime
-// query, the first call on each device should come before any stream
-// capture.
+// it names a stand-in object): the device address is fetched with
+// cudaGetSymbolAddress on the first call made while a device is current,
+// and cached once the lookup has succeeded (a failed lookup is retried by
+// the next call).  Because that set-up runs a CUDA runtime query, the first
+// call on each device should come before any stream capture.
 //
 // Every call on a device shares the same array and leaves its contents
-// behind; the counters that must start at zero are cleared (with
-// cudaMemsetAsync, which allocates nothing) on the caller's stream at the
-// start of every call.  Two calls whose GPU work overlaps -- on different
-// streams without ordering between them -- race on the array.
+// behind.  Nothing needs clearing between calls: the decode schedule's
+// block counters carry a per-launch tag, a count under another tag reads as
+// zero, and a completed launch leaves them at zero.  Two calls whose GPU
+// work overlaps -- on different streams without ordering between them --
+// race on the array.
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <mutex>
@@ -40,21 +41,26 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 
-constexpr int kMaxDevices = 64;
 void* g_scratch_dev_ptr[kMaxDevices];
-cudaError_t g_scratch_status[kMaxDevices];
-std::once_flag g_scratch_once[kMaxDevices];
+std::mutex g_scratch_mutex;
 
-// Device address of the scratch array on the current device (set-up on the
-// first call per device).
+// Device address of the scratch array on the current device.  The first
+// call per device looks it up; only a successful lookup is cached, so a
+// failed one (for instance a call made while a stream capture forbids the
+// query) is retried on the next call instead of failing for good.
 cudaError_t scratch_address(int dev, void** out) {
-  std::call_once(g_scratch_once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_dev_ptr[dev]) {
     void* p = nullptr;
-    g_scratch_status[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    g_scratch_dev_ptr[dev] = g_scratch_status[dev] == cudaSuccess ? p : nullptr;
-  });
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      *out = nullptr;
+      return e != cudaSuccess ? e : cudaErrorInvalidSymbol;
+    }
+    g_scratch_dev_ptr[dev] = p;
+  }
   *out = g_scratch_dev_ptr[dev];
-  return g_scratch_status[dev];
+  return cudaSuccess;
 }
 
 bool is_aligned(const void* p, uintptr_t a) {

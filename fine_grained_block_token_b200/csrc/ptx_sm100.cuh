@@ -130,6 +130,17 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   return p;
 }
 
+// L2 prefetch of one 2-D tile of a tensor map (no shared-memory
+// destination, no completion).  Only warms the L2; it is safe to issue
+// before the data's producer has finished, since a later write updates the
+// line in L2 and the real load that follows reads the new value.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* m, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // 2-D tiled store shared -> global (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int32_t c0,
                                              int32_t c1) {
@@ -156,6 +167,21 @@ __device__ __forceinline__ void bulk_wait_group() {
 // (TMA store source, tcgen05.mma operands) after this fence.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------- programmatic dependent launch
+//
+// A kernel launched with the programmatic-serialization attribute may start
+// while the previous kernel on its stream is still running.  grid_dep_wait()
+// blocks until that kernel has completed and its memory writes are visible;
+// a kernel calls it before its first access to global memory that another
+// kernel may write or read.  Without the attribute it returns at once.
+// grid_dep_launch() lets the next such kernel start launching.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------- tensor memory

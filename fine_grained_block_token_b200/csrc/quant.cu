@@ -22,6 +22,7 @@
 #include <cuda_runtime.h>
 
 #include "fp8bl_internal.h"
+#include "ptx_sm100.cuh"
 #include "quant_math.cuh"
 
 namespace fp8bl {
@@ -87,6 +88,8 @@ template <int kMode>
 __global__ void __launch_bounds__(kAqThreads, 4)
 act_quant_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, void* __restrict__ s,
                  int64_t num_groups, const float* __restrict__ s_given) {
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch();
   const float given = kMode == kModeStatic ? __ldg(s_given) : 0.0f;
   const int lane = threadIdx.x & 31;
   const int half = lane >> 4;
@@ -143,6 +146,8 @@ template <int kMode>
 __global__ void __launch_bounds__(kAqThreads, 4)
 act_quant32_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, void* __restrict__ s,
                    int64_t num_groups, const float* __restrict__ s_given) {
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch();
   const float given = kMode == kModeStatic ? __ldg(s_given) : 0.0f;
   const int lane = threadIdx.x & 31;
   const int sub = lane >> 3;      // group within the warp's 4
@@ -226,6 +231,22 @@ weight_quant_kernel(const uint4* __restrict__ w, uint2* __restrict__ q, void* __
 
 namespace {
 
+// Launch with programmatic stream serialization (the kernels wait for the
+// previous kernel before their first global access).
+template <class Kernel, class... Args>
+cudaError_t launch_pdl(Kernel k, int blocks, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(kAqThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  set_programmatic_serialization(at[0]);
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, args...);
+}
+
 template <int kMode>
 cudaError_t act_quant(const void* x, int64_t M, int64_t K, void* q, void* s, int sm_count,
                       cudaStream_t st, const float* s_given = nullptr) {
@@ -237,10 +258,8 @@ cudaError_t act_quant(const void* x, int64_t M, int64_t K, void* q, void* s, int
     const int64_t blocks_needed = (warps_needed + (kAqThreads / 32) - 1) / (kAqThreads / 32);
     const int64_t max_blocks = static_cast<int64_t>(sm_count) * 4;
     const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
-    act_quant32_kernel<kMode><<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
-                                                             static_cast<uint4*>(q), s, groups,
-                                                             s_given);
-    return cudaGetLastError();
+    return launch_pdl(act_quant32_kernel<kMode>, blocks, st, static_cast<const uint4*>(x),
+                      static_cast<uint4*>(q), s, groups, s_given);
   }
   const int64_t pairs = (groups + 1) / 2;
   const int64_t warps_needed = (pairs + kAqUnroll - 1) / kAqUnroll;
@@ -249,9 +268,8 @@ cudaError_t act_quant(const void* x, int64_t M, int64_t K, void* q, void* s, int
   // loop inside the kernel.
   const int64_t max_blocks = static_cast<int64_t>(sm_count) * 4;
   const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
-  act_quant_kernel<kMode><<<blocks, kAqThreads, 0, st>>>(static_cast<const uint4*>(x),
-                                                         static_cast<uint2*>(q), s, groups, s_given);
-  return cudaGetLastError();
+  return launch_pdl(act_quant_kernel<kMode>, blocks, st, static_cast<const uint4*>(x),
+                    static_cast<uint2*>(q), s, groups, s_given);
 }
 
 template <int kMode>

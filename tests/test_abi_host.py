@@ -248,7 +248,7 @@ def test_decode_workspace_covers_every_partial_slot(lib, seed):
         KB, U = K // 128, (N // 128) * (K // 128)
         G = max(1, min(148, U // ((KB + 7) // 8)))
         mpad = (M + 15) // 16 * 16
-        counters = ((N // 128) * 4 + 255) // 256 * 256
+        counters = ((N // 128) * 8 + 255) // 256 * 256     # 64-bit tagged counters
         ws = f(M, N, K)
         per_slot = G * mpad * 128 * 4
         assert ws > counters and (ws - counters) % per_slot == 0, (M, N, K, ws)
@@ -271,3 +271,24 @@ def test_fused_workspace_holds_the_staged_activations(lib):
         assert fw(M, N, K) >= up(ws(M, N, K)) + up(M * K) + up(M * (K // 128) * 4), (M, N, K)
     for M, N, K in [(65, 4096, 4096), (8192, 7168, 18432)]:
         assert fw(M, N, K) == 0 and ws(M, N, K) == 0
+
+
+def test_noalloc_scratch_covers_the_decode_workloads(lib):
+    """The no-allocation entry point serves a decode shape only while its
+    schedule's scratch fits the built-in array (FP8BL_NOALLOC_SCRATCH_BYTES,
+    16 MiB).  Every Llama-3-8B and DeepSeek-V3 linear at the decode token
+    counts must fit, so that a change to the schedule's geometry cannot
+    silently turn those shapes into FP8BL_ERR_WORKSPACE.  (Planned for 148
+    SMs, the B200's count, as the library does without a GPU.)"""
+    f = lib.fp8_block_linear_workspace_bytes
+    f.argtypes = [ctypes.c_int64] * 3
+    f.restype = ctypes.c_size_t
+    hdr = open(os.path.join(ROOT, "include", "fp8bl.h")).read()
+    m = re.search(r"#define FP8BL_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", hdr)
+    limit = int(m.group(1)) << int(m.group(2))
+    llama3_8b = [(4096, 4096), (1024, 4096), (28672, 4096), (4096, 14336)]
+    deepseek_v3 = [(18432, 7168), (7168, 18432), (2048, 7168), (7168, 2048), (4096, 7168)]
+    for M in (1, 8, 32, 64):
+        for N, K in llama3_8b + deepseek_v3:
+            need = f(M, N, K)
+            assert 0 < need <= limit, (M, N, K, need, limit)

@@ -91,7 +91,7 @@ def test_full_size_prefill(fp8, which):
 
 
 @pytest.mark.parametrize("name", ["qo", "kv", "gate_up", "down"])
-@pytest.mark.parametrize("M", [1, 8, 64])
+@pytest.mark.parametrize("M", [1, 8, 32, 64])
 def test_full_size_decode(fp8, name, M):
     xb, wb = wl.llama3_decode(M, name)
     y, R, _ = _run(fp8, xb, wb)
@@ -159,7 +159,7 @@ def test_decode_workspace_too_small(fp8):
     assert ei.value.status == 7
 
 
-@pytest.mark.parametrize("M", [512, 16384])
+@pytest.mark.parametrize("M", [512, 1024, 2048, 4096, 8192, 16384])
 def test_full_size_sweep_unfused_and_fused(fp8, M):
     """Sweep workload: X [M, 7168] Student-t(3) with outlier channels and
     zeroed groups against W [2048, 7168]; the fused entry point must equal the
@@ -211,4 +211,83 @@ def test_fused_repeated_runs_bit_identical(fp8, M, N, K):
         fp8.block_linear_fused(x, q_w, s_w, y2)
         torch.cuda.synchronize()
         assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), (M, N, K, rep)
+    fp8.check()
+
+
+def test_decode_workspace_needs_no_clearing(fp8):
+    """The decode schedule's block counters carry a per-launch tag, so a
+    workspace holding leftover bytes -- all ones, random bytes, or another
+    shape's leftovers -- gives the same Y, bit for bit, as a fresh one, and
+    calls that reuse one workspace across shapes stay exact."""
+    shapes = [(1, 4096, 4096), (64, 1024, 4096), (17, 2048, 3072)]
+    runs = []
+    size = 0
+    for M, N, K in shapes:
+        xb = wl.normal((M, K), 1.0, 0, 7 + M)
+        wb = wl.normal((N, K), 0.02, 1, 7 + M)
+        x, w = to_dev(xb), to_dev(wb)
+        q_a, s_a = fp8.quant_act(x)
+        q_w, s_w = fp8.quant_weight(w)
+        size = max(size, fp8.workspace_bytes(M, N, K))
+        runs.append((q_a, s_a, q_w, s_w, M, N, K))
+    shared = torch.empty(size, dtype=torch.uint8, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(11)
+    for q_a, s_a, q_w, s_w, M, N, K in runs:
+        ref = fp8.block_linear(q_a, s_a, q_w, s_w)
+        R = oracle.block_linear(u8(q_a), f32(s_a), u8(q_w), f32(s_w), nthreads=8)
+        check_gemm(f32(ref), R, f"decode {M}x{N}x{K}")
+        for fill in ("ones", "random", "reuse", "reuse"):
+            if fill == "ones":
+                shared.fill_(255)
+            elif fill == "random":
+                shared.random_(0, 256, generator=g)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            fp8.block_linear(q_a, s_a, q_w, s_w, y, shared[:fp8.workspace_bytes(M, N, K)])
+            torch.cuda.synchronize()
+            assert torch.equal(y.view(torch.int16), ref.view(torch.int16)), (M, N, K, fill)
+    fp8.check()
+
+
+def test_decode_graph_replay_bit_identical(fp8):
+    """A CUDA graph replays its decode launches with the tags they were
+    captured with; every completed launch leaves its counters at zero, so
+    replays give the eager result bit for bit.  The graph holds the
+    activation quantizer and the decode linear back to back (both launched
+    with programmatic serialization), for two shapes on one workspace."""
+    items = []
+    size = 0
+    for M, N, K in [(8, 4096, 4096), (64, 28672, 4096)]:
+        x = to_dev(wl.normal((M, K), 1.0, 0, 21 + M))
+        w = to_dev(wl.normal((N, K), 0.02, 1, 21 + M))
+        q_w, s_w = fp8.quant_weight(w)
+        q_a, s_a = fp8.quant_act(x)
+        ref = fp8.block_linear(q_a, s_a, q_w, s_w)
+        size = max(size, fp8.workspace_bytes(M, N, K))
+        items.append(dict(x=x, q_w=q_w, s_w=s_w, q_a=torch.empty_like(q_a), s_a=torch.empty_like(s_a),
+                          y=torch.empty_like(ref), ref=ref, M=M, N=N, K=K))
+    ws = torch.empty(size, dtype=torch.uint8, device="cuda")
+
+    def step():
+        for it in items:
+            fp8.quant_act(it["x"], it["q_a"], it["s_a"])
+            fp8.block_linear(it["q_a"], it["s_a"], it["q_w"], it["s_w"], it["y"],
+                             ws[:fp8.workspace_bytes(it["M"], it["N"], it["K"])])
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for rep in range(4):
+        for it in items:
+            it["y"].fill_(0)
+        graph.replay()
+        torch.cuda.synchronize()
+        for it in items:
+            assert torch.equal(it["y"].view(torch.int16), it["ref"].view(torch.int16)), (it["M"], rep)
+    del graph
     fp8.check()

@@ -3,10 +3,12 @@ on scratch memory built into the library instead of a caller workspace (for
 callers that cannot allocate device memory where they run the layer).
 
 The entry point is called through the C ABI and its output is compared with
-fp8_block_linear's (same inputs, caller workspace) using the GEMM tolerance
-of the other tests, on two calls in a row: the second call runs on scratch
-that still holds the first call's contents.  Sizes beyond what the built-in
-scratch or the decode schedule cover must be refused.
+fp8_block_linear's (same inputs, caller workspace) on two calls in a row:
+the second call runs on scratch that still holds the first call's contents.
+Both run the same deterministic decode schedule, so the outputs must be
+equal bit for bit; one shape is also held to the oracle within the GEMM
+tolerance of the other tests.  Sizes beyond what the built-in scratch or
+the decode schedule cover must be refused.
 
 This file sorts last so that a run that stops at the first failure has
 already run every other test; it also passes on its own in a new process.
@@ -18,7 +20,7 @@ import pytest
 import torch
 
 import workloads as wl
-from tests.parity import FRO_REL, PW_REL, PW_RMS
+from tests.parity import FRO_REL, PW_REL, PW_RMS, check_gemm
 
 pytestmark = pytest.mark.gpu
 
@@ -61,7 +63,27 @@ def test_noalloc_matches_workspace_path_twice(fp8, M, N, K):
         y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         assert _c_call(fp8, q_a, s_a, q_w, s_w, y, M, N, K) == 0
         fp8.check()
-        _within_tolerance(y, ref, f"noalloc call {call} {M}x{N}x{K}")
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16)), \
+            f"noalloc call {call} {M}x{N}x{K} differs from fp8_block_linear"
+
+
+def test_noalloc_against_the_oracle(fp8):
+    """One decode shape with ragged tokens and zeroed weight blocks: the
+    no-allocation output meets the GEMM tolerance against the oracle's fp64
+    result computed from the same codes and scales."""
+    import oracle
+    M, N, K = 37, 2048, 3072
+    xb = wl.normal((M, K), 1.0, 0, 91)
+    wb = wl.zero_blocks(wl.normal((N, K), 0.02, 1, 91), 0.05)
+    x, w = wl.to_torch_bf16(xb).cuda(), wl.to_torch_bf16(wb).cuda()
+    q_a, s_a = fp8.quant_act(x)
+    q_w, s_w = fp8.quant_weight(w)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    assert _c_call(fp8, q_a, s_a, q_w, s_w, y, M, N, K) == 0
+    fp8.check()
+    R = oracle.block_linear(q_a.view(torch.uint8).cpu().numpy(), s_a.cpu().numpy(),
+                            q_w.view(torch.uint8).cpu().numpy(), s_w.cpu().numpy(), nthreads=8)
+    check_gemm(y.float().cpu().numpy(), R, "noalloc vs oracle")
 
 
 def test_noalloc_binding_allocates_nothing(fp8):

@@ -124,9 +124,19 @@ def tiny():
 
 
 def llama3_decode(M: int, name: str):
+    return llama3_decode_x(M, name), llama3_decode_w(name)
+
+
+def llama3_decode_x(M: int, name: str):
+    """X [M, K] of one decode linear (the same draw as llama3_decode)."""
+    _, K = LLAMA3_8B_LINEARS[name]
+    return normal((M, K), 1.0, SEED_X, hash_name(name))
+
+
+def llama3_decode_w(name: str):
+    """W [N, K] of one decode linear; it does not depend on M."""
     N, K = LLAMA3_8B_LINEARS[name]
-    salt = hash_name(name)
-    return normal((M, K), 1.0, SEED_X, salt), normal((N, K), 0.02, SEED_W, salt)
+    return normal((N, K), 0.02, SEED_W, hash_name(name))
 
 
 def llama3_prefill(name: str, M: int = PREFILL_M):
