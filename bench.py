@@ -889,7 +889,20 @@ def legs_json(legs, world, args, hbm_peak, fp8_peak, peak_src):
     the same thing)."""
     out = {}
     cpu_ok = world == 1 and not args.no_cpu
-    dec, lay, acts, wsets = legs["decode"]
+    if "decode" in legs:
+        out.update(decode_json(legs["decode"], cpu_ok, hbm_peak, peak_src))
+    if "deepseek_mlp" in legs:
+        out.update(deepseek_json(legs["deepseek_mlp"], world, args, cpu_ok, fp8_peak))
+    if "sweep" in legs:
+        out.update(sweep_json(legs["sweep"], cpu_ok, hbm_peak, fp8_peak))
+    if "tiny" in legs:
+        out.update(tiny_json(legs["tiny"], cpu_ok))
+    return out
+
+
+def decode_json(leg, cpu_ok, hbm_peak, peak_src):
+    out = {}
+    dec, lay, acts, wsets = leg
     lin = {}
     tb, tm = 0.0, 0.0
     for k, d in dec.items():
@@ -917,7 +930,12 @@ def legs_json(legs, world, args, hbm_peak, fp8_peak, peak_src):
                    "layer": "one decoder layer = 4 activation quantizations + q, k, v, o, gate+up, down; "
                             "4 layers' weight copies per replay"},
         "cpu_baseline": dcpu, "parity": dpar}
-    items, ds = legs["deepseek_mlp"]
+    return out
+
+
+def deepseek_json(leg, world, args, cpu_ok, fp8_peak):
+    out = {}
+    items, ds = leg
     tf = ds["flops"] * args.steps / (ds["gemm_ms"] * 1e-3) / 1e12
     step_tf = whole_job_rate(world, ds["flops"], args.steps, ds["ms"]) / 1e12
     dcpu, dpar = rows_oracle_check(items, 4) if cpu_ok else (None, None)
@@ -932,7 +950,12 @@ def legs_json(legs, world, args, hbm_peak, fp8_peak, peak_src):
         "fused": {"value": whole_job_rate(world, ds["flops"], args.steps, ds["fused_ms"]) / 1e12,
                   "vs_two_call": ds["ms"] / ds["fused_ms"], "identical_to_two_call": ds["identical"]},
         "cpu_baseline": dcpu, "parity": dpar}
-    sw, sitems = legs["sweep"]
+    return out
+
+
+def sweep_json(leg, cpu_ok, hbm_peak, fp8_peak):
+    out = {}
+    sw, sitems = leg
     per = {}
     for k, d in sw.items():
         q_gbs = d["qbytes"] / (d["quant_ms"] * 1e-3) / 1e9
@@ -948,7 +971,11 @@ def legs_json(legs, world, args, hbm_peak, fp8_peak, peak_src):
         "config": {"workload": "sweep", "M": list(wl.SWEEP_M), "N": wl.SWEEP_N, "K": wl.SWEEP_K,
                    "l2": "each launch reads another copy of its operands (a rotation moves >= 2.5 x L2)"},
         "per_M": per, "cpu_baseline": scpu, "parity": spar}
-    t = legs["tiny"]
+    return out
+
+
+def tiny_json(t, cpu_ok):
+    out = {}
     out["tiny"] = {"us_per_linear": t["ms"] * 1e3, "unit": "us (quant_act + block_linear)",
                    "TFLOPs": t["flops"] / (t["ms"] * 1e-3) / 1e12,
                    "config": {"workload": "tiny", "M": 32, "N": 256, "K": 512,
@@ -1204,13 +1231,18 @@ def run_ours(args):
             variants[name] = dict(items=v_items, ms=v_ms, gemm_ms=v_gemm_ms, kernel=sp["kernel"])
     # ---- the other workloads of the build, on the same line
     legs = {}
-    run_legs = args.workload == "llama3_prefill" and not args.no_legs
+    want = set(args.legs.split(",")) if args.legs else set()
+    run_legs = args.workload == "llama3_prefill" and not args.no_legs and bool(want)
     if run_legs:
-        legs["decode"] = leg_decode(fp8, dev, barrier, args, hbm_peak)
-        legs["deepseek_mlp"] = leg_gemm_workload(fp8, dev, barrier, args,
-                                                 workload_linears("deepseek_mlp"))
-        legs["sweep"] = leg_sweep(fp8, dev, barrier, args)
-        legs["tiny"] = leg_tiny(fp8, dev, barrier, args)
+        if "decode" in want:
+            legs["decode"] = leg_decode(fp8, dev, barrier, args, hbm_peak)
+        if "deepseek_mlp" in want:
+            legs["deepseek_mlp"] = leg_gemm_workload(fp8, dev, barrier, args,
+                                                     workload_linears("deepseek_mlp"))
+        if "sweep" in want:
+            legs["sweep"] = leg_sweep(fp8, dev, barrier, args)
+        if "tiny" in want:
+            legs["tiny"] = leg_tiny(fp8, dev, barrier, args)
     sampler.stop()
     fp8.check()
 
@@ -1219,17 +1251,20 @@ def run_ours(args):
     times = [elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms] + \
         [variants[v][k] for v in vnames for k in ("ms", "gemm_ms")]
     leg_slots = []
-    if run_legs:
+    if "decode" in legs:
         dec, lay, _, _ = legs["decode"]
         for k in sorted(dec):
             leg_slots.append((dec[k], "ms"))
         for k in sorted(lay):
             leg_slots.append((lay[k], "ms"))
+    if "deepseek_mlp" in legs:
         _, ds = legs["deepseek_mlp"]
         leg_slots += [(ds, "ms"), (ds, "gemm_ms"), (ds, "fused_ms")]
+    if "sweep" in legs:
         sw, _ = legs["sweep"]
         for k in sorted(sw):
             leg_slots += [(sw[k], "quant_ms"), (sw[k], "gemm_ms"), (sw[k], "fused_ms")]
+    if "tiny" in legs:
         leg_slots.append((legs["tiny"], "ms"))
     maxed = max_over_ranks(times + [d[k] for d, k in leg_slots], dev, world)
     elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms = maxed[:5]
@@ -1353,6 +1388,8 @@ def main():
     ap.add_argument("--eager", action="store_true", help="launch every step's kernels one by one")
     ap.add_argument("--no-legs", action="store_true",
                     help="headline prefill step only (skip the decode, deepseek_mlp, sweep, tiny keys)")
+    ap.add_argument("--legs", default="decode,deepseek_mlp,sweep,tiny",
+                    help="comma-separated per-config legs to run with the prefill workload")
     ap.add_argument("--decode-launches", type=int, default=96,
                     help="timed launches per decode linear (rounded up to whole weight rotations)")
     ap.add_argument("--sweep-launches", type=int, default=12,

@@ -16,24 +16,30 @@
 //     caller's workspace.
 //   - reduce: a block that one CTA covers alone is written as bf16 directly.
 //     For a shared block, every contributing CTA writes its partial and
-//     counts itself in on the block's counter; the last one to arrive sums
-//     the block's partials in increasing CTA order (a fixed order: results
-//     are bit-identical run to run), writes bf16 Y[m, n] and puts the
-//     counter back to zero.  A counter holds a 48-bit call tag next to the
-//     count, and a count whose tag differs from the launch's tag reads as
-//     zero, so the workspace needs no clearing before a launch (a cleared or
-//     reset counter is the zero word; a stale one carries another tag).
+//     counts itself in on the block's counter (one atomic add); the last one
+//     to arrive sums the block's partials in increasing CTA order (a fixed
+//     order: results are bit-identical run to run) and writes bf16 Y[m, n].
+//     The counter is set to zero at the start of the launch by the CTA that
+//     holds the block's first chunk, which then stores the launch's 64-bit
+//     tag in the block's ready flag; the other contributors wait for that
+//     flag before they count in, and the last one clears it.  A flag counts
+//     as set only when it holds this launch's tag, so the workspace needs no
+//     clearing (leftover bytes, other shapes' partials), and since a
+//     completed launch leaves the flags it used cleared, a CUDA graph can
+//     replay its launches with the tags they were captured with.
 // Warps: 0 TMA producer (W tile 128x128 + X tile Mpad x 128 per stage,
-// 8 stages), 1 MMA issuer, 2 TMEM owner, 3 scale products (for every chunk
-// the Mpad factors s_w[blk, j] * s_a[m, j], once per CTA, into a shared
-// ring), 4-11 promotion: two warps per TMEM lane quarter, one weight row
-// per thread, each warp a contiguous part of the token columns.
+// 9-12 stages), 1 MMA issuer, 2 TMEM owner and counter set-up, 3 scale
+// products (for every chunk the Mpad factors s_w[blk, j] * s_a[m, j], once
+// per CTA, into a shared ring), 4-11 promotion: two warps per TMEM lane
+// quarter, one weight row per thread, each warp a contiguous part of the
+// token columns.
 // The kernel is launched with programmatic stream serialization: its set-up
-// (barriers, TMEM, tensor-map prefetch, an L2 prefetch of its first weight
-// tiles) overlaps the previous kernel, and it waits for that kernel to
-// finish before its first access to anything another kernel can write.
-// Every mbarrier wait is bounded; on expiry the kernel records an error
-// code, drains what it started and exits cleanly.
+// (barriers, TMEM, tensor-map prefetch) and an L2 prefetch of the weight
+// tiles its first ring fill loads overlap the previous kernel's tail, when
+// most of that kernel's CTAs have left and HBM would idle; it waits for the
+// previous kernel to finish before its first access to anything another
+// kernel can write.  Every wait is bounded; on expiry the kernel records an
+// error code, drains what it started and exits cleanly.
 #include <atomic>
 #include <chrono>
 #include <cstdint>
@@ -52,31 +58,58 @@ namespace {
 constexpr int DBM = 128;          // weight rows per block (MMA M)
 constexpr int DBK = 128;          // K per chunk (one scale block)
 constexpr int MAX_MPAD = 64;
-constexpr int DSTAGES = 8;
 constexpr int DTBUFS = 4;
 constexpr int DUMMA_K = 32;
 constexpr int CSLOTS = 16;                   // ring of per-chunk scale products
 constexpr int W_BYTES = DBM * DBK;           // 16 KB
-constexpr int X_BYTES = MAX_MPAD * DBK;      // 8 KB (box rows = Mpad <= 64)
 constexpr int DTMEM_COLS = 256;              // DTBUFS * MAX_MPAD
 constexpr int DNUM_THREADS = 384;
 constexpr int PROMO_THREADS = 256;           // warps 4-11
+constexpr int kSmemBudget = 227 * 1024;
 
-constexpr int DSMEM_W_OFF = 0;
-constexpr int DSMEM_X_OFF = DSMEM_W_OFF + DSTAGES * W_BYTES;
-constexpr int DSMEM_C_OFF = DSMEM_X_OFF + DSTAGES * X_BYTES;
-constexpr int DSMEM_BAR_OFF = DSMEM_C_OFF + CSLOTS * MAX_MPAD * 4;
-constexpr int DNUM_BARS = 2 * DSTAGES + 2 * DTBUFS + 2 * CSLOTS + 1;
-constexpr int DSMEM_MISC_OFF = DSMEM_BAR_OFF + DNUM_BARS * 8;
-constexpr int DSMEM_BYTES = DSMEM_MISC_OFF + 16 + 1024;   // + slack for 1024-byte alignment
+// Shared-memory layout for Mpad tokens: as many stages of [W tile 16 KB |
+// X tile Mpad x 128 B] as fit (12 at Mpad 16 down to 9 at Mpad 64: the
+// bytes in flight per SM are what sets the weight stream's rate), then the
+// scale-product ring, the barriers and a few words.
+template <int MPAD>
+struct DLayout {
+  static constexpr int SB = W_BYTES + MPAD * DBK;            // stage bytes, multiple of 1024
+  static constexpr int FIXED = CSLOTS * MAX_MPAD * 4 + (2 * DTBUFS + 2 * CSLOTS + 1) * 8 + 16 + 1024;
+  static constexpr int NS_FIT = (kSmemBudget - FIXED) / (SB + 16);
+  static constexpr int NS = NS_FIT < 12 ? NS_FIT : 12;       // stages
+  static constexpr int C_OFF = NS * SB;
+  static constexpr int BAR_OFF = C_OFF + CSLOTS * MAX_MPAD * 4;
+  static constexpr int NUM_BARS = 2 * NS + 2 * DTBUFS + 2 * CSLOTS + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr int BYTES = MISC_OFF + 16 + 1024;         // + slack for 1024-byte alignment
+  static_assert(BYTES <= kSmemBudget, "shared memory budget");
+  static_assert(SB % 1024 == 0, "stage alignment");
+  // barrier indices
+  static __device__ __forceinline__ int full(int s) { return s; }
+  static __device__ __forceinline__ int empty(int s) { return NS + s; }
+  static __device__ __forceinline__ int tfull(int b) { return 2 * NS + b; }
+  static __device__ __forceinline__ int tempty(int b) { return 2 * NS + DTBUFS + b; }
+  static __device__ __forceinline__ int cfull(int i) { return 2 * NS + 2 * DTBUFS + i; }
+  static __device__ __forceinline__ int cempty(int i) { return 2 * NS + 2 * DTBUFS + CSLOTS + i; }
+  static __device__ __forceinline__ int drain() { return 2 * NS + 2 * DTBUFS + 2 * CSLOTS; }
+  static __device__ __forceinline__ uint32_t bar(uint32_t smem_base, int i) {
+    return smem_base + BAR_OFF + 8u * i;
+  }
+};
+
+// misc words in shared memory
+constexpr int kMiscTmem = 0;       // TMEM base address
+constexpr int kMiscLast = 1;       // "this CTA reduces the block" flag
+constexpr int kMiscReady = 2;      // first block's counter usable: 0 not yet, 1 yes, 2 gave up
 
 struct DecodeArgs {
   const float* s_a;                 // [M, KB]
   const float* s_w;                 // [NB, KB]
   __nv_bfloat16* y;                 // [M, N]
-  unsigned long long* counters;     // [NB] tagged arrival counters
+  unsigned long long* flags;        // [NB] ready flags (the launch's tag when set)
+  unsigned int* counters;           // [NB] arrival counters
   float* partial;                   // [G * maxseg, Mpad, 128]
-  unsigned long long tag;           // this launch's tag, 1 .. 2^48 - 1
+  unsigned long long tag;           // this launch's tag, never zero
   int64_t units;                    // NB * KB
   int N, M, KB;
   int G;                            // CTAs
@@ -90,41 +123,15 @@ __device__ __forceinline__ int64_t range_start(int g, int64_t units, int G) {
 
 __device__ __forceinline__ void record_error(int* err, int code) { atomicCAS(err, 0, code); }
 
-// Counts one contributor in on a block counter and says whether it was the
-// last of `contributors`.  Word = tag << 16 | count; a word carrying another
-// tag (a zero word included) counts as zero.
-__device__ __forceinline__ bool arrive_last(unsigned long long* ctr, unsigned long long tag,
-                                            int contributors) {
-  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(ctr);
-  unsigned long long assumed, next;
-  do {
-    assumed = old;
-    const unsigned long long base = (assumed >> 16) == tag ? (assumed & 0xFFFFull) : 0ull;
-    next = (tag << 16) | (base + 1ull);
-    old = atomicCAS(ctr, assumed, next);
-  } while (old != assumed);
-  return (next & 0xFFFFull) == static_cast<unsigned long long>(contributors);
-}
 
 struct PromoCtx {
   uint32_t smem_base, tmem_base;
   const float* prods;       // shared ring [CSLOTS][MAX_MPAD]
-  volatile int* last_flag;  // shared
+  volatile int* misc;       // shared misc words
   int64_t u_begin, u_end;
   int g, quarter, lane;
 };
 
-__device__ __forceinline__ uint32_t dbar(uint32_t smem_base, int i) {
-  return smem_base + DSMEM_BAR_OFF + 8u * i;
-}
-// barrier indices
-__device__ __forceinline__ int bi_full(int s) { return s; }
-__device__ __forceinline__ int bi_empty(int s) { return DSTAGES + s; }
-__device__ __forceinline__ int bi_tfull(int b) { return 2 * DSTAGES + b; }
-__device__ __forceinline__ int bi_tempty(int b) { return 2 * DSTAGES + DTBUFS + b; }
-__device__ __forceinline__ int bi_cfull(int i) { return 2 * DSTAGES + 2 * DTBUFS + i; }
-__device__ __forceinline__ int bi_cempty(int i) { return 2 * DSTAGES + 2 * DTBUFS + CSLOTS + i; }
-__device__ __forceinline__ int bi_drain() { return 2 * DSTAGES + 2 * DTBUFS + 2 * CSLOTS; }
 
 // Promotion by one warp: token columns COL0 .. COL0 + NC - 1 of its lane
 // quarter's 32 weight rows (NC = 0: the warp only takes part in the
@@ -135,6 +142,7 @@ __device__ __forceinline__ int bi_drain() { return 2 * DSTAGES + 2 * DTBUFS + 2 
 // walking.
 template <int MPAD, int NC, int COL0>
 __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const PromoCtx& cx) {
+  using L = DLayout<MPAD>;
   const int lane = cx.lane;
   const int n_local = cx.quarter * 32 + lane;   // weight row within the block
   const uint32_t lane_off = static_cast<uint32_t>(cx.quarter * 32) << 16;
@@ -148,7 +156,7 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
   bool ok = true;
   int blk = first_blk;
   int kb = static_cast<int>(cx.u_begin - static_cast<int64_t>(first_blk) * KB) - 1;
-  for (int64_t u = cx.u_begin; u < cx.u_end; ++u) {
+  for (int64_t u = cx.u_begin; u < cx.u_end; ++u, ++c) {
     if (++kb == KB) {
       kb = 0;
       ++blk;
@@ -157,9 +165,8 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
     const uint32_t bph = (c / DTBUFS) & 1u;
     const int slot = c % CSLOTS;
     const uint32_t cph = (c / CSLOTS) & 1u;
-    ++c;
     if (NC > 0 && ok) {
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(dbar(cx.smem_base, bi_tfull(buf)), bph))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(L::bar(cx.smem_base, L::tfull(buf)), bph))) {
         if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
         ok = false;
       } else {
@@ -173,8 +180,8 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
         ptx::tmem_ld_wait();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(dbar(cx.smem_base, bi_tempty(buf)));
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(dbar(cx.smem_base, bi_cfull(slot)), cph))) {
+        if (lane == 0) ptx::mbar_arrive(L::bar(cx.smem_base, L::tempty(buf)));
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(L::bar(cx.smem_base, L::cfull(slot)), cph))) {
           if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
           ok = false;
         } else {
@@ -188,7 +195,7 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
             acc[4 * j + 3] = __fmaf_rn(__uint_as_float(v[4 * j + 3]), p.w, acc[4 * j + 3]);
           }
           __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(dbar(cx.smem_base, bi_cempty(slot)));
+          if (lane == 0) ptx::mbar_arrive(L::bar(cx.smem_base, L::cempty(slot)));
         }
       }
     }
@@ -215,23 +222,33 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
         const int g_lo = static_cast<int>(((blk_u0 + 1) * args.G - 1) / args.units);
         const int g_hi = static_cast<int>(((blk_u0 + KB) * args.G - 1) / args.units);
         if (threadIdx.x == 128) {
-          __threadfence();
-          const bool last = arrive_last(args.counters + blk, args.tag, g_hi - g_lo + 1);
-          if (last) {
-            // every contributor has counted in: the counter is free again
-            atomicExch(args.counters + blk, 0ull);
+          // the block's counter must have been set up for this launch (by
+          // this CTA's warp 2, or by the CTA holding the block's first chunk)
+          const uint64_t t0 = clock64();
+          while (cx.misc[kMiscReady] == 0 && clock64() - t0 < (1ull << 32)) __nanosleep(32);
+          bool last = false;
+          if (cx.misc[kMiscReady] == 1) {
             __threadfence();
+            last = atomicAdd(args.counters + blk, 1u) == static_cast<unsigned>(g_hi - g_lo);
+            if (last) {
+              // every contributor has counted in: the flag is free again
+              *reinterpret_cast<volatile unsigned long long*>(args.flags + blk) = 0ull;
+              __threadfence();
+            }
+          } else {
+            record_error(args.err, kErrTimeoutEpilogue);
           }
-          *cx.last_flag = last ? 1 : 0;
+          cx.misc[kMiscLast] = last ? 1 : 0;
         }
         ptx::named_barrier_sync(1, PROMO_THREADS);
-        if (*cx.last_flag) {
+        if (cx.misc[kMiscLast]) {
           // Sum the block's partials in increasing CTA order.  All 256
           // promotion threads take part: thread t sums row t % 128, token
-          // columns (t / 128) * MPAD / 2 .. + MPAD / 2 - 1; UR partials'
-          // loads are in flight together.
+          // columns (t / 128) * MPAD / 2 .. + MPAD / 2 - 1; the loads of UR
+          // partials (all of them for the usual contributor counts) are in
+          // flight together.
           constexpr int HALF = MPAD / 2;
-          constexpr int UR = HALF <= 8 ? 4 : (HALF <= 16 ? 2 : 1);
+          constexpr int UR = HALF <= 8 ? 8 : (HALF <= 16 ? 4 : 2);
           const int t = threadIdx.x - 128;
           const int rn = t & 127;
           const int m0 = (t >> 7) * HALF;
@@ -277,10 +294,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  using L = DLayout<MPAD>;
+  constexpr int NS = L::NS;
   const uint32_t smem_base = ptx::smem_u32(smem);
-  auto bar = [&](int i) { return dbar(smem_base, i); };
-  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + DSMEM_MISC_OFF);
-  float* prods = reinterpret_cast<float*>(smem + DSMEM_C_OFF);
+  auto bar = [&](int i) { return L::bar(smem_base, i); };
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* vmisc = reinterpret_cast<volatile int*>(misc);
+  float* prods = reinterpret_cast<float*>(smem + L::C_OFF);
   constexpr uint32_t IDESC = ptx::idesc_e4m3_f32(DBM, MPAD);
   constexpr uint32_t STAGE_TX = W_BYTES + MPAD * DBK;
   // token columns per promotion half: half 0 takes NC0, half 1 the rest
@@ -296,38 +316,41 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
   const int64_t u_end = range_start(g + 1, args.units, args.G);
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < DSTAGES; ++s) {
-      ptx::mbar_init(bar(bi_full(s)), 1);
-      ptx::mbar_init(bar(bi_empty(s)), 1);
+    for (int s = 0; s < NS; ++s) {
+      ptx::mbar_init(bar(L::full(s)), 1);
+      ptx::mbar_init(bar(L::empty(s)), 1);
     }
     for (int b = 0; b < DTBUFS; ++b) {
-      ptx::mbar_init(bar(bi_tfull(b)), 1);
-      ptx::mbar_init(bar(bi_tempty(b)), LOADERS);
+      ptx::mbar_init(bar(L::tfull(b)), 1);
+      ptx::mbar_init(bar(L::tempty(b)), LOADERS);
     }
     for (int i = 0; i < CSLOTS; ++i) {
-      ptx::mbar_init(bar(bi_cfull(i)), 32);
-      ptx::mbar_init(bar(bi_cempty(i)), LOADERS);
+      ptx::mbar_init(bar(L::cfull(i)), 32);
+      ptx::mbar_init(bar(L::cempty(i)), LOADERS);
     }
-    ptx::mbar_init(bar(bi_drain()), 1);
+    ptx::mbar_init(bar(L::drain()), 1);
     ptx::fence_barrier_init();
     ptx::prefetch_tmap(&tmap_w);
     ptx::prefetch_tmap(&tmap_x);
-    // Warm the L2 with the first weight tiles while the previous kernel may
-    // still run (a prefetch only; the loads below come after the wait).
+    vmisc[kMiscLast] = 0;
+    vmisc[kMiscReady] = 0;
+    // Warm the L2 with this CTA's first weight tiles while the previous
+    // kernel may still run (a prefetch only; the loads below come after the
+    // wait, and a later write by the previous kernel would update L2).
     int blk = static_cast<int>(u_begin / KB);
     int kb = static_cast<int>(u_begin - static_cast<int64_t>(blk) * KB);
-    for (int64_t u = u_begin; u < u_end && u < u_begin + DSTAGES;
+    for (int64_t u = u_begin; u < u_end && u < u_begin + NS;
          ++u, (++kb == KB ? (kb = 0, ++blk) : 0))
       ptx::tma_prefetch_2d(&tmap_w, kb * DBK, blk * DBM);
   }
   if (warp == 2) {
-    ptx::tmem_alloc(ptx::smem_u32(misc), DTMEM_COLS);
+    ptx::tmem_alloc(ptx::smem_u32(misc + kMiscTmem), DTMEM_COLS);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(misc);
+  const uint32_t tmem_base = vmisc[kMiscTmem];
   // From here on the kernel reads what earlier kernels wrote (activation
   // codes and scales) and writes what they may read (Y, the workspace).
   ptx::grid_dep_wait();
@@ -340,17 +363,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     int blk = static_cast<int>(u_begin / KB);
     int kb = static_cast<int>(u_begin - static_cast<int64_t>(blk) * KB);
     for (int64_t u = u_begin; u < u_end; ++u, ++c, (++kb == KB ? (kb = 0, ++blk) : 0)) {
-      const int s = c % DSTAGES;
-      const uint32_t ph = (c / DSTAGES) & 1u;
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(bar(bi_empty(s)), ph ^ 1u))) {
+      const int s = c % NS;
+      const uint32_t ph = (c / NS) & 1u;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::empty(s)), ph ^ 1u))) {
         if (lane == 0) record_error(args.err, kErrTimeoutProducer);
         break;
       }
       if (lane == 0) {
-        ptx::mbar_arrive_expect_tx(bar(bi_full(s)), STAGE_TX);
-        ptx::tma_load_2d(smem_base + DSMEM_W_OFF + s * W_BYTES, &tmap_w, bar(bi_full(s)), kb * DBK,
-                         blk * DBM);
-        ptx::tma_load_2d(smem_base + DSMEM_X_OFF + s * X_BYTES, &tmap_x, bar(bi_full(s)), kb * DBK, 0);
+        ptx::mbar_arrive_expect_tx(bar(L::full(s)), STAGE_TX);
+        ptx::tma_load_2d(smem_base + s * L::SB, &tmap_w, bar(L::full(s)), kb * DBK, blk * DBM);
+        ptx::tma_load_2d(smem_base + s * L::SB + W_BYTES, &tmap_x, bar(L::full(s)), kb * DBK, 0);
       }
       __syncwarp();
       issued_mask |= 1u << s;
@@ -358,8 +380,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     }
     // every load issued lands before the CTA may exit
     if (lane == 0)
-      for (int s = 0; s < DSTAGES; ++s)
-        if (((issued_mask >> s) & 1u) && !ptx::mbar_wait(bar(bi_full(s)), (phase_mask >> s) & 1u))
+      for (int s = 0; s < NS; ++s)
+        if (((issued_mask >> s) & 1u) && !ptx::mbar_wait(bar(L::full(s)), (phase_mask >> s) & 1u))
           record_error(args.err, kErrTimeoutProducer);
     __syncwarp();
   } else if (warp == 1) {
@@ -370,33 +392,65 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     uint32_t c = 0;
     bool issued = false;
     for (int64_t u = u_begin; u < u_end; ++u, ++c) {
-      const int s = c % DSTAGES;
-      const uint32_t sph = (c / DSTAGES) & 1u;
+      const int s = c % NS;
+      const uint32_t sph = (c / NS) & 1u;
       const int buf = c % DTBUFS;
       const uint32_t bph = (c / DTBUFS) & 1u;
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(bar(bi_tempty(buf)), bph ^ 1u) &&
-                                       ptx::mbar_wait_spin(bar(bi_full(s)), sph))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(bar(L::tempty(buf)), bph ^ 1u) &&
+                                       ptx::mbar_wait_spin(bar(L::full(s)), sph))) {
         if (lane == 0) record_error(args.err, kErrTimeoutMma);
         break;
       }
       ptx::tc_fence_after();
       if (lane == 0) {
-        const uint32_t w_addr = smem_base + DSMEM_W_OFF + s * W_BYTES;
-        const uint32_t x_addr = smem_base + DSMEM_X_OFF + s * X_BYTES;
+        const uint32_t w_addr = smem_base + s * L::SB;
+        const uint32_t x_addr = w_addr + W_BYTES;
         const uint32_t d = tmem_base + static_cast<uint32_t>(buf * MAX_MPAD);
 #pragma unroll
         for (int k = 0; k < DBK / DUMMA_K; ++k)
           ptx::mma_f8f6f4(d, ptx::sdesc_kmajor_sw128(w_addr + k * DUMMA_K),
                           ptx::sdesc_kmajor_sw128(x_addr + k * DUMMA_K), IDESC, k > 0 ? 1u : 0u);
-        ptx::mma_commit(bar(bi_tfull(buf)));
-        ptx::mma_commit(bar(bi_empty(s)));
+        ptx::mma_commit(bar(L::tfull(buf)));
+        ptx::mma_commit(bar(L::empty(s)));
       }
       __syncwarp();
       issued = true;
     }
     if (issued && lane == 0) {
-      ptx::mma_commit(bar(bi_drain()));
-      if (!ptx::mbar_wait(bar(bi_drain()), 0)) record_error(args.err, kErrTimeoutMma);
+      ptx::mma_commit(bar(L::drain()));
+      if (!ptx::mbar_wait(bar(L::drain()), 0)) record_error(args.err, kErrTimeoutMma);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------- counter set-up
+    // Zero the counters of the shared blocks whose first chunk lies in this
+    // CTA's range, then mark them ready with the launch's tag; if this CTA's
+    // range starts inside a block, wait until that block's first CTA has
+    // done the same for it.
+    if (lane == 0) {
+      const int64_t b_lo = (u_begin + KB - 1) / KB, b_hi = (u_end - 1) / KB;
+      for (int64_t b = b_lo; b <= b_hi; ++b)
+        if (((b * KB + KB) * args.G - 1) / args.units > ((b * KB + 1) * args.G - 1) / args.units)
+          args.counters[b] = 0u;
+      __threadfence();
+      for (int64_t b = b_lo; b <= b_hi; ++b)
+        if (((b * KB + KB) * args.G - 1) / args.units > ((b * KB + 1) * args.G - 1) / args.units)
+          *reinterpret_cast<volatile unsigned long long*>(args.flags + b) = args.tag;
+      int ready = 1;
+      if (u_begin % KB != 0) {
+        const volatile unsigned long long* f =
+            reinterpret_cast<const volatile unsigned long long*>(args.flags + u_begin / KB);
+        const uint64_t t0 = clock64();
+        while (*f != args.tag) {
+          if (clock64() - t0 > (1ull << 32)) {
+            ready = 2;
+            break;
+          }
+          __nanosleep(64);
+        }
+        __threadfence();
+      }
+      vmisc[kMiscReady] = ready;
     }
     __syncwarp();
   } else if (warp == 3) {
@@ -404,16 +458,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     // prods[slot][m] = s_w[blk, kb] * s_a[m, kb] for every chunk of the
     // range, up to CSLOTS chunks ahead of the promotion warps.  Lane l
     // covers tokens l and l + 32.  The scales of a chunk are loaded PF
-    // chunks ahead (L2 path: another kernel wrote them) into a register slot
-    // that is refilled right after its use.
-    constexpr int PF = 4;
+    // chunks ahead (L2 path: another kernel wrote them; under a full HBM
+    // stream an L2 read can take microseconds) into a register slot that is
+    // refilled right after its use.  s_w of unit u is s_w[u] (row-major
+    // [NB, KB]).
+    constexpr int PF = 8;
     float pw[PF], plo[PF], phi[PF];
     auto load_scales = [&](int64_t uu, float& w, float& lo, float& hi) {
       w = lo = hi = 0.0f;
       if (uu < u_end) {
-        const int b = static_cast<int>(uu / KB);
-        const int k = static_cast<int>(uu - static_cast<int64_t>(b) * KB);
-        w = __ldcg(args.s_w + static_cast<int64_t>(b) * KB + k);
+        const int k = static_cast<int>(uu % KB);
+        w = __ldcg(args.s_w + uu);
         if (lane < args.M) lo = __ldcg(args.s_a + static_cast<int64_t>(lane) * KB + k);
         if (MPAD > 32 && lane + 32 < args.M)
           hi = __ldcg(args.s_a + static_cast<int64_t>(lane + 32) * KB + k);
@@ -433,7 +488,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         const int slot = c % CSLOTS;
         const uint32_t ph = (c / CSLOTS) & 1u;
         ++c;
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(bar(bi_cempty(slot)), ph ^ 1u))) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::cempty(slot)), ph ^ 1u))) {
           if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
           ok = false;
           break;
@@ -441,7 +496,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         float* cr = prods + slot * MAX_MPAD;
         cr[lane] = cw * clo;
         if (MPAD > 32) cr[32 + lane] = cw * chi;
-        ptx::mbar_arrive(bar(bi_cfull(slot)));
+        ptx::mbar_arrive(bar(L::cfull(slot)));
       }
     }
   } else if (warp >= 4) {
@@ -450,7 +505,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     cx.smem_base = smem_base;
     cx.tmem_base = tmem_base;
     cx.prods = prods;
-    cx.last_flag = reinterpret_cast<volatile int*>(misc + 1);
+    cx.misc = vmisc;
     cx.u_begin = u_begin;
     cx.u_end = u_end;
     cx.g = g;
@@ -492,9 +547,9 @@ DecodeGeometry decode_geometry(int64_t M, int64_t N, int64_t K, int sm_count) {
 }
 
 // Tag of one launch: a per-process random start advanced by an odd constant
-// per launch, kept to 48 bits and never zero.  A graph replays its launches
-// with their tags; that is sound because every launch that completes leaves
-// its counters at zero.
+// per launch, never zero (a cleared flag).  A graph replays its launches
+// with their tags; that is sound because every launch that completes
+// leaves the ready flags it set cleared.
 unsigned long long next_launch_tag() {
   static std::atomic<unsigned long long> seq{0};
   static const unsigned long long salt = [] {
@@ -507,8 +562,7 @@ unsigned long long next_launch_tag() {
     return x;
   }();
   const unsigned long long t =
-      (salt + 0x9E3779B97F4A7C15ull * (seq.fetch_add(1, std::memory_order_relaxed) + 1)) &
-      ((1ull << 48) - 1);
+      salt + 0x9E3779B97F4A7C15ull * (seq.fetch_add(1, std::memory_order_relaxed) + 1);
   return t ? t : 1ull;
 }
 
@@ -519,13 +573,13 @@ cudaError_t launch_decode_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
   static cudaError_t status[kMaxDevices];
   const cudaError_t attr = once_per_device(once, status, [](int) {
     return cudaFuncSetAttribute(decode_kernel<MPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                DSMEM_BYTES);
+                                DLayout<MPAD>::BYTES);
   });
   if (attr != cudaSuccess) return attr;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.G), 1, 1);
   cfg.blockDim = dim3(DNUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = DSMEM_BYTES;
+  cfg.dynamicSmemBytes = DLayout<MPAD>::BYTES;
   cfg.stream = st;
   cudaLaunchAttribute at[1];
   set_programmatic_serialization(at[0]);
@@ -536,15 +590,15 @@ cudaError_t launch_decode_t(const CUtensorMap& tw, const CUtensorMap& tx, const 
 
 }  // namespace
 
-// Workspace: NB 64-bit block counters (rounded up to 256 bytes), then the
-// partials.
-size_t decode_counter_bytes(int64_t N) {
-  return static_cast<size_t>(((N / 128) * 8 + 255) / 256 * 256);
-}
+// Workspace: the ready flags [NB] (64-bit) and the counters [NB] (32-bit),
+// rounded up to 256 bytes, then the partials.
+namespace {
+size_t flag_bytes(int64_t N) { return static_cast<size_t>(((N / 128) * 12 + 255) / 256 * 256); }
+}  // namespace
 
 size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count) {
   const DecodeGeometry d = decode_geometry(M, N, K, sm_count);
-  return decode_counter_bytes(N) + static_cast<size_t>(d.G) * d.maxseg * d.Mpad * 128 * sizeof(float);
+  return flag_bytes(N) + static_cast<size_t>(d.G) * d.maxseg * d.Mpad * 128 * sizeof(float);
 }
 
 cudaError_t launch_block_linear_decode(const void* q_a, const float* s_a, const void* q_w,
@@ -555,12 +609,14 @@ cudaError_t launch_block_linear_decode(const void* q_a, const float* s_a, const 
   if (!make_tmap_u8(&tw, q_w, N, K, DBM, DBK) ||
       !make_tmap_u8(&tx, q_a, M, K, static_cast<uint32_t>(d.Mpad), DBK))
     return cudaErrorInvalidValue;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   DecodeArgs a;
   a.s_a = s_a;
   a.s_w = s_w;
   a.y = static_cast<__nv_bfloat16*>(y);
-  a.counters = static_cast<unsigned long long*>(workspace);
-  a.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + decode_counter_bytes(N));
+  a.flags = reinterpret_cast<unsigned long long*>(ws);
+  a.counters = reinterpret_cast<unsigned int*>(ws + (N / 128) * 8);
+  a.partial = reinterpret_cast<float*>(ws + flag_bytes(N));
   a.tag = next_launch_tag();
   a.units = d.units;
   a.N = static_cast<int>(N);

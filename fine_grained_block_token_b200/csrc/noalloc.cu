@@ -19,8 +19,9 @@
 //
 // Every call on a device shares the same array and leaves its contents
 // behind.  Nothing needs clearing between calls: the decode schedule's
-// block counters carry a per-launch tag, a count under another tag reads as
-// zero, and a completed launch leaves them at zero.  Two calls whose GPU
+// hand-over flags count as set only when they hold the launch's own tag,
+// and a completed launch leaves the flags it used cleared.  Two calls whose
+// GPU
 // work overlaps -- on different streams without ordering between them --
 // race on the array.
 #include <cstdint>

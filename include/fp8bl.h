@@ -141,13 +141,14 @@ fp8bl_status fp8_quant_weight(const void *w_bf16, int64_t N, int64_t K,
  *   workspace: device scratch of at least
  *              fp8_block_linear_workspace_bytes(M, N, K) bytes (16-byte
  *              aligned), or NULL when that size is 0.  It needs no
- *              clearing: it starts with one 64-bit counter per 128-row
- *              weight block that carries a per-launch tag, and a count under
- *              another tag reads as zero (any leftover content is
- *              accepted; a chance match of the 48-bit tag is the only way it
- *              could be misread).  A completed call leaves the counters at
- *              zero; after FP8BL_ERR_TIMEOUT, zero the workspace before a
- *              CUDA graph replays calls on it.
+ *              clearing: it starts with a ready flag and a counter per
+ *              128-row weight block, through which the CTAs that share a
+ *              block hand over their partial sums; a flag counts as set
+ *              only when it holds the launch's own 64-bit tag, so leftover
+ *              bytes read as "not set", and every completed call leaves the
+ *              flags it set cleared (so a CUDA graph may replay calls on
+ *              it).  After FP8BL_ERR_TIMEOUT, zero the workspace before a
+ *              graph replays calls on it.
  *   M >= 0, N, K > 0 and multiples of 128, all <= FP8BL_MAX_DIM.
  */
 fp8bl_status fp8_block_linear(const void *q_a, const float *s_a,
@@ -192,7 +193,7 @@ fp8bl_status fp8_block_linear_fused(const void *x_bf16,
  *   The first call on each device looks up the array's device address (a
  *   CUDA runtime query), so make that first call before any stream capture.
  *   All calls on a device share the array and leave its contents behind;
- *   nothing in it needs clearing between calls (the counters it holds are
+ *   nothing in it needs clearing between calls (its hand-over flags are
  *   tagged per launch, as in fp8_block_linear's workspace).  Calls
  *   whose GPU work may overlap (different streams with no ordering between
  *   them) race on the array and must not be issued.

@@ -230,8 +230,8 @@ def _decode_slots_needed(N, K, G):
 
 @pytest.mark.parametrize("seed", range(6))
 def test_decode_workspace_covers_every_partial_slot(lib, seed):
-    """The workspace the library asks for must hold the per-block counters
-    plus, for each of the G CTAs, a partial [Mpad, 128] fp32 for every block
+    """The workspace the library asks for must hold the per-block ready flags
+    and counters plus, for each of the G CTAs, a partial [Mpad, 128] fp32 for every block
     its range touches; a smaller stride would let a CTA write past its
     slots (and the last CTA past the buffer).  Without a GPU the library
     plans for 148 SMs; G = min(148, U / ceil(KB / 8)) CTAs."""
@@ -248,7 +248,8 @@ def test_decode_workspace_covers_every_partial_slot(lib, seed):
         KB, U = K // 128, (N // 128) * (K // 128)
         G = max(1, min(148, U // ((KB + 7) // 8)))
         mpad = (M + 15) // 16 * 16
-        counters = ((N // 128) * 8 + 255) // 256 * 256     # 64-bit tagged counters
+        # a 64-bit ready flag and a 32-bit counter per weight block
+        counters = ((N // 128) * 12 + 255) // 256 * 256
         ws = f(M, N, K)
         per_slot = G * mpad * 128 * 4
         assert ws > counters and (ws - counters) % per_slot == 0, (M, N, K, ws)

@@ -215,10 +215,11 @@ def test_fused_repeated_runs_bit_identical(fp8, M, N, K):
 
 
 def test_decode_workspace_needs_no_clearing(fp8):
-    """The decode schedule's block counters carry a per-launch tag, so a
-    workspace holding leftover bytes -- all ones, random bytes, or another
-    shape's leftovers -- gives the same Y, bit for bit, as a fresh one, and
-    calls that reuse one workspace across shapes stay exact."""
+    """The decode schedule's hand-over flags count as set only when they hold
+    the launch's own tag, so a workspace holding leftover bytes -- all ones,
+    random bytes, or another shape's leftovers -- gives the same Y, bit for
+    bit, as a fresh one, and calls that reuse one workspace across shapes
+    stay exact."""
     shapes = [(1, 4096, 4096), (64, 1024, 4096), (17, 2048, 3072)]
     runs = []
     size = 0
@@ -249,9 +250,9 @@ def test_decode_workspace_needs_no_clearing(fp8):
 
 
 def test_decode_graph_replay_bit_identical(fp8):
-    """A CUDA graph replays its decode launches with the tags they were
-    captured with; every completed launch leaves its counters at zero, so
-    replays give the eager result bit for bit.  The graph holds the
+    """A CUDA graph replays its decode launches with the arguments they were
+    captured with (tags included); every completed launch leaves the flags
+    it used cleared, so replays give the eager result bit for bit.  The graph holds the
     activation quantizer and the decode linear back to back (both launched
     with programmatic serialization), for two shapes on one workspace."""
     items = []
