@@ -121,9 +121,11 @@ cudaError_t launch_block_linear_decode(const void* q_a, const float* s_a, const 
                                        void* workspace, const DeviceInfo& dev, cudaStream_t st);
 
 // 2-D TMA map over a row-major byte matrix [rows, cols], box box_rows x
-// box_cols, 128-byte swizzle, out-of-range elements read as zero.
+// box_cols, 128-byte swizzle unless told otherwise; out-of-range elements
+// read as zero (and are not written by stores).
 bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                  uint32_t box_rows, uint32_t box_cols);
+                  uint32_t box_rows, uint32_t box_cols,
+                  CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
 
 cudaError_t launch_block_linear_fused(const void* x, const void* q_w, const float* s_w, void* y,
                                       int64_t M, int64_t N, int64_t K, const GemmPlan& plan,

@@ -21,24 +21,26 @@
 //               with a data-dependent exit, measured ~600 cycles per
 //               iteration on B200 whatever it waited for.)
 //   warp 2      owns the TMEM allocation (512 columns).
+//   warp 3      scale products: for every chunk the 256 factors
+//               s_a[row, j] * s_w[nblk, j] of the tile (128 rows x 2 weight
+//               blocks) into a shared ring, up to 8 chunks ahead.
 //   warps 4-11  promotion: warp w reads TMEM lanes 32 (w % 4) .. +31 (its
 //               rows) and column half (w - 4) / 4 (one 128-wide weight
 //               block) in 16-column loads, releases the buffer as soon as
-//               the last load has landed, and adds partial * s_a[row, j] *
-//               s_w[nblk, j] into 128 fp32 registers with packed f32x2
-//               FMAs; after the last chunk it converts to bf16 and stores.
-// What bounds it (measured on B200): every 128-deep chunk leaves a 128 KB
-// fp32 partial in TMEM that must be read into registers before the buffer
-// can take the chunk after next.  tcgen05.ld is latency-bound (a 64-column
-// load takes ~250 cycles; one warp moves at most ~36 B/cycle), so the read
-// rate equals the bytes in flight / ~250 cycles, and with the 128x256 fp32
-// accumulator occupying half the register file the promotion warps cannot
-// keep the ~64 KB in flight that the tensor core's 512 cycles per chunk
-// require.  Variants with two MMA-issuing warps, 64-column loads, 16
-// promotion warps, four 128-column TMEM buffers or CTA-pair tiles all land
-// at the same ~1.0-1.1 M flop per cycle (about 45% of the tensor core's
-// rate); the concurrent TMEM reads, FMAs and the power limit do not slow
-// the MMAs themselves.
+//               the last load has landed, and adds partial * factor into
+//               128 fp32 registers with packed f32x2 FMAs; after a tile's
+//               last chunk it writes bf16 through a shared staging box and
+//               TMA stores (coalesced; rows past M, columns past N clipped).
+// Where the time goes (cycle counters in the warps, B200): per 128 x 256 x
+// 128 chunk the MMA warp spends ~750 cycles issuing into a busy tensor pipe
+// (each chunk moves 48 KB into shared memory by TMA and 48 KB out of it
+// into the tensor core, which is about what shared memory delivers in that
+// time) and ~150-200 waiting for a free TMEM buffer, ~65 for operands.  The
+// read-out of a partial takes ~320 cycles of TMEM loads plus ~275 of the
+// FMAs interleaved with them.  Moving the scale loads to warp 3 (they
+// stalled the promotion ~110 cycles per chunk) and the bf16 stores to TMA
+// (the row-per-thread stores cost ~7,400 cycles per tile) took the chunk
+// from ~1,050-1,200 to ~940-1,010 cycles.
 // Every mbarrier wait is bounded in time; on expiry the kernel records an
 // error code in the error word, drains what it started and exits cleanly.
 #include <cstdint>
@@ -67,12 +69,22 @@ constexpr int NUM_THREADS = 384;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr uint32_t IDESC = ptx::idesc_e4m3_f32(BM, BN);
 
+constexpr int STAGE_ROWS = 32;     // epilogue staging: 32 rows x 64 bytes per warp
+constexpr int STAGE_COLS = 32;     // bf16 columns per staging pass
+constexpr int STAGE_WARP_BYTES = STAGE_ROWS * STAGE_COLS * 2;
+constexpr int PSLOTS = 8;          // ring of per-chunk scale products
+constexpr int PSLOT_FLOATS = 256;  // 128 rows x 2 weight blocks
+
 constexpr int SMEM_A_OFF = 0;
 constexpr int SMEM_B_OFF = SMEM_A_OFF + STAGES * A_BYTES;
-constexpr int SMEM_BAR_OFF = SMEM_B_OFF + STAGES * B_BYTES;
-constexpr int NUM_BARS = 2 * STAGES + 4 + 1;   // full, empty, tfull[2], tempty[2], drain
+constexpr int SMEM_Y_OFF = SMEM_B_OFF + STAGES * B_BYTES;
+constexpr int SMEM_P_OFF = SMEM_Y_OFF + NUM_EPI_WARPS * STAGE_WARP_BYTES;
+constexpr int SMEM_BAR_OFF = SMEM_P_OFF + PSLOTS * PSLOT_FLOATS * 4;
+// full, empty, tfull[2], tempty[2], drain, pfull[PSLOTS], pempty[PSLOTS]
+constexpr int NUM_BARS = 2 * STAGES + 4 + 1 + 2 * PSLOTS;
 constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NUM_BARS * 8;
 constexpr int SMEM_BYTES = SMEM_MISC_OFF + 16 + 1024;  // + slack for 1024-byte alignment
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
 struct GemmArgs {
   const float* s_a;
@@ -88,7 +100,8 @@ __device__ __forceinline__ void record_error(int* err, int code) {
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                    const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+                    const __grid_constant__ CUtensorMap tmap_b,
+                    const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -99,6 +112,9 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
   auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
   const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
+  auto pfull_bar = [&](int i) { return bar_base + 8u * (2 * STAGES + 5 + i); };
+  auto pempty_bar = [&](int i) { return bar_base + 8u * (2 * STAGES + 5 + PSLOTS + i); };
+  float* prods = reinterpret_cast<float*>(smem + SMEM_P_OFF);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SMEM_MISC_OFF);
 
   const int warp = threadIdx.x >> 5;
@@ -119,9 +135,14 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
       ptx::mbar_init(tempty_bar(b), NUM_EPI_WARPS);
     }
     ptx::mbar_init(drain_bar, 1);
+    for (int i = 0; i < PSLOTS; ++i) {
+      ptx::mbar_init(pfull_bar(i), 32);
+      ptx::mbar_init(pempty_bar(i), NUM_EPI_WARPS);
+    }
     ptx::fence_barrier_init();
     ptx::prefetch_tmap(&tmap_a);
     ptx::prefetch_tmap(&tmap_b);
+    ptx::prefetch_tmap(&tmap_y);
   }
   if (warp == 2) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_holder), TMEM_COLS);
@@ -203,37 +224,104 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
       }
       __syncwarp();
     }
+  } else if (warp == 3) {
+    // ------------------------------------------------------ scale products
+    // For every chunk of every tile: prods[slot][h * 128 + r] =
+    // s_a[row r, kb] * s_w[weight block h, kb], up to PSLOTS chunks ahead
+    // of the promotion warps.  Lane l covers rows l + 32 i, i = 0..3; the
+    // scales of a chunk are loaded PF chunks ahead into a register slot that
+    // is refilled right after its use.
+    const int nblk_count = N / 128;
+    constexpr int PF = 4;
+    uint32_t c = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int m_blk = tile % num_m, n_blk = tile / num_m;
+      const float* sa_r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int row = m_blk * BM + lane + 32 * i;
+        sa_r[i] = args.s_a + static_cast<int64_t>(row < M ? row : M - 1) * num_kb;
+      }
+      const float* sw_r[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int nb = n_blk * 2 + h;
+        sw_r[h] = args.s_w + static_cast<int64_t>(nb < nblk_count ? nb : nblk_count - 1) * num_kb;
+      }
+      float pa[PF][4], pw[PF][2];
+      auto load = [&](int kb, float (&a)[4], float (&w)[2]) {
+        if (kb < num_kb) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a[i] = __ldg(sa_r[i] + kb);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) w[h] = __ldg(sw_r[h] + kb);
+        }
+      };
+#pragma unroll
+      for (int j = 0; j < PF; ++j) load(j, pa[j], pw[j]);
+      for (int kb0 = 0; kb0 < num_kb && ok; kb0 += PF) {
+#pragma unroll
+        for (int j = 0; j < PF; ++j) {
+          const int kb = kb0 + j;
+          if (kb >= num_kb) break;
+          float a[4], w[2];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a[i] = pa[j][i];
+          w[0] = pw[j][0];
+          w[1] = pw[j][1];
+          load(kb + PF, pa[j], pw[j]);
+          const int slot = c % PSLOTS;
+          const uint32_t ph = (c / PSLOTS) & 1u;
+          ++c;
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(pempty_bar(slot), ph ^ 1u))) {
+            if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
+            ok = false;
+            break;
+          }
+          float* pr = prods + slot * PSLOT_FLOATS;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pr[h * 128 + lane + 32 * i] = a[i] * w[h];
+          ptx::mbar_arrive(pfull_bar(slot));
+        }
+      }
+    }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     const int half = (warp - 4) >> 2;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int nblk_count = N / 128;
+    const uint32_t stage = smem_base + SMEM_Y_OFF + static_cast<uint32_t>(warp - 4) * STAGE_WARP_BYTES;
     uint32_t c = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       const int m_blk = tile % num_m, n_blk = tile / num_m;
-      const int row = m_blk * BM + quarter * 32 + lane;
+      const int row0 = m_blk * BM + quarter * 32;   // this warp's first row
       const int nb = n_blk * 2 + half;
-      const bool row_ok = row < M;
-      const bool col_ok = nb < nblk_count;
-      const float* sa_row = args.s_a + static_cast<int64_t>(row_ok ? row : M - 1) * num_kb;
-      const float* sw_row = args.s_w + static_cast<int64_t>(col_ok ? nb : nblk_count - 1) * num_kb;
+      const bool box_ok = nb < nblk_count && row0 < M;
       float2 acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
-      float sa1 = __ldg(sa_row), sw1 = __ldg(sw_row);
-      float sa2 = num_kb > 1 ? __ldg(sa_row + 1) : 0.0f;
-      float sw2 = num_kb > 1 ? __ldg(sw_row + 1) : 0.0f;
       for (int kb = 0; kb < num_kb; ++kb, ++c) {
-        const float scale = sa1 * sw1;
-        const float2 sc2 = make_float2(scale, scale);
-        sa1 = sa2; sw1 = sw2;
-        if (kb + 2 < num_kb) { sa2 = __ldg(sa_row + kb + 2); sw2 = __ldg(sw_row + kb + 2); }
         const int buf = c & 1;
         const uint32_t bph = (c >> 1) & 1u;
+        const int slot = c % PSLOTS;
+        const uint32_t pph = (c / PSLOTS) & 1u;
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(pfull_bar(slot), pph))) {
+          if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
+          ok = false;
+          break;
+        }
+        // s_a[row, kb] * s_w[nb, kb], from the scale-product warp
+        const float scale = prods[slot * PSLOT_FLOATS + half * 128 + quarter * 32 + lane];
+        const float2 sc2 = make_float2(scale, scale);
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(pempty_bar(slot));
         if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(tfull_bar(buf), bph))) {
-          record_error(args.err, kErrTimeoutEpilogue);
+          if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
           ok = false;
           break;
         }
@@ -250,28 +338,43 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
           }
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            acc[j * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), sc2, acc[j * 8 + i]);
+          for (int q = 0; q < 8; ++q)
+            acc[j * 8 + q] = __ffma2_rn(make_float2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1])), sc2, acc[j * 8 + q]);
         }
       }
       if (!ok) break;
-      if (row_ok && col_ok) {
-        uint4* dst = reinterpret_cast<uint4*>(args.y + static_cast<int64_t>(row) * N + nb * 128);
+      // bf16 out through shared memory: in four passes of 32 columns the
+      // warp writes its 32 rows x 64 bytes (row r at r * 64) and one TMA
+      // store moves the box to Y (rows past M and columns past N are not
+      // written).
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          __nv_bfloat162 p0 = __float22bfloat162_rn(acc[4 * j + 0]);
-          __nv_bfloat162 p1 = __float22bfloat162_rn(acc[4 * j + 1]);
-          __nv_bfloat162 p2 = __float22bfloat162_rn(acc[4 * j + 2]);
-          __nv_bfloat162 p3 = __float22bfloat162_rn(acc[4 * j + 3]);
-          uint4 o;
-          o.x = *reinterpret_cast<uint32_t*>(&p0);
-          o.y = *reinterpret_cast<uint32_t*>(&p1);
-          o.z = *reinterpret_cast<uint32_t*>(&p2);
-          o.w = *reinterpret_cast<uint32_t*>(&p3);
-          dst[j] = o;
+      for (int pass = 0; pass < 128 / STAGE_COLS; ++pass) {
+        if (lane == 0) ptx::bulk_wait_group_read<0>();   // the staging box is free again
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < STAGE_COLS / 8; ++j) {
+          const int a0 = pass * (STAGE_COLS / 2) + j * 4;
+          __nv_bfloat162 p0 = __float22bfloat162_rn(acc[a0 + 0]);
+          __nv_bfloat162 p1 = __float22bfloat162_rn(acc[a0 + 1]);
+          __nv_bfloat162 p2 = __float22bfloat162_rn(acc[a0 + 2]);
+          __nv_bfloat162 p3 = __float22bfloat162_rn(acc[a0 + 3]);
+          const uint32_t addr = stage + static_cast<uint32_t>(lane * STAGE_COLS * 2 + j * 16);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                       "r"(*reinterpret_cast<uint32_t*>(&p0)), "r"(*reinterpret_cast<uint32_t*>(&p1)),
+                       "r"(*reinterpret_cast<uint32_t*>(&p2)), "r"(*reinterpret_cast<uint32_t*>(&p3))
+                       : "memory");
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && box_ok) {
+          ptx::tma_store_2d(&tmap_y, stage, (nb * 128 + pass * STAGE_COLS) * 2, row0);
+          ptx::bulk_commit_group();
         }
       }
     }
+    // every store has left shared memory before the CTA exits
+    if (lane == 0) ptx::bulk_wait_group<0>();
+    __syncwarp();
   }
 
   ptx::tc_fence_before();
@@ -312,7 +415,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // 2-D map over a row-major byte matrix [rows, cols] with a (box_rows x
 // box_cols) box and the 128-byte swizzle; out-of-range elements read zero.
 bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                  uint32_t box_rows, uint32_t box_cols) {
+                  uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swizzle) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -320,7 +423,7 @@ bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -358,8 +461,9 @@ cudaError_t launch_block_linear(const void* q_a, const float* s_a, const void* q
     return launch_block_linear_decode(q_a, s_a, q_w, s_w, y, M, N, K, workspace, dev, st);
   cudaError_t e = ensure_smem_attr();
   if (e != cudaSuccess) return e;
-  CUtensorMap ta, tb;
-  if (!make_tmap_u8(&ta, q_a, M, K, BM, BK) || !make_tmap_u8(&tb, q_w, N, K, BN, BK))
+  CUtensorMap ta, tb, ty;
+  if (!make_tmap_u8(&ta, q_a, M, K, BM, BK) || !make_tmap_u8(&tb, q_w, N, K, BN, BK) ||
+      !make_tmap_u8(&ty, y, M, 2 * N, STAGE_ROWS, STAGE_COLS * 2, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   GemmArgs a;
   a.s_a = s_a;
@@ -371,7 +475,7 @@ cudaError_t launch_block_linear(const void* q_a, const float* s_a, const void* q
   a.err = dev.error_flag;
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-  gemm_prefill_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, a);
+  gemm_prefill_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, ty, a);
   return cudaGetLastError();
 }
 
