@@ -109,6 +109,12 @@ struct GemmPlan {
 
 GemmPlan plan_block_linear(int64_t M, int64_t N, int64_t K, int sm_count, bool fused);
 
+// Block-scaled GEMM on CTA pairs (256 x 256 tiles), used for M > 128.
+bool block_linear_use_pairs(int64_t M);
+cudaError_t launch_block_linear_pairs(const void* q_a, const float* s_a, const void* q_w,
+                                      const float* s_w, void* y, int64_t M, int64_t N, int64_t K,
+                                      const DeviceInfo& dev, cudaStream_t st);
+
 cudaError_t launch_block_linear(const void* q_a, const float* s_a, const void* q_w,
                                 const float* s_w, void* y, int64_t M, int64_t N, int64_t K,
                                 const GemmPlan& plan, void* workspace, const DeviceInfo& dev,

@@ -459,6 +459,8 @@ cudaError_t launch_block_linear(const void* q_a, const float* s_a, const void* q
   if (M == 0) return cudaSuccess;
   if (plan.kind == 1)
     return launch_block_linear_decode(q_a, s_a, q_w, s_w, y, M, N, K, workspace, dev, st);
+  if (block_linear_use_pairs(M))
+    return launch_block_linear_pairs(q_a, s_a, q_w, s_w, y, M, N, K, dev, st);
   cudaError_t e = ensure_smem_attr();
   if (e != cudaSuccess) return e;
   CUtensorMap ta, tb, ty;

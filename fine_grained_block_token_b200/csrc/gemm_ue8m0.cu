@@ -35,7 +35,10 @@
 //   warps 4-11  epilogue: after the tile's last MMA, warp w reads TMEM lanes
 //               32 (w % 4) .. +31 and columns 128 ((w - 4) / 4) .. +127 with
 //               two 64-column loads, releases the accumulator, and converts
-//               and stores the bf16 row segment.
+//               to bf16 and stores through a shared staging box, 32 columns
+//               at a time, so that each store instruction of the warp writes
+//               eight 64-byte row segments instead of 32 scattered 16-byte
+//               pieces (rows past the segment end are skipped).
 // A single 256-column accumulator is what fits next to the scale-factor
 // columns, so the MMAs of the next tile wait for the epilogue's TMEM reads
 // (not for its stores).
@@ -88,7 +91,11 @@ constexpr int SMEM_BAR_OFF = SMEM_B_OFF + STAGES * B_BYTES;
 constexpr int NUM_BARS = 2 * STAGES + 3;  // full, empty, tfull, tempty, drain
 constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NUM_BARS * 8;
 constexpr int SMEM_TAB_OFF = SMEM_MISC_OFF + 16;   // expert table: offsets, block prefix
-constexpr int SMEM_BYTES = SMEM_TAB_OFF + 2 * (kMaxExperts + 1) * 4 + 1024;  // + alignment slack
+// epilogue staging: 32 rows x 64 bytes (32 bf16 columns) per epilogue warp
+constexpr int STAGE_COLS = 32;
+constexpr int STAGE_WARP_BYTES = 32 * STAGE_COLS * 2;
+constexpr int SMEM_Y_OFF = (SMEM_TAB_OFF + 2 * (kMaxExperts + 1) * 4 + 127) / 128 * 128;
+constexpr int SMEM_BYTES = SMEM_Y_OFF + NUM_EPI_WARPS * STAGE_WARP_BYTES + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(SF_COL0 >= ACC_COL + BN && SF_COL0 + 16 * STAGES <= TMEM_COLS, "TMEM columns");
 
@@ -353,7 +360,6 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
       }
       int e, row0, row_end, n_blk;
       map_tile(tile, e, row0, row_end, n_blk);
-      const int row = row0 + quarter * 32 + lane;
       const int nb = n_blk * 2 + half;
       if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(tfull_bar, t_local & 1u))) {
         if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
@@ -368,19 +374,43 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(tempty_bar);
-      if (row < row_end && nb < nblk_count) {
-        uint4* dst = reinterpret_cast<uint4*>(args.y + static_cast<int64_t>(row) * N + nb * 128);
+      if (nb < nblk_count) {
+        const int wrow0 = row0 + quarter * 32;   // this warp's first row
+        const uint32_t stage =
+            smem_base + SMEM_Y_OFF + static_cast<uint32_t>(warp - 4) * STAGE_WARP_BYTES;
+        const uint8_t* stage_g = smem + SMEM_Y_OFF + (warp - 4) * STAGE_WARP_BYTES;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t* src = j < 8 ? v0 + 8 * j : v1 + 8 * (j - 8);
-          uint32_t o[4];
+        for (int pass = 0; pass < 128 / STAGE_COLS; ++pass) {
+          // my row's 32 columns -> 64 bytes of the staging box
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            __nv_bfloat162 p = __float22bfloat162_rn(
-                make_float2(__uint_as_float(src[2 * i]), __uint_as_float(src[2 * i + 1])));
-            o[i] = *reinterpret_cast<uint32_t*>(&p);
+          for (int j = 0; j < STAGE_COLS / 8; ++j) {
+            const int col = pass * STAGE_COLS + 8 * j;
+            const uint32_t* src = col < 64 ? v0 + col : v1 + (col - 64);
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              __nv_bfloat162 p = __float22bfloat162_rn(
+                  make_float2(__uint_as_float(src[2 * i]), __uint_as_float(src[2 * i + 1])));
+              o[i] = *reinterpret_cast<uint32_t*>(&p);
+            }
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             stage + static_cast<uint32_t>(lane * STAGE_COLS * 2 + 16 * j)),
+                         "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                         : "memory");
           }
-          dst[j] = make_uint4(o[0], o[1], o[2], o[3]);
+          __syncwarp();
+          // out: lane l writes 16 bytes of row (8 it + l / 4); the warp's
+          // instruction covers eight rows' 64-byte segments
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int r = 8 * it + (lane >> 2);
+            const int q = lane & 3;
+            const uint4 val = *reinterpret_cast<const uint4*>(stage_g + r * STAGE_COLS * 2 + 16 * q);
+            if (wrow0 + r < row_end)
+              *reinterpret_cast<uint4*>(args.y + static_cast<int64_t>(wrow0 + r) * N + nb * 128 +
+                                        pass * STAGE_COLS + 8 * q) = val;
+          }
+          __syncwarp();
         }
       }
     }
