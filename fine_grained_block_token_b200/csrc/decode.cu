@@ -28,11 +28,13 @@
 //     completed launch leaves the flags it used cleared, a CUDA graph can
 //     replay its launches with the tags they were captured with.
 // Warps: 0 TMA producer (W tile 128x128 + X tile Mpad x 128 per stage,
-// 9-12 stages), 1 MMA issuer, 2 TMEM owner and counter set-up, 3 scale
+// 8 stages), 1 MMA issuer, 2 TMEM owner and counter set-up, 3 scale
 // products (for every chunk the Mpad factors s_w[blk, j] * s_a[m, j], once
 // per CTA, into a shared ring), 4-11 promotion: two warps per TMEM lane
 // quarter, one weight row per thread, each warp a contiguous part of the
-// token columns.
+// token columns.  Every warp polls its barriers without suspending
+// (mbarrier.test_wait): with suspending waits the weight stream of the large
+// linears ran 5-10% slower on B200.
 // The kernel is launched with programmatic stream serialization: its set-up
 // (barriers, TMEM, tensor-map prefetch) and an L2 prefetch of the weight
 // tiles its first ring fill loads overlap the previous kernel's tail, when
@@ -67,16 +69,16 @@ constexpr int DNUM_THREADS = 384;
 constexpr int PROMO_THREADS = 256;           // warps 4-11
 constexpr int kSmemBudget = 227 * 1024;
 
-// Shared-memory layout for Mpad tokens: as many stages of [W tile 16 KB |
-// X tile Mpad x 128 B] as fit (12 at Mpad 16 down to 9 at Mpad 64: the
-// bytes in flight per SM are what sets the weight stream's rate), then the
-// scale-product ring, the barriers and a few words.
+// Shared-memory layout for Mpad tokens: 8 stages of [W tile 16 KB | X tile
+// Mpad x 128 B] (measured on B200: 9-12 stages streamed no faster and
+// slightly slower at Mpad 16), then the scale-product ring, the barriers and
+// a few words.
 template <int MPAD>
 struct DLayout {
   static constexpr int SB = W_BYTES + MPAD * DBK;            // stage bytes, multiple of 1024
   static constexpr int FIXED = CSLOTS * MAX_MPAD * 4 + (2 * DTBUFS + 2 * CSLOTS + 1) * 8 + 16 + 1024;
   static constexpr int NS_FIT = (kSmemBudget - FIXED) / (SB + 16);
-  static constexpr int NS = NS_FIT < 12 ? NS_FIT : 12;       // stages
+  static constexpr int NS = NS_FIT < 8 ? NS_FIT : 8;         // stages
   static constexpr int C_OFF = NS * SB;
   static constexpr int BAR_OFF = C_OFF + CSLOTS * MAX_MPAD * 4;
   static constexpr int NUM_BARS = 2 * NS + 2 * DTBUFS + 2 * CSLOTS + 1;
@@ -166,7 +168,7 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
     const int slot = c % CSLOTS;
     const uint32_t cph = (c / CSLOTS) & 1u;
     if (NC > 0 && ok) {
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(L::bar(cx.smem_base, L::tfull(buf)), bph))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(L::bar(cx.smem_base, L::tfull(buf)), bph))) {
         if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
         ok = false;
       } else {
@@ -181,7 +183,7 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(L::bar(cx.smem_base, L::tempty(buf)));
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(L::bar(cx.smem_base, L::cfull(slot)), cph))) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(L::bar(cx.smem_base, L::cfull(slot)), cph))) {
           if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
           ok = false;
         } else {
@@ -365,7 +367,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     for (int64_t u = u_begin; u < u_end; ++u, ++c, (++kb == KB ? (kb = 0, ++blk) : 0)) {
       const int s = c % NS;
       const uint32_t ph = (c / NS) & 1u;
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::empty(s)), ph ^ 1u))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(bar(L::empty(s)), ph ^ 1u))) {
         if (lane == 0) record_error(args.err, kErrTimeoutProducer);
         break;
       }
@@ -458,11 +460,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     // prods[slot][m] = s_w[blk, kb] * s_a[m, kb] for every chunk of the
     // range, up to CSLOTS chunks ahead of the promotion warps.  Lane l
     // covers tokens l and l + 32.  The scales of a chunk are loaded PF
-    // chunks ahead (L2 path: another kernel wrote them; under a full HBM
-    // stream an L2 read can take microseconds) into a register slot that is
-    // refilled right after its use.  s_w of unit u is s_w[u] (row-major
-    // [NB, KB]).
-    constexpr int PF = 8;
+    // chunks ahead (L2 path: another kernel wrote them) into a register
+    // slot that is refilled right after its use.  s_w of unit u is s_w[u]
+    // (row-major [NB, KB]).
+    constexpr int PF = 4;
     float pw[PF], plo[PF], phi[PF];
     auto load_scales = [&](int64_t uu, float& w, float& lo, float& hi) {
       w = lo = hi = 0.0f;
@@ -488,7 +489,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         const int slot = c % CSLOTS;
         const uint32_t ph = (c / CSLOTS) & 1u;
         ++c;
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::cempty(slot)), ph ^ 1u))) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin(bar(L::cempty(slot)), ph ^ 1u))) {
           if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
           ok = false;
           break;
