@@ -83,6 +83,7 @@ def peaks():
 KERNEL_SOURCES = {
     "gemm_prefill_kernel": ("gemm.cu", "ptx_sm100.cuh", "quant_math.cuh"),
     "gemm_ue8m0_kernel": ("gemm_ue8m0.cu", "ptx_sm100.cuh"),
+    "gemm_ue8m0_pair_kernel": ("gemm_ue8m0_pair.cu", "ptx_sm100.cuh"),
     "gemm_rowwise_kernel": ("gemm_rowwise.cu", "ptx_sm100.cuh"),
     "gemm_rowwise_pair_kernel": ("gemm_rowwise.cu", "ptx_sm100.cuh"),
 }
@@ -1180,7 +1181,8 @@ def run_ours(args):
         wbits = {lb: wb for lb, _, wb in lins}
         specs = {
             "ue8m0": dict(wq=fp8.quant_weight_ue8m0, aq=fp8.quant_act_ue8m0,
-                          gemm=fp8.block_linear_ue8m0, kernel="gemm_ue8m0_kernel",
+                          gemm=fp8.block_linear_ue8m0, kernel="gemm_ue8m0_pair_kernel",
+                          ws=fp8.ue8m0_workspace_bytes,
                           s_a=lambda it: torch.empty((it["M"], it["K"] // 128),
                                                      dtype=torch.float8_e8m0fnu, device=dev)),
             "fp8r": dict(wq=fp8.quant_rowwise, aq=fp8.quant_rowwise,
@@ -1195,15 +1197,21 @@ def run_ours(args):
                 w = wl.to_torch_bf16(wbits[it["label"]]).to(dev)
                 q_wv, s_wv = sp["wq"](w)
                 del w
+                ws_n = sp["ws"](it["M"], it["N"], it["K"]) if "ws" in sp else 0
                 v_items.append(dict(it=it, q_w=q_wv, s_w=s_wv, q_a=torch.empty_like(it["q_a"]),
-                                    s_a=sp["s_a"](it), y=torch.empty_like(it["y"])))
+                                    s_a=sp["s_a"](it), y=torch.empty_like(it["y"]),
+                                    ws=torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
+                                    if ws_n else None))
 
             def v_step(ev=None, v_items=v_items, sp=sp):
                 for i, u in enumerate(v_items):
                     sp["aq"](u["it"]["x"], u["q_a"], u["s_a"])
                     if ev is not None:
                         ev[2 * i].record()
-                    sp["gemm"](u["q_a"], u["s_a"], u["q_w"], u["s_w"], u["y"])
+                    if u["ws"] is not None:
+                        sp["gemm"](u["q_a"], u["s_a"], u["q_w"], u["s_w"], u["y"], workspace=u["ws"])
+                    else:
+                        sp["gemm"](u["q_a"], u["s_a"], u["q_w"], u["s_w"], u["y"])
                     if ev is not None:
                         ev[2 * i + 1].record()
 

@@ -23,6 +23,7 @@ __all__ = [
     "Fp8blError", "BLOCK", "lib_path", "quant_act", "quant_weight", "block_linear",
     "block_linear_fused", "block_linear_noalloc", "workspace_bytes", "fused_workspace_bytes",
     "check", "version", "quant_act_ue8m0", "quant_weight_ue8m0", "block_linear_ue8m0",
+    "ue8m0_workspace_bytes",
     "quant_rowwise", "linear_rowwise", "quant_act_static", "grouped_linear_ue8m0",
 ]
 
@@ -48,6 +49,9 @@ _lib.fp8_block_linear_fused_workspace_bytes.restype = _sz
 _lib.fp8_quant_act_ue8m0.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_quant_weight_ue8m0.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_block_linear_ue8m0.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
+_lib.fp8_block_linear_ue8m0_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp]
+_lib.fp8_block_linear_ue8m0_workspace_bytes.argtypes = [_i64, _i64, _i64]
+_lib.fp8_block_linear_ue8m0_workspace_bytes.restype = _sz
 _lib.fp8_quant_rowwise.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_quant_act_static.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp, _vp]
 _lib.fp8_grouped_linear_ue8m0.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]
@@ -58,7 +62,8 @@ _lib.fp8bl_status_string.restype = ctypes.c_char_p
 _lib.fp8bl_version.restype = ctypes.c_int
 for _f in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_linear_fused",
            "fp8_block_linear_noalloc", "fp8bl_check", "fp8_quant_act_ue8m0",
-           "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0", "fp8_quant_rowwise",
+           "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0", "fp8_block_linear_ue8m0_ws",
+           "fp8_quant_rowwise",
            "fp8_linear_rowwise", "fp8_quant_act_static", "fp8_grouped_linear_ue8m0"):
     getattr(_lib, _f).restype = ctypes.c_int
 
@@ -246,9 +251,12 @@ def quant_weight_ue8m0(w: torch.Tensor, q: torch.Tensor | None = None,
     return q, s
 
 
-def block_linear_ue8m0(q_a, s_a, q_w, s_w, y=None) -> torch.Tensor:
+def block_linear_ue8m0(q_a, s_a, q_w, s_w, y=None, workspace=None, pairs=True) -> torch.Tensor:
     """(e4m3 [M,K], e8m0 [M,K/128], e4m3 [N,K], e8m0 [N/128,K/128]) -> bf16 [M,N],
-    on the tensor core's block-scaled MMA."""
+    on the tensor core's block-scaled MMA.  With pairs=True (the default) the
+    call goes through fp8_block_linear_ue8m0_ws, which runs M > 128 on CTA
+    pairs with a workspace (allocated here unless given); pairs=False calls
+    the workspace-free single-CTA fp8_block_linear_ue8m0."""
     dev = _device_of(q_a, "q_a")
     M, K = _dims2(q_a, "q_a")
     N = _dims2(q_w, "q_w")[0]
@@ -259,9 +267,19 @@ def block_linear_ue8m0(q_a, s_a, q_w, s_w, y=None) -> torch.Tensor:
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
     _need(y, "y", _BF16, (M, N), dev)
-    _ok(_lib.fp8_block_linear_ue8m0(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
-                                    _stream(q_a)), "fp8_block_linear_ue8m0")
+    if not pairs:
+        _ok(_lib.fp8_block_linear_ue8m0(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
+                                        _stream(q_a)), "fp8_block_linear_ue8m0")
+        return y
+    ws, wsb = _workspace(ue8m0_workspace_bytes(M, N, K), q_a.device, workspace)
+    _ok(_lib.fp8_block_linear_ue8m0_ws(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
+                                       _ptr(ws), wsb, _stream(q_a)), "fp8_block_linear_ue8m0_ws")
     return y
+
+
+def ue8m0_workspace_bytes(M: int, N: int, K: int) -> int:
+    """Workspace bytes fp8_block_linear_ue8m0_ws needs for these sizes."""
+    return int(_lib.fp8_block_linear_ue8m0_workspace_bytes(M, N, K))
 
 
 def grouped_linear_ue8m0(q_a, s_a, q_w, s_w, expert_offsets, y=None) -> torch.Tensor:

@@ -14,7 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp8bl.so")
-SOURCES = ["api.cu", "quant.cu", "gemm.cu", "gemm_pair.cu", "gemm_ue8m0.cu", "gemm_rowwise.cu", "decode.cu", "fused.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quant.cu", "gemm.cu", "gemm_pair.cu", "gemm_ue8m0.cu", "gemm_ue8m0_pair.cu", "gemm_rowwise.cu", "decode.cu", "fused.cu", "noalloc.cu"]
 HEADERS = ["fp8bl_internal.h", "ptx_sm100.cuh", "quant_math.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include", "fp8bl.h")
 

@@ -271,6 +271,45 @@ fp8bl_status fp8_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const v
       launch_block_linear_ue8m0(q_a, s_a, q_w, s_w, y_bf16, M, N, K, *d, as_cuda(stream)));
 }
 
+size_t fp8_block_linear_ue8m0_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (!linear_dims_ok(M, N, K)) return 0;
+  return ue8m0_pair_workspace_bytes(M, N, K);
+}
+
+fp8bl_status fp8_block_linear_ue8m0_ws(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                       const uint8_t* s_w, void* y_bf16, int64_t M, int64_t N,
+                                       int64_t K, void* workspace, size_t workspace_bytes,
+                                       fp8bl_stream_t stream) {
+  if (!linear_dims_ok(M, N, K)) return FP8BL_ERR_SHAPE;
+  if (M == 0) return FP8BL_OK;
+  if (!q_a || !s_a || !q_w || !s_w || !y_bf16) return FP8BL_ERR_NULL;
+  if (!aligned(q_a, 16) || !aligned(q_w, 16) || !aligned(y_bf16, 16) || !aligned(workspace, 16))
+    return FP8BL_ERR_ALIGN;
+  const size_t ny = static_cast<size_t>(M * N) * 2;
+  const size_t na = static_cast<size_t>(M * K), nw = static_cast<size_t>(N * K);
+  const size_t nsa = static_cast<size_t>(M * (K / 128)), nsw = static_cast<size_t>((N / 128) * (K / 128));
+  if (overlap(y_bf16, ny, q_a, na) || overlap(y_bf16, ny, q_w, nw) || overlap(y_bf16, ny, s_a, nsa) ||
+      overlap(y_bf16, ny, s_w, nsw))
+    return FP8BL_ERR_OVERLAP;
+  const size_t need = ue8m0_pair_workspace_bytes(M, N, K);
+  if (need > 0) {
+    if (!workspace) return FP8BL_ERR_NULL;
+    if (workspace_bytes < need) return FP8BL_ERR_WORKSPACE;
+    if (overlap(workspace, need, y_bf16, ny) || overlap(workspace, need, q_a, na) ||
+        overlap(workspace, need, q_w, nw) || overlap(workspace, need, s_a, nsa) ||
+        overlap(workspace, need, s_w, nsw))
+      return FP8BL_ERR_OVERLAP;
+  }
+  const DeviceInfo* d = nullptr;
+  fp8bl_status st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  if (need == 0)
+    return from_cuda(
+        launch_block_linear_ue8m0(q_a, s_a, q_w, s_w, y_bf16, M, N, K, *d, as_cuda(stream)));
+  return from_cuda(launch_block_linear_ue8m0_pairs(q_a, s_a, q_w, s_w, y_bf16, M, N, K, workspace,
+                                                   *d, as_cuda(stream)));
+}
+
 fp8bl_status fp8_grouped_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
                                       const uint8_t* s_w, const int32_t* expert_offsets,
                                       void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t E,

@@ -77,6 +77,15 @@ cudaError_t launch_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const
                                       const uint8_t* s_w, void* y, int64_t M, int64_t N,
                                       int64_t K, const DeviceInfo& dev, cudaStream_t st);
 
+// UE8M0 block-scaled GEMM on CTA pairs (M > 128): the workspace holds the
+// scale factors rewritten in the tensor core's order.
+bool ue8m0_use_pairs(int64_t M);
+size_t ue8m0_pair_workspace_bytes(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_block_linear_ue8m0_pairs(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                            const uint8_t* s_w, void* y, int64_t M, int64_t N,
+                                            int64_t K, void* workspace, const DeviceInfo& dev,
+                                            cudaStream_t st);
+
 // Row-wise e4m3 quantization ("BFL (fp8r / nvfp4)"): bf16 [R, K] -> e4m3
 // [R, K] + one fp32 scale per row; K % 16 == 0.
 cudaError_t launch_rowwise_quant(const void* x, int64_t R, int64_t K, void* q, float* s,

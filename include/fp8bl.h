@@ -244,6 +244,26 @@ fp8bl_status fp8_block_linear_ue8m0(const void *q_a, const uint8_t *s_a,
                                     fp8bl_stream_t stream);
 
 /*
+ * fp8_block_linear_ue8m0_ws -- the same linear with a caller workspace, which
+ * lets M > 128 run on CTA pairs (tcgen05.mma.cta_group::2, 256 x 256 tiles):
+ * two small kernels first rewrite s_a and s_w into the workspace in the
+ * order the tensor core reads scale factors, so that they travel with the
+ * operands.  Same passage, arguments and result as fp8_block_linear_ue8m0
+ * (bit for bit: the same MMAs in the same K order), plus
+ *   workspace: device scratch of at least
+ *              fp8_block_linear_ue8m0_workspace_bytes(M, N, K) bytes
+ *              (16-byte aligned), or NULL when that size is 0 (M <= 128:
+ *              the single-CTA kernel, no workspace).  Contents on entry are
+ *              ignored; it must not overlap any argument.
+ */
+size_t fp8_block_linear_ue8m0_workspace_bytes(int64_t M, int64_t N, int64_t K);
+fp8bl_status fp8_block_linear_ue8m0_ws(const void *q_a, const uint8_t *s_a,
+                                       const void *q_w, const uint8_t *s_w,
+                                       void *y_bf16, int64_t M, int64_t N, int64_t K,
+                                       void *workspace, size_t workspace_bytes,
+                                       fp8bl_stream_t stream);
+
+/*
  * fp8_grouped_linear_ue8m0 -- grouped (MoE expert) form of
  * fp8_block_linear_ue8m0.
  * Passage: "Fine-grained FP8" page, "DeepGEMM fast path" section (MoE expert

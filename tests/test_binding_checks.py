@@ -126,3 +126,14 @@ def test_binding_argtypes_match_the_header():
         assert len(f.argtypes) == n, (name, len(f.argtypes), n)
         checked += 1
     assert checked >= 15
+
+
+def test_package_exports_every_binding_name():
+    """Every public name of the ctypes binding is reachable from the package
+    (its lazy re-export list), so a new entry point cannot go missing there."""
+    import fine_grained_block_token_b200 as pkg
+    from fine_grained_block_token_b200 import _binding
+    missing = set(_binding.__all__) - set(pkg.__all__)
+    assert not missing, missing
+    for name in _binding.__all__:
+        assert getattr(pkg, name) is getattr(_binding, name)

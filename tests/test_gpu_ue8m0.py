@@ -184,3 +184,45 @@ def test_full_size_sweep(fp8):
 
 def test_no_timeout_recorded(fp8):
     fp8.check()
+
+
+@pytest.mark.parametrize("M,N,K", [(129, 384, 384), (256, 512, 512), (300, 1152, 1280),
+                                   (4096 + 128, 1024, 2048), (1000, 28672, 512)])
+def test_pairs_equal_single_cta(fp8, M, N, K):
+    """The CTA-pair schedule (fp8_block_linear_ue8m0_ws, M > 128) runs the
+    same block-scaled MMAs in the same K order as the single-CTA kernel
+    (fp8_block_linear_ue8m0): the outputs must be equal bit for bit, here on
+    random codes with scale codes spread over 2^+-20 so that a scale factor
+    copied to the wrong TMEM lane, column or slice shows."""
+    g = np.random.default_rng(7 * M + N + K)
+    qa = g.integers(0, 256, (M, K), dtype=np.uint8)
+    qw = g.integers(0, 256, (N, K), dtype=np.uint8)
+    qa[(qa & 0x7F) == 0x7F] = 0x00
+    qw[(qw & 0x7F) == 0x7F] = 0x00
+    ca = g.integers(107, 148, (M, K // 128), dtype=np.uint8)
+    cw = g.integers(107, 148, (N // 128, K // 128), dtype=np.uint8)
+    dev = lambda a: torch.from_numpy(a).cuda()
+    args = (dev(qa).view(torch.float8_e4m3fn), dev(ca).view(torch.float8_e8m0fnu),
+            dev(qw).view(torch.float8_e4m3fn), dev(cw).view(torch.float8_e8m0fnu))
+    assert fp8.ue8m0_workspace_bytes(M, N, K) > 0
+    y_pair = fp8.block_linear_ue8m0(*args)
+    y_single = fp8.block_linear_ue8m0(*args, pairs=False)
+    fp8.check()
+    assert torch.equal(y_pair.view(torch.int16), y_single.view(torch.int16)), (M, N, K)
+    rows = _sample_rows(M, 8, seed=M)
+    R = oracle.block_linear_ue8m0(qa, ca, qw, cw, rows=rows, nthreads=8)
+    check_gemm(f32(y_pair[torch.as_tensor(rows, device=y_pair.device)]), R, f"pairs {M}x{N}x{K}")
+
+
+def test_pairs_workspace_checks(fp8):
+    M, N, K = 256, 256, 256
+    need = fp8.ue8m0_workspace_bytes(M, N, K)
+    assert need > 0 and fp8.ue8m0_workspace_bytes(128, N, K) == 0
+    z = lambda *s: torch.zeros(s, dtype=torch.uint8, device="cuda")
+    q_a, q_w = z(M, K).view(torch.float8_e4m3fn), z(N, K).view(torch.float8_e4m3fn)
+    s_a = torch.full((M, K // 128), 127, dtype=torch.uint8, device="cuda").view(torch.float8_e8m0fnu)
+    s_w = torch.full((N // 128, K // 128), 127, dtype=torch.uint8, device="cuda").view(torch.float8_e8m0fnu)
+    with pytest.raises(fp8.Fp8blError) as ei:
+        fp8.block_linear_ue8m0(q_a, s_a, q_w, s_w, workspace=z(need - 16))
+    assert ei.value.status == 7
+    fp8.check()
