@@ -119,8 +119,17 @@ struct DecodeArgs {
   int* err;
 };
 
+// a / b for a >= 0, b > 0, by a 32-bit division when a fits in 32 bits
+// (always, for the sizes a decode meets; the 64-bit division is a long
+// software sequence on the reduction's critical path).
+__device__ __forceinline__ int64_t div_nonneg(int64_t a, int64_t b) {
+  if ((static_cast<uint64_t>(a) | static_cast<uint64_t>(b)) <= 0xffffffffull)
+    return static_cast<uint32_t>(a) / static_cast<uint32_t>(b);
+  return a / b;
+}
+
 __device__ __forceinline__ int64_t range_start(int g, int64_t units, int G) {
-  return (static_cast<int64_t>(g) * units) / G;
+  return div_nonneg(static_cast<int64_t>(g) * units, G);
 }
 
 __device__ __forceinline__ void record_error(int* err, int code) { atomicCAS(err, 0, code); }
@@ -191,10 +200,17 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
 #pragma unroll
           for (int j = 0; j < NC / 4; ++j) {
             const float4 p = cr[j];
-            acc[4 * j + 0] = __fmaf_rn(__uint_as_float(v[4 * j + 0]), p.x, acc[4 * j + 0]);
-            acc[4 * j + 1] = __fmaf_rn(__uint_as_float(v[4 * j + 1]), p.y, acc[4 * j + 1]);
-            acc[4 * j + 2] = __fmaf_rn(__uint_as_float(v[4 * j + 2]), p.z, acc[4 * j + 2]);
-            acc[4 * j + 3] = __fmaf_rn(__uint_as_float(v[4 * j + 3]), p.w, acc[4 * j + 3]);
+            // packed f32x2 FMAs: each lane an IEEE fma, as fmaf would give
+            const float2 lo = __ffma2_rn(
+                make_float2(__uint_as_float(v[4 * j + 0]), __uint_as_float(v[4 * j + 1])),
+                make_float2(p.x, p.y), make_float2(acc[4 * j + 0], acc[4 * j + 1]));
+            const float2 hi = __ffma2_rn(
+                make_float2(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])),
+                make_float2(p.z, p.w), make_float2(acc[4 * j + 2], acc[4 * j + 3]));
+            acc[4 * j + 0] = lo.x;
+            acc[4 * j + 1] = lo.y;
+            acc[4 * j + 2] = hi.x;
+            acc[4 * j + 3] = hi.y;
           }
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(L::bar(cx.smem_base, L::cempty(slot)));
@@ -215,14 +231,16 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
         float* dst = args.partial +
                      (static_cast<int64_t>(cx.g) * args.maxseg + (blk - first_blk)) * (MPAD * 128);
 #pragma unroll
-        for (int m = 0; m < NC; ++m) dst[(COL0 + m) * 128 + n_local] = acc[m];
+        for (int m = 0; m < NC; ++m)
+          if (COL0 + m < args.M) dst[(COL0 + m) * 128 + n_local] = acc[m];
         // Publish the partial and count this CTA in; the last one reduces.
         // The barrier orders every thread's stores before one thread's
-        // fence + atomic (the fence is cumulative), as a grid-wide barrier
-        // does; the last CTA fences again before reading.
+        // acquire-release atomic (a release covers what the barrier ordered
+        // before it); the last CTA's acquire makes the other partials
+        // visible, and the second barrier orders its threads' reads after it.
         ptx::named_barrier_sync(1, PROMO_THREADS);
-        const int g_lo = static_cast<int>(((blk_u0 + 1) * args.G - 1) / args.units);
-        const int g_hi = static_cast<int>(((blk_u0 + KB) * args.G - 1) / args.units);
+        const int g_lo = static_cast<int>(div_nonneg((blk_u0 + 1) * args.G - 1, args.units));
+        const int g_hi = static_cast<int>(div_nonneg((blk_u0 + KB) * args.G - 1, args.units));
         if (threadIdx.x == 128) {
           // the block's counter must have been set up for this launch (by
           // this CTA's warp 2, or by the CTA holding the block's first chunk)
@@ -230,12 +248,12 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
           while (cx.misc[kMiscReady] == 0 && clock64() - t0 < (1ull << 32)) __nanosleep(32);
           bool last = false;
           if (cx.misc[kMiscReady] == 1) {
-            __threadfence();
-            last = atomicAdd(args.counters + blk, 1u) == static_cast<unsigned>(g_hi - g_lo);
+            last = ptx::atomic_add_acq_rel_gpu(args.counters + blk, 1u) ==
+                   static_cast<unsigned>(g_hi - g_lo);
             if (last) {
               // every contributor has counted in: the flag is free again
+              // (the launch's end orders this store before the next launch)
               *reinterpret_cast<volatile unsigned long long*>(args.flags + blk) = 0ull;
-              __threadfence();
             }
           } else {
             record_error(args.err, kErrTimeoutEpilogue);
@@ -253,6 +271,36 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
           constexpr int UR = HALF <= 8 ? 8 : (HALF <= 16 ? 4 : 2);
           const int t = threadIdx.x - 128;
           const int rn = t & 127;
+          const int64_t yo = static_cast<int64_t>(blk) * 128 + rn;
+          // Partial of contributor gi for this block: segment 0 of CTA gi,
+          // except for g_lo, whose range may start in an earlier block.
+          const int seg_lo =
+              blk - static_cast<int>(div_nonneg(range_start(g_lo, args.units, args.G), KB));
+          auto part = [&](int gi) {
+            return args.partial +
+                   (static_cast<int64_t>(gi) * args.maxseg + (gi == g_lo ? seg_lo : 0)) * (MPAD * 128);
+          };
+          if (args.M <= 2) {
+            // one or two tokens: thread t sums row t % 128 of token t / 128,
+            // with up to 16 partials' loads in flight (same order, same sums)
+            constexpr int URS = 16;
+            const int m = t >> 7;
+            if (m < args.M) {
+              float acc1 = 0.0f;
+              for (int gg = g_lo; gg <= g_hi; gg += URS) {
+                float tv[URS];
+#pragma unroll
+                for (int r = 0; r < URS; ++r) {
+                  const int gi = gg + r <= g_hi ? gg + r : g_hi;
+                  tv[r] = __ldcg(part(gi) + m * 128 + rn);
+                }
+#pragma unroll
+                for (int r = 0; r < URS; ++r)
+                  if (gg + r <= g_hi) acc1 += tv[r];
+              }
+              args.y[static_cast<int64_t>(m) * args.N + yo] = __float2bfloat16_rn(acc1);
+            }
+          } else {
           const int m0 = (t >> 7) * HALF;
           float sum[HALF];
 #pragma unroll
@@ -262,12 +310,9 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
 #pragma unroll
             for (int r = 0; r < UR; ++r) {
               const int gi = gg + r <= g_hi ? gg + r : g_hi;
-              const int fb = static_cast<int>(range_start(gi, args.units, args.G) / KB);
-              const float* src = args.partial +
-                                 (static_cast<int64_t>(gi) * args.maxseg + (blk - fb)) * (MPAD * 128) +
-                                 m0 * 128 + rn;
+              const float* src = part(gi) + m0 * 128 + rn;
 #pragma unroll
-              for (int m = 0; m < HALF; ++m) tv[r][m] = __ldcg(src + m * 128);
+              for (int m = 0; m < HALF; ++m) tv[r][m] = m0 + m < args.M ? __ldcg(src + m * 128) : 0.0f;
             }
 #pragma unroll
             for (int r = 0; r < UR; ++r)
@@ -276,11 +321,11 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
                 for (int m = 0; m < HALF; ++m) sum[m] += tv[r][m];
               }
           }
-          const int64_t yo = static_cast<int64_t>(blk) * 128 + rn;
 #pragma unroll
           for (int m = 0; m < HALF; ++m)
             if (m0 + m < args.M)
               args.y[static_cast<int64_t>(m0 + m) * args.N + yo] = __float2bfloat16_rn(sum[m]);
+          }
         }
       }
 #pragma unroll
@@ -389,8 +434,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     // The whole warp runs the loop (the wait results are made warp-uniform
-    // with a vote) and lane 0 issues: measured on B200, a loop run by lane 0
-    // alone with a data-dependent exit costs ~600 cycles per chunk.
+    // with a vote) and an elected lane issues.  Measured on B200 (cycle
+    // counters per chunk): a loop run by lane 0 alone with a data-dependent
+    // exit cost ~600 cycles; issuing the 4 MMAs from a `lane == 0` branch
+    // took ~270 cycles against ~25 from an elect.sync block, which moved the
+    // gate+up stream from ~1,050 to ~800 cycles per chunk.
+    const uint64_t desc0 = ptx::sdesc_kmajor_sw128(smem_base);
     uint32_t c = 0;
     bool issued = false;
     for (int64_t u = u_begin; u < u_end; ++u, ++c) {
@@ -404,21 +453,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         break;
       }
       ptx::tc_fence_after();
-      if (lane == 0) {
-        const uint32_t w_addr = smem_base + s * L::SB;
-        const uint32_t x_addr = w_addr + W_BYTES;
-        const uint32_t d = tmem_base + static_cast<uint32_t>(buf * MAX_MPAD);
+      const uint64_t dw = ptx::sdesc_advance(desc0, s * L::SB);
+      const uint64_t dx = ptx::sdesc_advance(dw, W_BYTES);
+      const uint32_t d = tmem_base + static_cast<uint32_t>(buf * MAX_MPAD);
+      if (ptx::elect_one()) {
 #pragma unroll
         for (int k = 0; k < DBK / DUMMA_K; ++k)
-          ptx::mma_f8f6f4(d, ptx::sdesc_kmajor_sw128(w_addr + k * DUMMA_K),
-                          ptx::sdesc_kmajor_sw128(x_addr + k * DUMMA_K), IDESC, k > 0 ? 1u : 0u);
+          ptx::mma_f8f6f4(d, ptx::sdesc_advance(dw, k * DUMMA_K), ptx::sdesc_advance(dx, k * DUMMA_K),
+                          IDESC, k > 0 ? 1u : 0u);
         ptx::mma_commit(bar(L::tfull(buf)));
         ptx::mma_commit(bar(L::empty(s)));
       }
-      __syncwarp();
       issued = true;
     }
-    if (issued && lane == 0) {
+    if (issued && ptx::elect_one()) {
       ptx::mma_commit(bar(L::drain()));
       if (!ptx::mbar_wait(bar(L::drain()), 0)) record_error(args.err, kErrTimeoutMma);
     }

@@ -26,7 +26,7 @@
 //                stage s of every CTA of the cluster, in the K-major 128-byte
 //                swizzled layout the MMA reads, and the scales into a ring,
 //                once every CTA's MMA has released stage s (multicast commit).
-//   warp 1       MMA issuer (warp-wide loop, lane 0 issues): 4 MMAs per chunk
+//   warp 1       MMA issuer (warp-wide loop, one elected lane issues): 4 MMAs per chunk
 //                (M=128, N=256, K=32) into one of two 256-column TMEM buffers.
 //   warp 2       TMEM owner, then the slice sender: once the quantizers
 //                have written their rows, bulk-copies them (and the scales)
@@ -285,7 +285,7 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
           break;
         }
         ptx::tc_fence_after();
-        if (lane == 0) {
+        if (ptx::elect_one()) {
           const uint32_t a_addr = smem_base + SMEM_A_OFF + s * A_BYTES;
           const uint32_t b_addr = smem_base + SMEM_B_OFF + s * B_BYTES;
           const uint32_t d = tmem_base + buf * BN;
@@ -301,7 +301,7 @@ gemm_fused_kernel(const __grid_constant__ CUtensorMap tmap_x,
         issued = true;
       }
     }
-    if (issued && lane == 0) {
+    if (issued && ptx::elect_one()) {
       // All MMAs (and the arrivals their commits make) finish first.
       ptx::mma_commit(drain_bar);
       if (!ptx::mbar_wait(drain_bar, 0)) record_error(args.err, kErrTimeoutMma);

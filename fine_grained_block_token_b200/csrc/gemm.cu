@@ -14,7 +14,7 @@
 //   warp 0      TMA producer: A tile 128x128 and W tile 256x128 (e4m3,
 //               128-byte swizzle) into a 4-deep shared-memory ring.
 //   warp 1      MMA issuer: the whole warp runs the loop and waits (the
-//               wait results made warp-uniform by a vote), lane 0 issues
+//               wait results made warp-uniform by a vote), an elected lane issues
 //               4 MMAs per chunk (M=128, N=256, K=32) into one of two
 //               256-column TMEM buffers, then commits to release the stage
 //               and to mark the buffer full.  (A loop run by lane 0 alone,
@@ -186,6 +186,8 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     {
+      const uint64_t desc_a = ptx::sdesc_kmajor_sw128(smem_base + SMEM_A_OFF);
+      const uint64_t desc_b = ptx::sdesc_kmajor_sw128(smem_base + SMEM_B_OFF);
       uint32_t c = 0;
       bool ok = true, issued = false;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
@@ -201,23 +203,21 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             break;
           }
           ptx::tc_fence_after();
-          if (lane == 0) {
-            const uint32_t a_addr = smem_base + SMEM_A_OFF + s * A_BYTES;
-            const uint32_t b_addr = smem_base + SMEM_B_OFF + s * B_BYTES;
-            const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+          const uint64_t da = ptx::sdesc_advance(desc_a, s * A_BYTES);
+          const uint64_t db = ptx::sdesc_advance(desc_b, s * B_BYTES);
+          const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+          if (ptx::elect_one()) {
 #pragma unroll
-            for (int k = 0; k < BK / UMMA_K; ++k) {
-              ptx::mma_f8f6f4(d, ptx::sdesc_kmajor_sw128(a_addr + k * UMMA_K),
-                              ptx::sdesc_kmajor_sw128(b_addr + k * UMMA_K), IDESC, k > 0 ? 1u : 0u);
-            }
+            for (int k = 0; k < BK / UMMA_K; ++k)
+              ptx::mma_f8f6f4(d, ptx::sdesc_advance(da, k * UMMA_K), ptx::sdesc_advance(db, k * UMMA_K),
+                              IDESC, k > 0 ? 1u : 0u);
             ptx::mma_commit(empty_bar(s));
             ptx::mma_commit(tfull_bar(buf));
           }
-          __syncwarp();
           issued = true;
         }
       }
-      if (issued && lane == 0) {
+      if (issued && ptx::elect_one()) {
         // All MMAs finish before the TMEM they write is released.
         ptx::mma_commit(drain_bar);
         if (!ptx::mbar_wait(drain_bar, 0)) record_error(args.err, kErrTimeoutMma);

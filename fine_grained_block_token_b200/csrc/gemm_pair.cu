@@ -190,7 +190,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             break;
           }
           ptx::tc_fence_after();
-          if (lane == 0) {
+          if (ptx::elect_one()) {
             const uint32_t a_addr = smem_base + SMEM_A_OFF + s * HALF_A;
             const uint32_t b_addr = smem_base + SMEM_B_OFF + s * HALF_B;
             const uint32_t d = tmem_base + static_cast<uint32_t>(buf * PBN);
@@ -205,7 +205,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           issued = true;
         }
       }
-      if (issued && lane == 0) ptx::mma_commit_pair_multicast(drain_bar, kBoth);
+      if (issued && ptx::elect_one()) ptx::mma_commit_pair_multicast(drain_bar, kBoth);
       __syncwarp();
     }
     // both CTAs: every MMA into this CTA's TMEM and shared memory is done

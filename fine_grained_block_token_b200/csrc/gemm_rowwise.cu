@@ -13,7 +13,7 @@
 //   warp 0      TMA producer: A 128x128 and W 256x128 e4m3 tiles (128-byte
 //               swizzle; the tail of K past the matrix reads as zero) into a
 //               4-deep shared-memory ring.
-//   warp 1      MMA issuer (whole warp loops and waits, lane 0 issues): 4
+//   warp 1      MMA issuer (whole warp loops and waits, an elected lane issues): 4
 //               MMAs (M=128, N=256, K=32) per stage into the tile's
 //               accumulator, one of two 256-column TMEM buffers (tile t uses
 //               buffer t % 2, so a tile's epilogue overlaps the next tile's
@@ -177,7 +177,7 @@ gemm_rowwise_kernel(const __grid_constant__ CUtensorMap tmap_a,
           break;
         }
         ptx::tc_fence_after();
-        if (lane == 0) {
+        if (ptx::elect_one()) {
           const uint32_t a_addr = smem_base + SMEM_A_OFF + s * A_BYTES;
           const uint32_t b_addr = smem_base + SMEM_B_OFF + s * B_BYTES;
 #pragma unroll
@@ -192,7 +192,7 @@ gemm_rowwise_kernel(const __grid_constant__ CUtensorMap tmap_a,
         issued = true;
       }
     }
-    if (issued && lane == 0) {
+    if (issued && ptx::elect_one()) {
       // All MMAs finish before the TMEM they write is released.
       ptx::mma_commit(drain_bar);
       if (!ptx::mbar_wait(drain_bar, 0)) record_error(args.err, kErrTimeoutMma);
@@ -384,7 +384,7 @@ gemm_rowwise_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
             break;
           }
           ptx::tc_fence_after();
-          if (lane == 0) {
+          if (ptx::elect_one()) {
             const uint32_t a_addr = smem_base + PSMEM_A_OFF + s * PA_BYTES;
             const uint32_t b_addr = smem_base + PSMEM_B_OFF + s * PB_BYTES;
 #pragma unroll
@@ -399,7 +399,7 @@ gemm_rowwise_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
           issued = true;
         }
       }
-      if (issued && lane == 0) ptx::mma_commit_pair_multicast(drain_bar, kBoth);
+      if (issued && ptx::elect_one()) ptx::mma_commit_pair_multicast(drain_bar, kBoth);
       __syncwarp();
     }
     // both CTAs: every MMA into this CTA's TMEM and shared memory is done

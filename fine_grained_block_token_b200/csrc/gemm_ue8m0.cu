@@ -16,7 +16,7 @@
 // M-fastest.  12 warps:
 //   warp 0      TMA producer: A 128x128 and W 256x128 e4m3 tiles (128-byte
 //               swizzle) into a 4-deep shared-memory ring.
-//   warp 1      MMA issuer (whole warp loops and waits, lane 0 issues): 4
+//   warp 1      MMA issuer (whole warp loops and waits, an elected lane issues): 4
 //               block-scaled MMAs per 128-deep stage (M=128, N=256, K=32,
 //               scale-factor id = 32-K slice) into TMEM columns 0..255,
 //               reading the stage's scale factors from its own 16 TMEM
@@ -265,7 +265,7 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
           break;
         }
         ptx::tc_fence_after();
-        if (lane == 0) {
+        if (ptx::elect_one()) {
           const uint32_t a_addr = smem_base + SMEM_A_OFF + s * A_BYTES;
           const uint32_t b_addr = smem_base + SMEM_B_OFF + s * B_BYTES;
           const uint32_t sf = tmem_base + SF_COL0 + 16u * static_cast<uint32_t>(s);
@@ -283,7 +283,7 @@ gemm_ue8m0_kernel(const __grid_constant__ CUtensorMap tmap_a,
         issued = true;
       }
     }
-    if (issued && lane == 0) {
+    if (issued && ptx::elect_one()) {
       // All MMAs finish before the TMEM they write is released.
       ptx::mma_commit(drain_bar);
       if (!ptx::mbar_wait(drain_bar, 0)) record_error(args.err, kErrTimeoutMma);

@@ -230,7 +230,7 @@ gemm_ue8m0_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_
             break;
           }
           ptx::tc_fence_after();
-          if (lane == 0) {
+          if (ptx::elect_one()) {
             const uint32_t a_addr = smem_base + SMEM_A_OFF + s * PA_BYTES;
             const uint32_t b_addr = smem_base + SMEM_B_OFF + s * PB_BYTES;
             const uint32_t sfa_addr = smem_base + SMEM_SFA_OFF + s * SFA_BYTES;
@@ -251,7 +251,7 @@ gemm_ue8m0_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_
           issued = true;
         }
       }
-      if (issued && lane == 0) ptx::mma_commit_pair_multicast(drain_bar, kBoth);
+      if (issued && ptx::elect_one()) ptx::mma_commit_pair_multicast(drain_bar, kBoth);
       __syncwarp();
     }
     // both CTAs: every MMA into this CTA's TMEM and shared memory is done
