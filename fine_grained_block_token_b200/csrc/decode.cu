@@ -103,6 +103,7 @@ struct DLayout {
 constexpr int kMiscTmem = 0;       // TMEM base address
 constexpr int kMiscLast = 1;       // "this CTA reduces the block" flag
 constexpr int kMiscReady = 2;      // first block's counter usable: 0 not yet, 1 yes, 2 gave up
+constexpr int kMiscPending = 3;    // the first block, published by warp 2, is left to reduce
 
 struct DecodeArgs {
   const float* s_a;                 // [M, KB]
@@ -135,14 +136,137 @@ __device__ __forceinline__ int64_t range_start(int g, int64_t units, int G) {
 __device__ __forceinline__ void record_error(int* err, int code) { atomicCAS(err, 0, code); }
 
 
+// Partial of contributor gi for block blk: segment 0 of CTA gi, except for
+// the block's first contributor g_lo, whose range may start in an earlier
+// block (segment seg_lo).
+template <int MPAD>
+__device__ __forceinline__ const float* partial_of(const DecodeArgs& args, int gi, int g_lo,
+                                                   int seg_lo) {
+  return args.partial +
+         (static_cast<int64_t>(gi) * args.maxseg + (gi == g_lo ? seg_lo : 0)) * (MPAD * 128);
+}
+
+// Contributors of block blk: the CTAs whose ranges hold its chunks.
+__device__ __forceinline__ void block_contributors(const DecodeArgs& args, int blk, int& g_lo,
+                                                   int& g_hi) {
+  const int64_t blk_u0 = static_cast<int64_t>(blk) * args.KB;
+  g_lo = static_cast<int>(div_nonneg((blk_u0 + 1) * args.G - 1, args.units));
+  g_hi = static_cast<int>(div_nonneg((blk_u0 + args.KB) * args.G - 1, args.units));
+}
+
 struct PromoCtx {
   uint32_t smem_base, tmem_base;
   const float* prods;       // shared ring [CSLOTS][MAX_MPAD]
   volatile int* misc;       // shared misc words
   int64_t u_begin, u_end;
   int g, quarter, lane;
+  bool async_first;         // warp 2 publishes the first segment (see below)
 };
 
+
+template <int MPAD>
+__device__ __forceinline__ void reduce_block_promo(const DecodeArgs& args, int blk, int g_lo, int g_hi);
+
+// End of the range inside a shared block: publish this CTA's partial and
+// count it in; the last contributor reduces the block with the 256
+// promotion threads.
+template <int MPAD>
+__device__ __forceinline__ void publish_at_range_end(const DecodeArgs& args, const PromoCtx& cx,
+                                                     int blk) {
+  const int KB = args.KB;
+  // Publish the partial and count this CTA in; the last one reduces.
+  // The barrier orders every thread's stores before one thread's
+  // acquire-release atomic (a release covers what the barrier ordered
+  // before it); the last CTA's acquire makes the other partials
+  // visible, and the second barrier orders its threads' reads after it.
+  ptx::named_barrier_sync(1, PROMO_THREADS);
+  int g_lo, g_hi;
+  block_contributors(args, blk, g_lo, g_hi);
+  if (threadIdx.x == 128) {
+    // the block's counter must have been set up for this launch (by
+    // this CTA's warp 2, or by the CTA holding the block's first chunk)
+    const uint64_t t0 = clock64();
+    while (cx.misc[kMiscReady] == 0 && clock64() - t0 < (1ull << 32)) __nanosleep(32);
+    bool last = false;
+    if (cx.misc[kMiscReady] == 1) {
+      last = ptx::atomic_add_acq_rel_gpu(args.counters + blk, 1u) ==
+             static_cast<unsigned>(g_hi - g_lo);
+      if (last) {
+        // every contributor has counted in: the flag is free again
+        // (the launch's end orders this store before the next launch)
+        *reinterpret_cast<volatile unsigned long long*>(args.flags + blk) = 0ull;
+      }
+    } else {
+      record_error(args.err, kErrTimeoutEpilogue);
+    }
+    cx.misc[kMiscLast] = last ? 1 : 0;
+  }
+  ptx::named_barrier_sync(1, PROMO_THREADS);
+  if (cx.misc[kMiscLast]) reduce_block_promo<MPAD>(args, blk, g_lo, g_hi);
+}
+
+// Sum block blk's partials in increasing CTA order with the 256 promotion
+// threads: thread t sums row t % 128, token columns (t / 128) * MPAD / 2 ..
+// + MPAD / 2 - 1; the loads of UR partials (all of them for the usual
+// contributor counts) are in flight together.
+template <int MPAD>
+__device__ __forceinline__ void reduce_block_promo(const DecodeArgs& args, int blk, int g_lo, int g_hi) {
+  const int KB = args.KB;
+  constexpr int HALF = MPAD / 2;
+  constexpr int UR = HALF <= 8 ? 8 : (HALF <= 16 ? 4 : 2);
+  const int t = threadIdx.x - 128;
+  const int rn = t & 127;
+  const int64_t yo = static_cast<int64_t>(blk) * 128 + rn;
+  const int seg_lo =
+      blk - static_cast<int>(div_nonneg(range_start(g_lo, args.units, args.G), KB));
+  auto part = [&](int gi) { return partial_of<MPAD>(args, gi, g_lo, seg_lo); };
+  if (args.M <= 2) {
+    // one or two tokens: thread t sums row t % 128 of token t / 128,
+    // with up to 16 partials' loads in flight (same order, same sums)
+    constexpr int URS = 16;
+    const int m = t >> 7;
+    if (m < args.M) {
+      float acc1 = 0.0f;
+      for (int gg = g_lo; gg <= g_hi; gg += URS) {
+        float tv[URS];
+#pragma unroll
+        for (int r = 0; r < URS; ++r) {
+          const int gi = gg + r <= g_hi ? gg + r : g_hi;
+          tv[r] = __ldcg(part(gi) + m * 128 + rn);
+        }
+#pragma unroll
+        for (int r = 0; r < URS; ++r)
+          if (gg + r <= g_hi) acc1 += tv[r];
+      }
+      args.y[static_cast<int64_t>(m) * args.N + yo] = __float2bfloat16_rn(acc1);
+    }
+  } else {
+    const int m0 = (t >> 7) * HALF;
+    float sum[HALF];
+#pragma unroll
+    for (int m = 0; m < HALF; ++m) sum[m] = 0.0f;
+    for (int gg = g_lo; gg <= g_hi; gg += UR) {
+      float tv[UR][HALF];
+#pragma unroll
+      for (int r = 0; r < UR; ++r) {
+        const int gi = gg + r <= g_hi ? gg + r : g_hi;
+        const float* src = part(gi) + m0 * 128 + rn;
+#pragma unroll
+        for (int m = 0; m < HALF; ++m) tv[r][m] = m0 + m < args.M ? __ldcg(src + m * 128) : 0.0f;
+      }
+#pragma unroll
+      for (int r = 0; r < UR; ++r)
+        if (gg + r <= g_hi) {
+#pragma unroll
+          for (int m = 0; m < HALF; ++m) sum[m] += tv[r][m];
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < HALF; ++m)
+      if (m0 + m < args.M)
+        args.y[static_cast<int64_t>(m0 + m) * args.N + yo] = __float2bfloat16_rn(sum[m]);
+  }
+}
 
 // Promotion by one warp: token columns COL0 .. COL0 + NC - 1 of its lane
 // quarter's 32 weight rows (NC = 0: the warp only takes part in the
@@ -233,103 +357,28 @@ __device__ __forceinline__ void decode_promote(const DecodeArgs& args, const Pro
 #pragma unroll
         for (int m = 0; m < NC; ++m)
           if (COL0 + m < args.M) dst[(COL0 + m) * 128 + n_local] = acc[m];
-        // Publish the partial and count this CTA in; the last one reduces.
-        // The barrier orders every thread's stores before one thread's
-        // acquire-release atomic (a release covers what the barrier ordered
-        // before it); the last CTA's acquire makes the other partials
-        // visible, and the second barrier orders its threads' reads after it.
-        ptx::named_barrier_sync(1, PROMO_THREADS);
-        const int g_lo = static_cast<int>(div_nonneg((blk_u0 + 1) * args.G - 1, args.units));
-        const int g_hi = static_cast<int>(div_nonneg((blk_u0 + KB) * args.G - 1, args.units));
-        if (threadIdx.x == 128) {
-          // the block's counter must have been set up for this launch (by
-          // this CTA's warp 2, or by the CTA holding the block's first chunk)
-          const uint64_t t0 = clock64();
-          while (cx.misc[kMiscReady] == 0 && clock64() - t0 < (1ull << 32)) __nanosleep(32);
-          bool last = false;
-          if (cx.misc[kMiscReady] == 1) {
-            last = ptx::atomic_add_acq_rel_gpu(args.counters + blk, 1u) ==
-                   static_cast<unsigned>(g_hi - g_lo);
-            if (last) {
-              // every contributor has counted in: the flag is free again
-              // (the launch's end orders this store before the next launch)
-              *reinterpret_cast<volatile unsigned long long*>(args.flags + blk) = 0ull;
-            }
-          } else {
-            record_error(args.err, kErrTimeoutEpilogue);
-          }
-          cx.misc[kMiscLast] = last ? 1 : 0;
-        }
-        ptx::named_barrier_sync(1, PROMO_THREADS);
-        if (cx.misc[kMiscLast]) {
-          // Sum the block's partials in increasing CTA order.  All 256
-          // promotion threads take part: thread t sums row t % 128, token
-          // columns (t / 128) * MPAD / 2 .. + MPAD / 2 - 1; the loads of UR
-          // partials (all of them for the usual contributor counts) are in
-          // flight together.
-          constexpr int HALF = MPAD / 2;
-          constexpr int UR = HALF <= 8 ? 8 : (HALF <= 16 ? 4 : 2);
-          const int t = threadIdx.x - 128;
-          const int rn = t & 127;
-          const int64_t yo = static_cast<int64_t>(blk) * 128 + rn;
-          // Partial of contributor gi for this block: segment 0 of CTA gi,
-          // except for g_lo, whose range may start in an earlier block.
-          const int seg_lo =
-              blk - static_cast<int>(div_nonneg(range_start(g_lo, args.units, args.G), KB));
-          auto part = [&](int gi) {
-            return args.partial +
-                   (static_cast<int64_t>(gi) * args.maxseg + (gi == g_lo ? seg_lo : 0)) * (MPAD * 128);
-          };
-          if (args.M <= 2) {
-            // one or two tokens: thread t sums row t % 128 of token t / 128,
-            // with up to 16 partials' loads in flight (same order, same sums)
-            constexpr int URS = 16;
-            const int m = t >> 7;
-            if (m < args.M) {
-              float acc1 = 0.0f;
-              for (int gg = g_lo; gg <= g_hi; gg += URS) {
-                float tv[URS];
-#pragma unroll
-                for (int r = 0; r < URS; ++r) {
-                  const int gi = gg + r <= g_hi ? gg + r : g_hi;
-                  tv[r] = __ldcg(part(gi) + m * 128 + rn);
-                }
-#pragma unroll
-                for (int r = 0; r < URS; ++r)
-                  if (gg + r <= g_hi) acc1 += tv[r];
-              }
-              args.y[static_cast<int64_t>(m) * args.N + yo] = __float2bfloat16_rn(acc1);
-            }
-          } else {
-          const int m0 = (t >> 7) * HALF;
-          float sum[HALF];
-#pragma unroll
-          for (int m = 0; m < HALF; ++m) sum[m] = 0.0f;
-          for (int gg = g_lo; gg <= g_hi; gg += UR) {
-            float tv[UR][HALF];
-#pragma unroll
-            for (int r = 0; r < UR; ++r) {
-              const int gi = gg + r <= g_hi ? gg + r : g_hi;
-              const float* src = part(gi) + m0 * 128 + rn;
-#pragma unroll
-              for (int m = 0; m < HALF; ++m) tv[r][m] = m0 + m < args.M ? __ldcg(src + m * 128) : 0.0f;
-            }
-#pragma unroll
-            for (int r = 0; r < UR; ++r)
-              if (gg + r <= g_hi) {
-#pragma unroll
-                for (int m = 0; m < HALF; ++m) sum[m] += tv[r][m];
-              }
-          }
-#pragma unroll
-          for (int m = 0; m < HALF; ++m)
-            if (m0 + m < args.M)
-              args.y[static_cast<int64_t>(m0 + m) * args.N + yo] = __float2bfloat16_rn(sum[m]);
-          }
+        if (u + 1 < cx.u_end) {
+          // The range goes on into the next block (this is its first
+          // segment, the tail of a block): warp 2 publishes the partial and
+          // reduces the block if it arrives last, while the promotion warps
+          // go on with the next chunks.
+          ptx::named_barrier_arrive(2, PROMO_THREADS + 32);
+        } else {
+          publish_at_range_end<MPAD>(args, cx, blk);
         }
       }
 #pragma unroll
       for (int m = 0; m < NA; ++m) acc[m] = 0.0f;
+    }
+  }
+  if (cx.async_first) {
+    // Warp 2 published the first segment; if that made this CTA the block's
+    // last contributor, the block is reduced here, by all 256 threads.
+    ptx::named_barrier_sync(3, PROMO_THREADS + 32);
+    if (cx.misc[kMiscPending]) {
+      int g_lo, g_hi;
+      block_contributors(args, first_blk, g_lo, g_hi);
+      reduce_block_promo<MPAD>(args, first_blk, g_lo, g_hi);
     }
   }
 }
@@ -381,6 +430,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     ptx::prefetch_tmap(&tmap_x);
     vmisc[kMiscLast] = 0;
     vmisc[kMiscReady] = 0;
+    vmisc[kMiscPending] = 0;
     // Warm the L2 with this CTA's first weight tiles while the previous
     // kernel may still run (a prefetch only; the loads below come after the
     // wait, and a later write by the previous kernel would update L2).
@@ -503,6 +553,30 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
       vmisc[kMiscReady] = ready;
     }
     __syncwarp();
+    const int b0 = static_cast<int>(u_begin / KB);
+    if (u_begin % KB != 0 && static_cast<int64_t>(b0 + 1) * KB < u_end) {
+      // The range starts inside block b0 and goes on past it: once the
+      // promotion warps have stored b0's partial (named barrier 2), count
+      // this CTA in and, if it is the last contributor, reduce b0 here.
+      ptx::named_barrier_sync(2, PROMO_THREADS + 32);
+      int g_lo, g_hi;
+      block_contributors(args, b0, g_lo, g_hi);
+      if (lane == 0) {
+        int last = 0;
+        if (vmisc[kMiscReady] == 1) {
+          last = ptx::atomic_add_acq_rel_gpu(args.counters + b0, 1u) ==
+                 static_cast<unsigned>(g_hi - g_lo);
+          if (last) *reinterpret_cast<volatile unsigned long long*>(args.flags + b0) = 0ull;
+        } else {
+          record_error(args.err, kErrTimeoutEpilogue);
+        }
+        vmisc[kMiscPending] = last;
+      }
+      // The promotion warps reduce the block at the end of their range
+      // (named barrier 3 orders this acquire and the flag before them).
+      __syncwarp();
+      ptx::named_barrier_arrive(3, PROMO_THREADS + 32);
+    }
   } else if (warp == 3) {
     // ------------------------------------------------------ scale products
     // prods[slot][m] = s_w[blk, kb] * s_a[m, kb] for every chunk of the
@@ -560,6 +634,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     cx.g = g;
     cx.quarter = warp & 3;
     cx.lane = lane;
+    cx.async_first = u_begin % KB != 0 && (u_begin / KB + 1) * KB < u_end;
     if (warp < 8)
       decode_promote<MPAD, NC0, 0>(args, cx);
     else
