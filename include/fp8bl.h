@@ -38,10 +38,9 @@
  *   - The device must be compute capability 10.0 (B200 / sm_100a).
  *   - No exceptions cross this interface; all calls are thread-safe as long
  *     as concurrent calls do not share output buffers or workspaces.
- *   - One device per process: the GEMM kernels' opt-in to more than 48 KB
- *     of shared memory is made once per process, on the device current at
- *     their first launch, so a GEMM call on any other device returns
- *     FP8BL_ERR_CUDA (the quantizers run on any device).
+ *   - Several devices per process are supported: each kernel's opt-in to
+ *     more than 48 KB of shared memory is made once per device (device
+ *     ordinals 0 .. 63), at its first launch on that device.
  */
 #ifndef FP8BL_H
 #define FP8BL_H
