@@ -22,7 +22,7 @@ __all__ = [
     "block_linear_fused", "block_linear_noalloc", "workspace_bytes", "fused_workspace_bytes",
     "check", "version", "quant_act_ue8m0", "quant_weight_ue8m0", "block_linear_ue8m0",
     "ue8m0_workspace_bytes", "quant_rowwise", "linear_rowwise", "quant_act_static",
-    "grouped_linear_ue8m0",
+    "grouped_linear_ue8m0", "grouped_ue8m0_workspace_bytes",
 ]
 
 

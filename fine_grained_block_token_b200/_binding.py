@@ -25,6 +25,7 @@ __all__ = [
     "check", "version", "quant_act_ue8m0", "quant_weight_ue8m0", "block_linear_ue8m0",
     "ue8m0_workspace_bytes",
     "quant_rowwise", "linear_rowwise", "quant_act_static", "grouped_linear_ue8m0",
+    "grouped_ue8m0_workspace_bytes",
 ]
 
 BLOCK = 128
@@ -55,6 +56,10 @@ _lib.fp8_block_linear_ue8m0_workspace_bytes.restype = _sz
 _lib.fp8_quant_rowwise.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.fp8_quant_act_static.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp, _vp]
 _lib.fp8_grouped_linear_ue8m0.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]
+_lib.fp8_grouped_linear_ue8m0_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                             _vp, _sz, _vp]
+_lib.fp8_grouped_linear_ue8m0_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64]
+_lib.fp8_grouped_linear_ue8m0_workspace_bytes.restype = _sz
 _lib.fp8_linear_rowwise.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
 _lib.fp8bl_check.argtypes = [_vp]
 _lib.fp8bl_status_string.argtypes = [ctypes.c_int]
@@ -64,7 +69,8 @@ for _f in ("fp8_quant_act", "fp8_quant_weight", "fp8_block_linear", "fp8_block_l
            "fp8_block_linear_noalloc", "fp8bl_check", "fp8_quant_act_ue8m0",
            "fp8_quant_weight_ue8m0", "fp8_block_linear_ue8m0", "fp8_block_linear_ue8m0_ws",
            "fp8_quant_rowwise",
-           "fp8_linear_rowwise", "fp8_quant_act_static", "fp8_grouped_linear_ue8m0"):
+           "fp8_linear_rowwise", "fp8_quant_act_static", "fp8_grouped_linear_ue8m0",
+           "fp8_grouped_linear_ue8m0_ws"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 STATUS = {0: "FP8BL_OK", 1: "FP8BL_ERR_NULL", 2: "FP8BL_ERR_SHAPE", 3: "FP8BL_ERR_ALIGN",
@@ -282,10 +288,14 @@ def ue8m0_workspace_bytes(M: int, N: int, K: int) -> int:
     return int(_lib.fp8_block_linear_ue8m0_workspace_bytes(M, N, K))
 
 
-def grouped_linear_ue8m0(q_a, s_a, q_w, s_w, expert_offsets, y=None) -> torch.Tensor:
+def grouped_linear_ue8m0(q_a, s_a, q_w, s_w, expert_offsets, y=None, workspace=None,
+                         pairs=True) -> torch.Tensor:
     """Grouped (MoE expert) UE8M0 linear: rows [off[e], off[e+1]) of
     (e4m3 [M,K], e8m0 [M,K/128]) times expert e of (e4m3 [E,N,K],
-    e8m0 [E,N/128,K/128]); expert_offsets int32 [E+1] on the device."""
+    e8m0 [E,N/128,K/128]); expert_offsets int32 [E+1] on the device.  With
+    pairs=True (the default) the call goes through fp8_grouped_linear_ue8m0_ws,
+    which runs M > 128 on CTA pairs with a workspace (allocated here unless
+    given); pairs=False calls the single-CTA fp8_grouped_linear_ue8m0."""
     dev = _device_of(q_a, "q_a")
     M, K = _dims2(q_a, "q_a")
     if q_w.dim() != 3:
@@ -299,10 +309,21 @@ def grouped_linear_ue8m0(q_a, s_a, q_w, s_w, expert_offsets, y=None) -> torch.Te
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
     _need(y, "y", _BF16, (M, N), dev)
-    _ok(_lib.fp8_grouped_linear_ue8m0(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w),
-                                      _ptr(expert_offsets), _ptr(y), M, N, K, E, _stream(q_a)),
-        "fp8_grouped_linear_ue8m0")
+    if not pairs:
+        _ok(_lib.fp8_grouped_linear_ue8m0(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w),
+                                          _ptr(expert_offsets), _ptr(y), M, N, K, E, _stream(q_a)),
+            "fp8_grouped_linear_ue8m0")
+        return y
+    ws, wsb = _workspace(grouped_ue8m0_workspace_bytes(M, N, K, E), q_a.device, workspace)
+    _ok(_lib.fp8_grouped_linear_ue8m0_ws(_ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w),
+                                         _ptr(expert_offsets), _ptr(y), M, N, K, E, _ptr(ws), wsb,
+                                         _stream(q_a)), "fp8_grouped_linear_ue8m0_ws")
     return y
+
+
+def grouped_ue8m0_workspace_bytes(M: int, N: int, K: int, E: int) -> int:
+    """Workspace bytes fp8_grouped_linear_ue8m0_ws needs for these sizes."""
+    return int(_lib.fp8_grouped_linear_ue8m0_workspace_bytes(M, N, K, E))
 
 
 # Row-wise variant ("BFL (fp8r / nvfp4)" page): one fp32 scale per row of

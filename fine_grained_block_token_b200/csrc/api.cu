@@ -273,7 +273,7 @@ fp8bl_status fp8_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const v
 
 size_t fp8_block_linear_ue8m0_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (!linear_dims_ok(M, N, K)) return 0;
-  return ue8m0_pair_workspace_bytes(M, N, K);
+  return ue8m0_pair_workspace_bytes(M, N, K, 1);
 }
 
 fp8bl_status fp8_block_linear_ue8m0_ws(const void* q_a, const uint8_t* s_a, const void* q_w,
@@ -291,7 +291,7 @@ fp8bl_status fp8_block_linear_ue8m0_ws(const void* q_a, const uint8_t* s_a, cons
   if (overlap(y_bf16, ny, q_a, na) || overlap(y_bf16, ny, q_w, nw) || overlap(y_bf16, ny, s_a, nsa) ||
       overlap(y_bf16, ny, s_w, nsw))
     return FP8BL_ERR_OVERLAP;
-  const size_t need = ue8m0_pair_workspace_bytes(M, N, K);
+  const size_t need = ue8m0_pair_workspace_bytes(M, N, K, 1);
   if (need > 0) {
     if (!workspace) return FP8BL_ERR_NULL;
     if (workspace_bytes < need) return FP8BL_ERR_WORKSPACE;
@@ -306,17 +306,22 @@ fp8bl_status fp8_block_linear_ue8m0_ws(const void* q_a, const uint8_t* s_a, cons
   if (need == 0)
     return from_cuda(
         launch_block_linear_ue8m0(q_a, s_a, q_w, s_w, y_bf16, M, N, K, *d, as_cuda(stream)));
-  return from_cuda(launch_block_linear_ue8m0_pairs(q_a, s_a, q_w, s_w, y_bf16, M, N, K, workspace,
-                                                   *d, as_cuda(stream)));
+  return from_cuda(launch_linear_ue8m0_pairs(q_a, s_a, q_w, s_w, nullptr, y_bf16, M, N, K, 1,
+                                             workspace, *d, as_cuda(stream)));
 }
 
-fp8bl_status fp8_grouped_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
-                                      const uint8_t* s_w, const int32_t* expert_offsets,
-                                      void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t E,
-                                      fp8bl_stream_t stream) {
+namespace {
+// Checks shared by the grouped calls; sets *done when there is no work.
+fp8bl_status check_grouped(const void* q_a, const uint8_t* s_a, const void* q_w,
+                           const uint8_t* s_w, const int32_t* expert_offsets, void* y_bf16,
+                           int64_t M, int64_t N, int64_t K, int64_t E, bool* done) {
+  *done = false;
   if (!linear_dims_ok(M, N, K) || E < 1 || E > kMaxExperts || N * E > FP8BL_MAX_DIM)
     return FP8BL_ERR_SHAPE;
-  if (M == 0) return FP8BL_OK;
+  if (M == 0) {
+    *done = true;
+    return FP8BL_OK;
+  }
   if (!q_a || !s_a || !q_w || !s_w || !expert_offsets || !y_bf16) return FP8BL_ERR_NULL;
   if (!aligned(q_a, 16) || !aligned(q_w, 16) || !aligned(y_bf16, 16) || !aligned(expert_offsets, 4))
     return FP8BL_ERR_ALIGN;
@@ -327,11 +332,58 @@ fp8bl_status fp8_grouped_linear_ue8m0(const void* q_a, const uint8_t* s_a, const
       overlap(y_bf16, ny, s_w, static_cast<size_t>(E * (N / 128) * (K / 128))) ||
       overlap(y_bf16, ny, expert_offsets, static_cast<size_t>(E + 1) * 4))
     return FP8BL_ERR_OVERLAP;
+  return FP8BL_OK;
+}
+}  // namespace
+
+fp8bl_status fp8_grouped_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                      const uint8_t* s_w, const int32_t* expert_offsets,
+                                      void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t E,
+                                      fp8bl_stream_t stream) {
+  bool done = false;
+  fp8bl_status st = check_grouped(q_a, s_a, q_w, s_w, expert_offsets, y_bf16, M, N, K, E, &done);
+  if (st != FP8BL_OK || done) return st;
   const DeviceInfo* d = nullptr;
-  fp8bl_status st = current_device(&d);
+  st = current_device(&d);
   if (st != FP8BL_OK) return st;
   return from_cuda(launch_grouped_linear_ue8m0(q_a, s_a, q_w, s_w, expert_offsets, y_bf16, M, N,
                                                K, E, *d, as_cuda(stream)));
+}
+
+size_t fp8_grouped_linear_ue8m0_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t E) {
+  if (!linear_dims_ok(M, N, K) || E < 1 || E > kMaxExperts || N * E > FP8BL_MAX_DIM) return 0;
+  return ue8m0_pair_workspace_bytes(M, N, K, E);
+}
+
+fp8bl_status fp8_grouped_linear_ue8m0_ws(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                         const uint8_t* s_w, const int32_t* expert_offsets,
+                                         void* y_bf16, int64_t M, int64_t N, int64_t K, int64_t E,
+                                         void* workspace, size_t workspace_bytes,
+                                         fp8bl_stream_t stream) {
+  bool done = false;
+  fp8bl_status st = check_grouped(q_a, s_a, q_w, s_w, expert_offsets, y_bf16, M, N, K, E, &done);
+  if (st != FP8BL_OK || done) return st;
+  if (!aligned(workspace, 16)) return FP8BL_ERR_ALIGN;
+  const size_t need = ue8m0_pair_workspace_bytes(M, N, K, E);
+  if (need > 0) {
+    if (!workspace) return FP8BL_ERR_NULL;
+    if (workspace_bytes < need) return FP8BL_ERR_WORKSPACE;
+    if (overlap(workspace, need, y_bf16, static_cast<size_t>(M * N) * 2) ||
+        overlap(workspace, need, q_a, static_cast<size_t>(M * K)) ||
+        overlap(workspace, need, q_w, static_cast<size_t>(E * N * K)) ||
+        overlap(workspace, need, s_a, static_cast<size_t>(M * (K / 128))) ||
+        overlap(workspace, need, s_w, static_cast<size_t>(E * (N / 128) * (K / 128))) ||
+        overlap(workspace, need, expert_offsets, static_cast<size_t>(E + 1) * 4))
+      return FP8BL_ERR_OVERLAP;
+  }
+  const DeviceInfo* d = nullptr;
+  st = current_device(&d);
+  if (st != FP8BL_OK) return st;
+  if (need == 0)
+    return from_cuda(launch_grouped_linear_ue8m0(q_a, s_a, q_w, s_w, expert_offsets, y_bf16, M, N,
+                                                 K, E, *d, as_cuda(stream)));
+  return from_cuda(launch_linear_ue8m0_pairs(q_a, s_a, q_w, s_w, expert_offsets, y_bf16, M, N, K,
+                                             E, workspace, *d, as_cuda(stream)));
 }
 
 fp8bl_status fp8_quant_rowwise(const void* x_bf16, int64_t R, int64_t K, void* q_e4m3, float* s,

@@ -77,14 +77,16 @@ cudaError_t launch_block_linear_ue8m0(const void* q_a, const uint8_t* s_a, const
                                       const uint8_t* s_w, void* y, int64_t M, int64_t N,
                                       int64_t K, const DeviceInfo& dev, cudaStream_t st);
 
-// UE8M0 block-scaled GEMM on CTA pairs (M > 128): the workspace holds the
-// scale factors rewritten in the tensor core's order.
+// UE8M0 block-scaled GEMM on CTA pairs (M > 128), plain (offsets = null,
+// E = 1) or grouped: the workspace holds the scale factors rewritten in the
+// tensor core's order.
+constexpr int kMaxExperts = 1024;
 bool ue8m0_use_pairs(int64_t M);
-size_t ue8m0_pair_workspace_bytes(int64_t M, int64_t N, int64_t K);
-cudaError_t launch_block_linear_ue8m0_pairs(const void* q_a, const uint8_t* s_a, const void* q_w,
-                                            const uint8_t* s_w, void* y, int64_t M, int64_t N,
-                                            int64_t K, void* workspace, const DeviceInfo& dev,
-                                            cudaStream_t st);
+size_t ue8m0_pair_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t E);
+cudaError_t launch_linear_ue8m0_pairs(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                      const uint8_t* s_w, const int* offsets, void* y, int64_t M,
+                                      int64_t N, int64_t K, int64_t E, void* workspace,
+                                      const DeviceInfo& dev, cudaStream_t st);
 
 // Row-wise e4m3 quantization ("BFL (fp8r / nvfp4)"): bf16 [R, K] -> e4m3
 // [R, K] + one fp32 scale per row; K % 16 == 0.
@@ -99,7 +101,6 @@ cudaError_t launch_linear_rowwise(const void* q_a, const float* s_a, const void*
 
 // Grouped (MoE expert) UE8M0 linear: row segments [off[e], off[e+1]) of
 // q_a times expert e's weights, q_w [E, N, K], s_w [E, N/128, K/128].
-constexpr int kMaxExperts = 1024;
 cudaError_t launch_grouped_linear_ue8m0(const void* q_a, const uint8_t* s_a, const void* q_w,
                                         const uint8_t* s_w, const int32_t* offsets, void* y,
                                         int64_t M, int64_t N, int64_t K, int64_t E,

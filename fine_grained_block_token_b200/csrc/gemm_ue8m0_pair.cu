@@ -24,8 +24,16 @@
 //   weights: sfw[(kb * NBp + nb) * 32 + r] = the code of block (nb, kb)
 //     replicated into all 16 bytes;
 //   rows / blocks past the matrix hold 127, the code of 1.0.
+// Grouped (MoE expert) form, same kernel: rows of A split into E contiguous
+// segments [off[e], off[e+1]), segment e times expert e's W[e] ([E, N, K],
+// scales [E, N/128, K/128]).  Each CTA's warp 3 turns the offsets into a
+// shared-memory table at start-up (clamped to [0, M], made non-decreasing)
+// with each expert's count of 256-row blocks; tiles run expert by expert.
+// The activation factors are packed per expert, each segment padded to 256
+// rows (so a tile's 128-row halves start on a packed group), and the weight
+// factors per expert.  The plain linear is E = 1, off = {0, M}.
 // Warps: 0 producer (both CTAs), 1 MMA issuer (even CTA), 2 TMEM owner,
-// 4-11 epilogue (both CTAs): after a tile's last MMA each warp reads its 32
+// 3 expert table, 4-11 epilogue (both CTAs): after a tile's last MMA each warp reads its 32
 // TMEM lanes x 128 columns, releases the accumulator (the odd CTA's warps
 // arrive on the even CTA's barrier, once per tile) and stores bf16 through a
 // shared staging box, 32 columns at a time, in 64-byte row segments.
@@ -61,7 +69,8 @@ constexpr int SMEM_Y_OFF = SMEM_SFB_OFF + PSTAGES * SFB_BYTES;
 constexpr int SMEM_BAR_OFF = SMEM_Y_OFF + NUM_EPI_WARPS * STAGE_WARP_BYTES;
 constexpr int NUM_BARS = 2 * PSTAGES + 3;     // full, empty, tfull, tempty, drain
 constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NUM_BARS * 8;
-constexpr int SMEM_BYTES = SMEM_MISC_OFF + 16 + 1024;
+constexpr int SMEM_TAB_OFF = SMEM_MISC_OFF + 16;   // expert table: offsets, 256-row block prefix
+constexpr int SMEM_BYTES = SMEM_TAB_OFF + 2 * (kMaxExperts + 1) * 4 + 1024;
 constexpr uint32_t STAGE_TX = 2u * (PA_BYTES + PB_BYTES + SFA_BYTES + SFB_BYTES);
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(SFB_COL + 8 <= TMEM_COLS && SFA_COL + 4 <= SFB_COL && ACC_COL + PBN <= SFA_COL, "TMEM");
@@ -91,40 +100,114 @@ __device__ __forceinline__ void mma_block_scale_pair(uint32_t d_tmem, uint64_t a
       : "memory");
 }
 
-__global__ void pack_sfa_kernel(const uint8_t* __restrict__ s, int R, int KB, int RBp,
-                                uint4* __restrict__ out) {
+// Expert table, built by one warp: tab_off[0..E] = the segment starts
+// clamped to [0, M] and made non-decreasing (running maximum), tab_pre[e] =
+// the 256-row blocks of the experts before e.  offsets == nullptr means one
+// segment {0, M}.
+__device__ void build_expert_table(const int* offsets, int E, int M, int lane, int* tab_off,
+                                   int* tab_pre) {
+  int carry = 0;
+  for (int base = 0; base <= E; base += 32) {
+    const int i = base + lane;
+    int o = 0;
+    if (i <= E) {
+      o = offsets != nullptr ? __ldg(offsets + i) : (i == 0 ? 0 : M);
+      o = min(max(o, 0), M);
+    }
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, o, d);
+      if (lane >= d) o = max(o, t);
+    }
+    o = max(o, carry);
+    if (i <= E) tab_off[i] = o;
+    carry = __shfl_sync(0xffffffffu, o, 31);
+  }
+  __syncwarp();
+  carry = 0;
+  for (int base = 0; base < E; base += 32) {
+    const int e = base + lane;
+    int b = e < E ? (tab_off[e + 1] - tab_off[e] + PBM - 1) / PBM : 0;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, b, d);
+      if (lane >= d) b += t;
+    }
+    b += carry;
+    if (e < E) tab_pre[e + 1] = b;
+    carry = __shfl_sync(0xffffffffu, b, 31);
+  }
+  if (lane == 0) tab_pre[0] = 0;
+  __syncwarp();
+}
+
+// The last expert whose first 256-row block is at or before block `blk`
+// (an expert with no rows never matches, since the next one starts at the
+// same block).
+__device__ __forceinline__ int expert_of_block(const int* tab_pre, int E, int blk) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tab_pre[mid] <= blk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Activation factors in MMA order, per expert, every segment padded to a
+// multiple of 256 rows: packed 128-row group t holds padded rows 128 t ..;
+// padded row p of expert e is row off[e] + (p - 256 tab_pre[e]) of A, or
+// padding (127) past the segment.  Grid: KB * MBp * 32 threads.
+__global__ void pack_sfa_kernel(const uint8_t* __restrict__ s, int M, int KB, int MBp,
+                                const int* offsets, int E, uint4* __restrict__ out) {
+  __shared__ int tab_off[kMaxExperts + 1], tab_pre[kMaxExperts + 1];
+  if (threadIdx.x < 32) build_expert_table(offsets, E, M, threadIdx.x, tab_off, tab_pre);
+  __syncthreads();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(KB) * RBp * 32;
+  const int64_t total = static_cast<int64_t>(KB) * MBp * 32;
   if (i >= total) return;
   const int r = static_cast<int>(i & 31);
   const int64_t t = i >> 5;
-  const int rb = static_cast<int>(t % RBp);
-  const int kb = static_cast<int>(t / RBp);
+  const int rb = static_cast<int>(t % MBp);
+  const int kb = static_cast<int>(t / MBp);
+  const int padded_rows = tab_pre[E] * PBM;
   uint32_t w[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const int row = rb * 128 + 32 * j + r;
-    w[j] = rep4(row < R ? s[static_cast<int64_t>(row) * KB + kb] : 127u);
+    const int p = rb * 128 + 32 * j + r;
+    uint32_t code = 127u;
+    if (p < padded_rows) {
+      const int e = expert_of_block(tab_pre, E, p / PBM);
+      const int local = p - tab_pre[e] * PBM;
+      if (local < tab_off[e + 1] - tab_off[e])
+        code = s[static_cast<int64_t>(tab_off[e] + local) * KB + kb];
+    }
+    w[j] = rep4(code);
   }
   out[i] = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__global__ void pack_sfw_kernel(const uint8_t* __restrict__ s, int NB, int KB, int NBp,
+// Weight factors in MMA order, per expert: row ((e * KB + kb) * NBp + nb) *
+// 32 + r holds block (nb, kb) of expert e replicated into 16 bytes.
+__global__ void pack_sfw_kernel(const uint8_t* __restrict__ s, int NB, int KB, int NBp, int E,
                                 uint4* __restrict__ out) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(KB) * NBp * 32;
+  const int64_t total = static_cast<int64_t>(E) * KB * NBp * 32;
   if (i >= total) return;
   const int64_t t = i >> 5;
   const int nb = static_cast<int>(t % NBp);
-  const int kb = static_cast<int>(t / NBp);
-  const uint32_t w = rep4(nb < NB ? s[static_cast<int64_t>(nb) * KB + kb] : 127u);
+  const int64_t ekb = t / NBp;
+  const int kb = static_cast<int>(ekb % KB);
+  const int e = static_cast<int>(ekb / KB);
+  const uint32_t w =
+      rep4(nb < NB ? s[(static_cast<int64_t>(e) * NB + nb) * KB + kb] : 127u);
   out[i] = make_uint4(w, w, w, w);
 }
 
 struct PairArgs {
   __nv_bfloat16* y;
-  int M, N, K;
-  int MBp, NBp;   // padded 128-row tile counts of the packed factor arrays
+  const int* offsets;   // [E + 1] segment starts (device), or null for one segment {0, M}
+  int M, N, K, E;
+  int MBp, NBp;   // padded 128-row group counts of the packed factor arrays (per expert for W)
   int* err;
 };
 
@@ -149,13 +232,14 @@ gemm_ue8m0_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_
   const uint32_t rank = ptx::cluster_ctarank();      // 0 = the pair's MMA issuer
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
-  const int M = args.M, N = args.N, K = args.K;
-  const int num_m = (M + PBM - 1) / PBM;
+  const int M = args.M, N = args.N, K = args.K, E = args.E;
   const int num_n = (N + PBN - 1) / PBN;
   const int num_kb = K / BK;
-  const int num_tiles = num_m * num_n;
   const int nblk_count = N / 128;
   constexpr uint16_t kBoth = 0x3;
+  int* tab_off = reinterpret_cast<int*>(smem + SMEM_TAB_OFF);   // [E + 1]
+  int* tab_pre = tab_off + (kMaxExperts + 1);                    // [E + 1]
+  if (warp == 3) build_expert_table(args.offsets, E, M, lane, tab_off, tab_pre);
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < PSTAGES; ++s) {
@@ -180,7 +264,24 @@ gemm_ue8m0_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_
   ptx::cluster_sync();   // both CTAs' barriers initialised before any cross-CTA use
   ptx::tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+  const int num_tiles = tab_pre[E] * num_n;
   const bool has_tiles = pair < num_tiles;
+  // tile -> (expert, its global 256-row block, first row, end of its rows,
+  // N tile); expert-major, M-fastest within an expert.
+  auto map_tile = [&](int tile, int& e, int& gblk, int& row0, int& row_end, int& n_blk) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (tab_pre[mid] * num_n <= tile) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+    const int local = tile - tab_pre[e] * num_n;
+    const int blocks = tab_pre[e + 1] - tab_pre[e];
+    n_blk = local / blocks;
+    gblk = tab_pre[e] + local % blocks;
+    row0 = tab_off[e] + (local % blocks) * PBM;
+    row_end = tab_off[e + 1];
+  };
 
   if (warp == 0) {
     // ------------------------------------------------- producer (both CTAs)
@@ -188,8 +289,9 @@ gemm_ue8m0_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_
       uint32_t c = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int m_blk = tile % num_m, n_blk = tile / num_m;
-        const int mt = m_blk * 2 + static_cast<int>(rank);     // this CTA's 128-row tile
+        int e, gblk, row0, row_end, n_blk;
+        map_tile(tile, e, gblk, row0, row_end, n_blk);
+        const int mt = gblk * 2 + static_cast<int>(rank);      // this CTA's packed 128-row group
         for (int kb = 0; kb < num_kb; ++kb, ++c) {
           const int s = c % PSTAGES;
           const uint32_t ph = (c / PSTAGES) & 1u;
@@ -200,13 +302,14 @@ gemm_ue8m0_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_
           }
           const uint32_t fb = ptx::map_to_cta(full_bar(s), 0);
           if (leader) ptx::mbar_arrive_expect_tx(full_bar(s), STAGE_TX);
-          ptx::tma_load_2d_pair(smem_base + SMEM_A_OFF + s * PA_BYTES, &tmap_a, fb, kb * BK, mt * 128);
+          ptx::tma_load_2d_pair(smem_base + SMEM_A_OFF + s * PA_BYTES, &tmap_a, fb, kb * BK,
+                                row0 + 128 * static_cast<int>(rank));
           ptx::tma_load_2d_pair(smem_base + SMEM_B_OFF + s * PB_BYTES, &tmap_b, fb, kb * BK,
-                                n_blk * PBN + 128 * static_cast<int>(rank));
+                                e * N + n_blk * PBN + 128 * static_cast<int>(rank));
           ptx::tma_load_2d_pair(smem_base + SMEM_SFA_OFF + s * SFA_BYTES, &tmap_sfa, fb, 0,
                                 (kb * args.MBp + mt) * 32);
           ptx::tma_load_2d_pair(smem_base + SMEM_SFB_OFF + s * SFB_BYTES, &tmap_sfb, fb, 0,
-                                (kb * args.NBp + n_blk * 2) * 32);
+                                ((e * num_kb + kb) * args.NBp + n_blk * 2) * 32);
         }
       }
     }
@@ -268,8 +371,9 @@ gemm_ue8m0_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_
     const uint8_t* stage_g = smem + SMEM_Y_OFF + (warp - 4) * STAGE_WARP_BYTES;
     uint32_t t_local = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++t_local) {
-      const int m_blk = tile % num_m, n_blk = tile / num_m;
-      const int wrow0 = m_blk * PBM + 128 * static_cast<int>(rank) + quarter * 32;
+      int e, gblk, row0, row_end, n_blk;
+      map_tile(tile, e, gblk, row0, row_end, n_blk);
+      const int wrow0 = row0 + 128 * static_cast<int>(rank) + quarter * 32;
       const int nb = n_blk * 2 + half;
       if (!__all_sync(0xffffffffu, ptx::mbar_wait_spin_cluster(tfull_bar, t_local & 1u))) {
         if (lane == 0) record_error(args.err, kErrTimeoutEpilogue);
@@ -315,7 +419,7 @@ gemm_ue8m0_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_
             const int r = 8 * it + (lane >> 2);
             const int q = lane & 3;
             const uint4 val = *reinterpret_cast<const uint4*>(stage_g + r * STAGE_COLS * 2 + 16 * q);
-            if (wrow0 + r < M)
+            if (wrow0 + r < row_end)
               *reinterpret_cast<uint4*>(args.y + static_cast<int64_t>(wrow0 + r) * N + nb * 128 +
                                         pass * STAGE_COLS + 8 * q) = val;
           }
@@ -334,7 +438,9 @@ gemm_ue8m0_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_
   }
 }
 
-int64_t mbp_of(int64_t M) { return 2 * ((M + PBM - 1) / PBM); }
+// Packed activation groups: 2 per 256-row block of every expert's segment;
+// sum_e ceil(len_e / 256) <= ceil(M / 256) + E bounds the grouped case.
+int64_t mbp_of(int64_t M, int64_t E) { return 2 * ((M + PBM - 1) / PBM + (E > 1 ? E : 0)); }
 int64_t nbp_of(int64_t N) { return 2 * ((N + PBN - 1) / PBN); }
 
 cudaError_t ensure_ue8m0_pair_ready(int* max_clusters) {
@@ -373,45 +479,51 @@ cudaError_t ensure_ue8m0_pair_ready(int* max_clusters) {
 // would only compute padding); smaller M run on the single-CTA kernel.
 bool ue8m0_use_pairs(int64_t M) { return M > 128; }
 
-size_t ue8m0_pair_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+size_t ue8m0_pair_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t E) {
   if (!ue8m0_use_pairs(M)) return 0;
   const int64_t KB = K / 128;
-  return static_cast<size_t>(KB * mbp_of(M) * 512 + KB * nbp_of(N) * 512);
+  return static_cast<size_t>(KB * mbp_of(M, E) * 512 + E * KB * nbp_of(N) * 512);
 }
 
-cudaError_t launch_block_linear_ue8m0_pairs(const void* q_a, const uint8_t* s_a, const void* q_w,
-                                            const uint8_t* s_w, void* y, int64_t M, int64_t N,
-                                            int64_t K, void* workspace, const DeviceInfo& dev,
-                                            cudaStream_t st) {
+cudaError_t launch_linear_ue8m0_pairs(const void* q_a, const uint8_t* s_a, const void* q_w,
+                                      const uint8_t* s_w, const int* offsets, void* y, int64_t M,
+                                      int64_t N, int64_t K, int64_t E, void* workspace,
+                                      const DeviceInfo& dev, cudaStream_t st) {
+  if (E < 1 || E > kMaxExperts) return cudaErrorInvalidValue;
   int max_clusters = 0;
   cudaError_t e = ensure_ue8m0_pair_ready(&max_clusters);
   if (e != cudaSuccess) return e;
   const int KB = static_cast<int>(K / 128);
-  const int MBp = static_cast<int>(mbp_of(M)), NBp = static_cast<int>(nbp_of(N));
+  const int MBp = static_cast<int>(mbp_of(M, E)), NBp = static_cast<int>(nbp_of(N));
   uint8_t* psa = static_cast<uint8_t*>(workspace);
   uint8_t* psw = psa + static_cast<int64_t>(KB) * MBp * 512;
-  const int64_t ta = static_cast<int64_t>(KB) * MBp * 32, tw = static_cast<int64_t>(KB) * NBp * 32;
+  const int64_t ta = static_cast<int64_t>(KB) * MBp * 32, tw = E * KB * NBp * 32;
   if ((ta + 255) / 256 > 0x7FFFFFFFll || (tw + 255) / 256 > 0x7FFFFFFFll) return cudaErrorInvalidValue;
   pack_sfa_kernel<<<static_cast<unsigned>((ta + 255) / 256), 256, 0, st>>>(
-      s_a, static_cast<int>(M), KB, MBp, reinterpret_cast<uint4*>(psa));
+      s_a, static_cast<int>(M), KB, MBp, offsets, static_cast<int>(E), reinterpret_cast<uint4*>(psa));
   pack_sfw_kernel<<<static_cast<unsigned>((tw + 255) / 256), 256, 0, st>>>(
-      s_w, static_cast<int>(N / 128), KB, NBp, reinterpret_cast<uint4*>(psw));
+      s_w, static_cast<int>(N / 128), KB, NBp, static_cast<int>(E), reinterpret_cast<uint4*>(psw));
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap ta_m, tb_m, tsa, tsb;
-  if (!make_tmap_u8(&ta_m, q_a, M, K, 128, BK) || !make_tmap_u8(&tb_m, q_w, N, K, 128, BK) ||
+  if (!make_tmap_u8(&ta_m, q_a, M, K, 128, BK) || !make_tmap_u8(&tb_m, q_w, E * N, K, 128, BK) ||
       !make_tmap_u8(&tsa, psa, static_cast<uint64_t>(ta), 16, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_tmap_u8(&tsb, psw, static_cast<uint64_t>(tw), 16, 64, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   PairArgs a;
   a.y = static_cast<__nv_bfloat16*>(y);
+  a.offsets = offsets;
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
+  a.E = static_cast<int>(E);
   a.MBp = MBp;
   a.NBp = NBp;
   a.err = dev.error_flag;
-  const int64_t tiles = ((M + PBM - 1) / PBM) * ((N + PBN - 1) / PBN);
+  // tiles: at most (ceil(M / 256) + E - 1) 256-row blocks over the experts
+  const int64_t mblocks = (M + PBM - 1) / PBM + (E > 1 ? E - 1 : 0);
+  const int64_t tiles = mblocks * ((N + PBN - 1) / PBN);
+  if (tiles == 0) return cudaSuccess;
   const int pairs = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);

@@ -290,6 +290,31 @@ fp8bl_status fp8_grouped_linear_ue8m0(const void *q_a, const uint8_t *s_a,
                                       fp8bl_stream_t stream);
 
 /*
+ * fp8_grouped_linear_ue8m0_ws -- the same grouped linear with a caller
+ * workspace, which lets M > 128 run on CTA pairs (256-row tiles within each
+ * expert's segment, as fp8_block_linear_ue8m0_ws): two small kernels first
+ * rewrite s_a (every segment padded to a multiple of 256 rows) and s_w (per
+ * expert) into the workspace in the order the tensor core reads scale
+ * factors.  Same passage, arguments and result as fp8_grouped_linear_ue8m0
+ * (bit for bit), plus
+ *   workspace: device scratch of at least
+ *              fp8_grouped_linear_ue8m0_workspace_bytes(M, N, K, E) bytes
+ *              (16-byte aligned), or NULL when that size is 0 (M <= 128:
+ *              the single-CTA kernel).  Contents on entry are ignored; it
+ *              must not overlap any argument.  The size bounds the padded
+ *              segments for any offsets: K/128 * 2 * (ceil(M/256) + E) * 512
+ *              bytes for s_a (E > 1) and E * K/128 * 2 * ceil(N/256) * 512
+ *              for s_w.
+ */
+size_t fp8_grouped_linear_ue8m0_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t E);
+fp8bl_status fp8_grouped_linear_ue8m0_ws(const void *q_a, const uint8_t *s_a,
+                                         const void *q_w, const uint8_t *s_w,
+                                         const int32_t *expert_offsets, void *y_bf16,
+                                         int64_t M, int64_t N, int64_t K, int64_t E,
+                                         void *workspace, size_t workspace_bytes,
+                                         fp8bl_stream_t stream);
+
+/*
  * Row-wise FP8 variant (fp8r).
  * Passage: "BFL (fp8r / nvfp4)" page of the diffusers docs, first bullet of
  * its list (an E4M3 weight with one fp32 weight scale per row; activations

@@ -43,10 +43,10 @@ def _quantized(fp8, M, N, K, E, seed):
     return q_a, s_a, q_w.view(E, N, K), s_w.view(E, N // 128, K // 128)
 
 
-def _check(fp8, q_a, s_a, q_w, s_w, off, rows=None, label=""):
+def _check(fp8, q_a, s_a, q_w, s_w, off, rows=None, label="", pairs=True):
     M = q_a.shape[0]
     y = torch.full((M, q_w.shape[1]), 7.0, dtype=torch.bfloat16, device="cuda")
-    fp8.grouped_linear_ue8m0(q_a, s_a, q_w, s_w, torch.from_numpy(off).cuda(), y)
+    fp8.grouped_linear_ue8m0(q_a, s_a, q_w, s_w, torch.from_numpy(off).cuda(), y, pairs=pairs)
     fp8.check()
     R = oracle.grouped_linear_ue8m0(u8(q_a), u8(s_a), u8(q_w), u8(s_w), off, rows=rows, nthreads=8)
     covered = np.zeros(M, bool)
@@ -57,14 +57,74 @@ def _check(fp8, q_a, s_a, q_w, s_w, off, rows=None, label=""):
     check_gemm(Y[idx], R[idx], label)
 
 
+@pytest.mark.parametrize("pairs", [True, False])
 @pytest.mark.parametrize("M,N,K,E,seed", [
     (300, 256, 256, 3, 0), (1000, 384, 512, 8, 1), (77, 256, 384, 5, 2), (2048, 512, 1024, 64, 3),
     (129, 128, 128, 1, 4),
 ])
-def test_random_segments(fp8, M, N, K, E, seed):
+def test_random_segments(fp8, M, N, K, E, seed, pairs):
     g = np.random.default_rng(seed)
     q_a, s_a, q_w, s_w = _quantized(fp8, M, N, K, E, 10 * seed)
-    _check(fp8, q_a, s_a, q_w, s_w, _segments(g, M, E), label=f"{M}x{N}x{K} E={E}")
+    _check(fp8, q_a, s_a, q_w, s_w, _segments(g, M, E), label=f"{M}x{N}x{K} E={E} pairs={pairs}",
+           pairs=pairs)
+
+
+@pytest.mark.parametrize("M,N,K,E,seed", [
+    (300, 256, 256, 3, 0), (1000, 384, 512, 8, 1), (2048, 512, 1024, 64, 3), (513, 256, 768, 16, 5),
+    (4100, 1280, 640, 7, 6),
+])
+def test_pairs_equal_single_cta(fp8, M, N, K, E, seed):
+    """The CTA-pair schedule (fp8_grouped_linear_ue8m0_ws, 256-row tiles in
+    each expert's segment, scale factors packed per expert) runs the same
+    block-scaled MMAs in the same K order as the single-CTA kernel: every
+    output equal bit for bit, rows outside the segments untouched by both.
+    Random codes with scale codes spread over 2^+-20, so that a factor taken
+    from the wrong expert, row or K block shows."""
+    g = np.random.default_rng(100 + seed)
+    qa = g.integers(0, 256, (M, K), dtype=np.uint8)
+    qw = g.integers(0, 256, (E * N, K), dtype=np.uint8)
+    qa[(qa & 0x7F) == 0x7F] = 0x00
+    qw[(qw & 0x7F) == 0x7F] = 0x00
+    ca = g.integers(107, 148, (M, K // 128), dtype=np.uint8)
+    cw = g.integers(107, 148, (E * N // 128, K // 128), dtype=np.uint8)
+    dev = lambda a: torch.from_numpy(a).cuda()
+    q_a, s_a = dev(qa).view(torch.float8_e4m3fn), dev(ca).view(torch.float8_e8m0fnu)
+    q_w = dev(qw).view(torch.float8_e4m3fn).view(E, N, K)
+    s_w = dev(cw).view(torch.float8_e8m0fnu).view(E, N // 128, K // 128)
+    off = _segments(g, M, E)
+    off[0], off[-1] = min(int(off[1]), 5), max(int(off[-2]), M - 3)     # a few rows left out
+    offd = torch.from_numpy(off).cuda()
+    assert fp8.grouped_ue8m0_workspace_bytes(M, N, K, E) > 0
+    ys = [torch.full((M, N), 3.0, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    fp8.grouped_linear_ue8m0(q_a, s_a, q_w, s_w, offd, ys[0])
+    fp8.grouped_linear_ue8m0(q_a, s_a, q_w, s_w, offd, ys[1], pairs=False)
+    fp8.check()
+    assert torch.equal(ys[0].view(torch.int16), ys[1].view(torch.int16)), (M, N, K, E)
+    rows = np.unique(np.concatenate([off[:-1], np.maximum(off[1:] - 1, 0), g.choice(M, 6, replace=False)]))
+    rows = rows[rows < M]
+    R = oracle.grouped_linear_ue8m0(qa, ca, qw.reshape(E, N, K), cw.reshape(E, N // 128, K // 128),
+                                    off, rows=rows, nthreads=8)
+    covered = np.zeros(M, bool)
+    covered[off[0]:off[-1]] = True
+    Y = f32(ys[0])
+    assert np.all(Y[~covered] == 3.0)
+    idx = np.intersect1d(rows, np.nonzero(covered)[0])
+    check_gemm(Y[idx], R[idx], f"grouped pairs {M}x{N}x{K} E={E}")
+
+
+def test_pairs_workspace_checks(fp8):
+    """The workspace call refuses a short or missing workspace before any
+    launch, and needs none at M <= 128."""
+    M, N, K, E = 300, 256, 256, 3
+    need = fp8.grouped_ue8m0_workspace_bytes(M, N, K, E)
+    assert need > 0 and fp8.grouped_ue8m0_workspace_bytes(128, N, K, E) == 0
+    q_a, s_a, q_w, s_w = _quantized(fp8, M, N, K, E, 3)
+    off = torch.tensor([0, 100, 200, 300], dtype=torch.int32, device="cuda")
+    with pytest.raises(fp8.Fp8blError) as ei:
+        fp8.grouped_linear_ue8m0(q_a, s_a, q_w, s_w, off,
+                                 workspace=torch.zeros(need - 16, dtype=torch.uint8, device="cuda"))
+    assert ei.value.status == 7
+    fp8.check()
 
 
 def test_segments_not_covering_all_rows(fp8):
