@@ -17,8 +17,9 @@ inputs copied from pinned host memory and the outputs copied back inside
 every step.  `roofline` covers the dominant kernel (the block-scaled GEMM;
 for the decode workload the weight-streaming decode kernel, against HBM)
 against the measured peaks in MEASURED_PEAKS.json, from a second pass with
-events around every kernel.  `fused` times fp8_block_linear_fused (the
-activation quantization inside the GEMM) on the same inputs and checks its
+events around every kernel.  `fused` times fp8_block_linear_fused on the
+same inputs with its workspace (codes staged in it) and, as `in_kernel`,
+without one (the quantization inside the GEMM's tiles), and checks each
 output equals the two-call path bit for bit.  `ue8m0` and `fp8r` time the
 two other scale formats on the same inputs (power-of-two scales on the
 tensor core's block-scaled MMA; one fp32 scale per activation row and weight
@@ -745,11 +746,9 @@ def leg_gemm_workload(fp8, dev, barrier, args, lins):
             if ev is not None:
                 ev[2 * i + 1].record()
 
-    g = capture_graph(step, dev)
-    ms = timed_replays(g.replay, args.steps, barrier)
-    del g
     n = len(items)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(args.steps)]
+    step()
     barrier()
     for k in range(args.steps):
         step(evs[k])
@@ -757,18 +756,38 @@ def leg_gemm_workload(fp8, dev, barrier, args, lins):
     gemm_ms = sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs for i in range(n))
     y_ref = [it["y"].clone() for it in items]
 
-    def fused():
-        for it in items:
-            fp8.block_linear_fused(it["x"], it["q_w"], it["s_w"], it["y"])
+    # The two-call step and the fused entry point (with its workspace, and
+    # in-GEMM without) are timed in alternating rounds, so that the clock
+    # drift of a long power-capped run does not favour whichever runs first.
+    def fused_fn(in_kernel):
+        def fused():
+            for it in items:
+                fp8.block_linear_fused(it["x"], it["q_w"], it["s_w"], it["y"], in_kernel=in_kernel)
+        return fused
 
-    g = capture_graph(fused, dev)
-    g.replay()
-    torch.cuda.synchronize(dev)
-    same = all(torch.equal(r.view(torch.int16), it["y"].view(torch.int16)) for r, it in zip(y_ref, items))
-    fused_ms = timed_replays(g.replay, args.steps, barrier)
-    del g
+    out = {}
+    graphs = {"two_call": capture_graph(step, dev)}
+    for key, in_kernel in (("fused", False), ("fused_ik", True)):
+        for it in items:
+            it["y"].zero_()
+        graphs[key] = capture_graph(fused_fn(in_kernel), dev)
+        graphs[key].replay()
+        torch.cuda.synchronize(dev)
+        out[key + "_same"] = all(torch.equal(r.view(torch.int16), it["y"].view(torch.int16))
+                                 for r, it in zip(y_ref, items))
+    rounds = max(1, min(4, args.steps))
+    per = [max(1, args.steps // rounds)] * rounds
+    per[-1] += args.steps - sum(per)
+    tot = {k: 0.0 for k in graphs}
+    for r in range(rounds):
+        for k, g in graphs.items():
+            tot[k] += timed_replays(g.replay, per[r], barrier)
+    ms = tot["two_call"]
+    out["fused_ms"], out["fused_ik_ms"] = tot["fused"], tot["fused_ik"]
+    del graphs
     flops = sum(2 * it["M"] * it["N"] * it["K"] for it in items)
-    return items, dict(ms=ms, gemm_ms=gemm_ms, fused_ms=fused_ms, flops=flops, identical=same)
+    return items, dict(ms=ms, gemm_ms=gemm_ms, fused_ms=out["fused_ms"], fused_ik_ms=out["fused_ik_ms"],
+                       flops=flops, identical=out["fused_same"], identical_ik=out["fused_ik_same"])
 
 
 def rows_oracle_check(items, rows_per_linear, seed=0):
@@ -834,22 +853,29 @@ def leg_sweep(fp8, dev, barrier, args):
                 fp8.block_linear(q, s, qw, sw, y)
 
         yf = [torch.empty_like(y) for y in ys]
+        yk = [torch.empty_like(y) for y in ys]
 
         def fused():
             for x, (qw, sw), y in zip(xs, ws, yf):
                 fp8.block_linear_fused(x, qw, sw, y)
 
+        def fused_ik():
+            for x, (qw, sw), y in zip(xs, ws, yk):
+                fp8.block_linear_fused(x, qw, sw, y, in_kernel=True)
+
         r = {}
-        for key, fn in (("quant", quant), ("gemm", gemm), ("fused", fused)):
+        for key, fn in (("quant", quant), ("gemm", gemm), ("fused", fused), ("fused_ik", fused_ik)):
             g = capture_graph(fn, dev)
             r[key] = timed_replays(g.replay, reps, barrier) / (reps * R)
             del g
         torch.cuda.synchronize(dev)
-        same = all(torch.equal(a.view(torch.int16), b.view(torch.int16)) for a, b in zip(ys, yf))
-        res[f"M{M}"] = dict(quant_ms=r["quant"], gemm_ms=r["gemm"], fused_ms=r["fused"], identical=same,
+        same = all(torch.equal(a.view(torch.int16), b.view(torch.int16)) for a, b in zip(ys, yf)) and \
+            all(torch.equal(a.view(torch.int16), b.view(torch.int16)) for a, b in zip(ys, yk))
+        res[f"M{M}"] = dict(quant_ms=r["quant"], gemm_ms=r["gemm"], fused_ms=r["fused"],
+                            fused_ik_ms=r["fused_ik"], identical=same,
                             qbytes=qbytes, flops=2.0 * M * N * K, copies=R)
         items.append(dict(label=f"M{M}", xb=xb, q_w=q_w0, s_w=s_w0, y=ys[0], M=M, N=N, K=K))
-        del xs, qs, ws, yf
+        del xs, qs, ws, yf, yk
     return res, items
 
 
@@ -955,7 +981,10 @@ def deepseek_json(leg, world, args, cpu_ok, fp8_peak):
                  "frac": tf / fp8_peak, "ms_per_launch": ds["gemm_ms"] / (args.steps * len(items)),
                  "traffic": recorded_traffic("gemm_prefill_kernel", "deepseek_mlp")},
         "fused": {"value": whole_job_rate(world, ds["flops"], args.steps, ds["fused_ms"]) / 1e12,
-                  "vs_two_call": ds["ms"] / ds["fused_ms"], "identical_to_two_call": ds["identical"]},
+                  "vs_two_call": ds["ms"] / ds["fused_ms"], "identical_to_two_call": ds["identical"],
+                  "in_kernel": {"value": whole_job_rate(world, ds["flops"], args.steps, ds["fused_ik_ms"]) / 1e12,
+                                "vs_two_call": ds["ms"] / ds["fused_ik_ms"],
+                                "identical_to_two_call": ds["identical_ik"]}},
         "cpu_baseline": dcpu, "parity": dpar}
     return out
 
@@ -971,6 +1000,7 @@ def sweep_json(leg, cpu_ok, hbm_peak, fp8_peak):
         per[k] = {"act_quant_GBps": q_gbs, "act_quant_frac": q_gbs / hbm_peak,
                   "gemm_TFLOPs": g_tf, "gemm_frac": g_tf / fp8_peak,
                   "fused_TFLOPs": f_tf, "fused_vs_two_call": (d["quant_ms"] + d["gemm_ms"]) / d["fused_ms"],
+                  "fused_in_kernel_vs_two_call": (d["quant_ms"] + d["gemm_ms"]) / d["fused_ik_ms"],
                   "identical_to_two_call": d["identical"], "copies": d["copies"]}
     scpu, spar = rows_oracle_check(sitems, 4, seed=1) if cpu_ok else (None, None)
     out["sweep"] = {
@@ -1146,36 +1176,49 @@ def run_ours(args):
     b.record()
     barrier()
     e2e_ms = a.elapsed_time(b)
-    # ---- the fused entry point (activation quantization inside the GEMM)
-    # on the same inputs and steps; its output must equal the two-call one
+    # ---- the fused entry point (bf16 activations in one call) on the same
+    # inputs and steps, with its workspace (staged codes) and without it
+    # (quantization inside the GEMM's tiles, prefill sizes only); its output
+    # must equal the two-call one
     y_ref = [it["y"].clone() for it in items]
     fws = []
     for it in items:
         nb = fp8.fused_workspace_bytes(it["M"], it["N"], it["K"])
         fws.append(torch.empty(max(nb, 16), dtype=torch.uint8, device=dev))
 
-    def fused_step():
-        for it, w in zip(items, fws):
-            fp8.block_linear_fused(it["x"], it["q_w"], it["s_w"], it["y"], w)
+    def time_fused(in_kernel):
+        def fused_step():
+            for it, w in zip(items, fws):
+                if in_kernel:
+                    fp8.block_linear_fused(it["x"], it["q_w"], it["s_w"], it["y"], in_kernel=True)
+                else:
+                    fp8.block_linear_fused(it["x"], it["q_w"], it["s_w"], it["y"], w)
 
-    for _ in range(min(args.warmup, 3)):
-        fused_step()
-    torch.cuda.synchronize()
-    fused_graph = None if args.eager else capture(fused_step)
-    run_fused = (lambda: fused_graph.replay()) if fused_graph is not None else fused_step
-    run_fused()
-    torch.cuda.synchronize()
-    fused_identical = all(torch.equal(r.view(torch.int16), it["y"].view(torch.int16))
-                          for r, it in zip(y_ref, items))
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    barrier()
-    a.record()
-    for _ in range(args.steps):
+        for _ in range(min(args.warmup, 3)):
+            fused_step()
+        torch.cuda.synchronize()
+        fgraph = None if args.eager else capture(fused_step)
+        run_fused = (lambda: fgraph.replay()) if fgraph is not None else fused_step
+        for it in items:
+            it["y"].zero_()
         run_fused()
-    b.record()
-    barrier()
-    fused_ms = a.elapsed_time(b)
+        torch.cuda.synchronize()
+        identical = all(torch.equal(r.view(torch.int16), it["y"].view(torch.int16))
+                        for r, it in zip(y_ref, items))
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        barrier()
+        a.record()
+        for _ in range(args.steps):
+            run_fused()
+        b.record()
+        barrier()
+        ms = a.elapsed_time(b)
+        del fgraph
+        return ms, identical
+
+    fused_ms, fused_identical = time_fused(False)
+    fused_ik_ms, fused_ik_identical = (None, None) if decode_workload(args.workload) else time_fused(True)
 
     # ---- the scale-format variants on the same inputs, each one step =
     # its activation quantization + its GEMM per linear, timed like the
@@ -1262,7 +1305,7 @@ def run_ours(args):
 
     # max over ranks (every device time below is the slowest rank's)
     vnames = sorted(variants)
-    times = [elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms] + \
+    times = [elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms, fused_ik_ms or 0.0] + \
         [variants[v][k] for v in vnames for k in ("ms", "gemm_ms")]
     leg_slots = []
     if "decode" in legs:
@@ -1273,17 +1316,18 @@ def run_ours(args):
             leg_slots.append((lay[k], "ms"))
     if "deepseek_mlp" in legs:
         _, ds = legs["deepseek_mlp"]
-        leg_slots += [(ds, "ms"), (ds, "gemm_ms"), (ds, "fused_ms")]
+        leg_slots += [(ds, "ms"), (ds, "gemm_ms"), (ds, "fused_ms"), (ds, "fused_ik_ms")]
     if "sweep" in legs:
         sw, _ = legs["sweep"]
         for k in sorted(sw):
-            leg_slots += [(sw[k], "quant_ms"), (sw[k], "gemm_ms"), (sw[k], "fused_ms")]
+            leg_slots += [(sw[k], "quant_ms"), (sw[k], "gemm_ms"), (sw[k], "fused_ms"), (sw[k], "fused_ik_ms")]
     if "tiny" in legs:
         leg_slots.append((legs["tiny"], "ms"))
     maxed = max_over_ranks(times + [d[k] for d, k in leg_slots], dev, world)
-    elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms = maxed[:5]
+    elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms, fused_ik_ms_max = maxed[:6]
+    fused_ik_ms = fused_ik_ms_max if fused_ik_ms is not None else None
     for i, v in enumerate(vnames):
-        variants[v]["ms"], variants[v]["gemm_ms"] = maxed[5 + 2 * i], maxed[6 + 2 * i]
+        variants[v]["ms"], variants[v]["gemm_ms"] = maxed[6 + 2 * i], maxed[7 + 2 * i]
     for (d, k), v in zip(leg_slots, maxed[len(times):]):
         d[k] = v
 
@@ -1365,8 +1409,15 @@ def run_ours(args):
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "fused": {"value": fused_value, "unit": "TFLOP/s", "ms_per_step": fused_ms / args.steps,
                       "vs_two_call": ms_per_step / (fused_ms / args.steps),
-                      "kernel": "decode_kernel after act_quant (staged)" if decode else "gemm_fused_kernel",
-                      "identical_to_two_call": fused_identical},
+                      "kernel": ("act_quant32_kernel into the workspace, then decode_kernel" if decode else
+                                 "act_quant32_kernel into the workspace, then gemm_prefill_kernel"),
+                      "identical_to_two_call": fused_identical,
+                      "in_kernel": None if fused_ik_ms is None else {
+                          "value": whole_job_rate(world, flops_step, args.steps, fused_ik_ms) / 1e12,
+                          "ms_per_step": fused_ik_ms / args.steps,
+                          "vs_two_call": ms_per_step / (fused_ik_ms / args.steps),
+                          "kernel": "gemm_fused_kernel (no workspace: quantization in the GEMM's tiles)",
+                          "identical_to_two_call": fused_ik_identical}},
             "ue8m0": variant_lines.get("ue8m0"),
             "fp8r": variant_lines.get("fp8r"),
             **(legs_json(legs, world, args, hbm_peak, fp8_peak, peak_src) if run_legs else {}),
@@ -1376,7 +1427,7 @@ def run_ours(args):
             "parity": parity,
         }
         print(json.dumps(line))
-    del graph, fused_graph   # released before the process group goes away
+    del graph   # released before the process group goes away
     variants.clear()
     torch.cuda.synchronize(dev)
     if world > 1:

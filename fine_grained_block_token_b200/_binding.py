@@ -391,9 +391,11 @@ def block_linear(q_a, s_a, q_w, s_w, y=None, workspace=None) -> torch.Tensor:
     return y
 
 
-def block_linear_fused(x, q_w, s_w, y=None, workspace=None) -> torch.Tensor:
-    """bf16 x [M,K] with quantized weights -> bf16 [M,N]; the activation
-    quantization happens inside the GEMM, bit-identical to quant_act."""
+def block_linear_fused(x, q_w, s_w, y=None, workspace=None, in_kernel=False) -> torch.Tensor:
+    """bf16 x [M,K] with quantized weights -> bf16 [M,N], bit-identical to
+    quant_act + block_linear.  By default the codes are staged in a workspace
+    (allocated here unless given); in_kernel=True (M > 64) passes no
+    workspace, so that the GEMM quantizes each activation tile itself."""
     dev = _device_of(x, "x")
     M, K = _dims2(x, "x")
     N = _dims2(q_w, "q_w")[0]
@@ -404,7 +406,12 @@ def block_linear_fused(x, q_w, s_w, y=None, workspace=None) -> torch.Tensor:
         _need(y, "y", _BF16, (M, N), dev)
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    ws, wsb = _workspace(fused_workspace_bytes(M, N, K), x.device, workspace)
+    if in_kernel:
+        if M <= 64:
+            raise ValueError("in_kernel=True needs M > 64 (decode sizes always stage)")
+        ws, wsb = None, 0
+    else:
+        ws, wsb = _workspace(fused_workspace_bytes(M, N, K), x.device, workspace)
     _ok(_lib.fp8_block_linear_fused(_ptr(x), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K,
                                     _ptr(ws), wsb, _stream(x)), "fp8_block_linear_fused")
     return y

@@ -204,12 +204,19 @@ fp8bl_status fp8_block_linear_fused(const void* x_bf16, const void* q_w, const f
   const DeviceInfo* d = nullptr;
   fp8bl_status st = current_device(&d);
   if (st != FP8BL_OK) return st;
-  const GemmPlan plan = plan_block_linear(M, N, K, d->sm_count, true);
+  GemmPlan plan = plan_block_linear(M, N, K, d->sm_count, true);
+  if (plan.in_kernel_ok && (!workspace || workspace_bytes < plan.workspace)) {
+    // prefill sizes without the staging workspace: quantize in the tiles
+    plan.kind = 2;
+    plan.workspace = 0;
+  }
   if (plan.workspace > 0) {
     if (!workspace) return FP8BL_ERR_NULL;
     if (workspace_bytes < plan.workspace) return FP8BL_ERR_WORKSPACE;
     if (overlap(workspace, plan.workspace, y_bf16, ny) ||
-        overlap(workspace, plan.workspace, x_bf16, static_cast<size_t>(M * K) * 2))
+        overlap(workspace, plan.workspace, x_bf16, static_cast<size_t>(M * K) * 2) ||
+        overlap(workspace, plan.workspace, q_w, static_cast<size_t>(N * K)) ||
+        overlap(workspace, plan.workspace, s_w, static_cast<size_t>((N / 128) * (K / 128)) * 4))
       return FP8BL_ERR_OVERLAP;
   }
   return from_cuda(launch_block_linear_fused(x_bf16, q_w, s_w, y_bf16, M, N, K, plan, workspace,

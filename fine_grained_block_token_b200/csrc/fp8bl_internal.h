@@ -114,7 +114,10 @@ struct GemmPlan {
   int kind = 0;          // 0 = prefill tile kernel, 1 = decode (swap-AB) kernel,
                          // 2 = fused prefill kernel (activation quantization in the tiles)
   int split_k = 1;       // number of K slices (decode / small grids)
-  size_t workspace = 0;  // bytes of fp32 partials needed
+  size_t workspace = 0;  // bytes of scratch the plan needs
+  // fused plans: true when the in-GEMM quantization kernel (kind 2, no
+  // workspace) may serve a call whose workspace is smaller than `workspace`
+  bool in_kernel_ok = false;
 };
 
 GemmPlan plan_block_linear(int64_t M, int64_t N, int64_t K, int sm_count, bool fused);

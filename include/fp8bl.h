@@ -157,12 +157,19 @@ fp8bl_status fp8_block_linear(const void *q_a, const float *s_a,
                               fp8bl_stream_t stream);
 
 /*
- * fp8_block_linear_fused -- the same linear with the activation
- * quantization done inside the GEMM: x_bf16 [M, K] is quantized exactly as
- * fp8_quant_act would (bit-identical codes and scales) and multiplied
- * without writing q_a / s_a to memory.  y equals
- * fp8_quant_act + fp8_block_linear bit for bit.
- *   workspace: at least fp8_block_linear_fused_workspace_bytes(M, N, K).
+ * fp8_block_linear_fused -- the same linear from bf16 activations in one
+ * call: x_bf16 [M, K] is quantized exactly as fp8_quant_act would
+ * (bit-identical codes and scales) and multiplied; y equals
+ * fp8_quant_act + fp8_block_linear bit for bit.  Two schedules:
+ *   - staged (the faster on B200 at every size measured): the codes and
+ *     scales are written into the workspace, where they stay in L2 for the
+ *     GEMM that follows; needs fp8_block_linear_fused_workspace_bytes(M, N, K)
+ *     bytes (M*K + M*K/128*4 plus the decode scratch, each rounded up to
+ *     256 bytes);
+ *   - in-GEMM (M > 64 only): the GEMM quantizes each activation tile itself
+ *     and the codes never reach memory; taken when workspace is NULL or
+ *     smaller than that size.
+ *   At M <= 64 the workspace is required.
  */
 fp8bl_status fp8_block_linear_fused(const void *x_bf16,
                                     const void *q_w, const float *s_w,

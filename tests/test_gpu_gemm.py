@@ -116,6 +116,10 @@ def test_fused_bit_identical(fp8):
         y2 = fp8.block_linear_fused(x, q_w, s_w)
         torch.cuda.synchronize()
         assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), (M, N, K)
+        if M > 64:
+            y3 = fp8.block_linear_fused(x, q_w, s_w, in_kernel=True)
+            torch.cuda.synchronize()
+            assert torch.equal(y1.view(torch.int16), y3.view(torch.int16)), (M, N, K)
 
 
 def test_no_timeout_recorded(fp8):
@@ -169,9 +173,10 @@ def test_full_size_sweep_unfused_and_fused(fp8, M):
     rows = _sample_rows(M, 16, seed=M)
     y, R, (x, q_a, s_a, q_w, s_w, y_full) = _run(fp8, xb, wb, rows=rows)
     check_gemm(y, R, f"sweep M={M}")
-    y_fused = fp8.block_linear_fused(x, q_w, s_w)
-    torch.cuda.synchronize()
-    assert torch.equal(y_full.view(torch.int16), y_fused.view(torch.int16))
+    for in_kernel in (False, True):
+        y_fused = fp8.block_linear_fused(x, q_w, s_w, in_kernel=in_kernel)
+        torch.cuda.synchronize()
+        assert torch.equal(y_full.view(torch.int16), y_fused.view(torch.int16)), in_kernel
 
 
 def test_full_size_deepseek_down(fp8):
@@ -187,9 +192,10 @@ def test_fused_prefill_size_bit_identical(fp8):
     q_w, s_w = fp8.quant_weight(w)
     q_a, s_a = fp8.quant_act(x)
     y1 = fp8.block_linear(q_a, s_a, q_w, s_w)
-    y2 = fp8.block_linear_fused(x, q_w, s_w)
-    torch.cuda.synchronize()
-    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    for in_kernel in (False, True):
+        y2 = fp8.block_linear_fused(x, q_w, s_w, in_kernel=in_kernel)
+        torch.cuda.synchronize()
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), in_kernel
 
 
 @pytest.mark.parametrize("M,N,K", [(8192, 2048, 1024), (4096, 4096, 2048), (640, 1280, 1152)])
@@ -208,7 +214,7 @@ def test_fused_repeated_runs_bit_identical(fp8, M, N, K):
     y2 = torch.empty_like(y1)
     for rep in range(10):
         y2.fill_(0)
-        fp8.block_linear_fused(x, q_w, s_w, y2)
+        fp8.block_linear_fused(x, q_w, s_w, y2, in_kernel=True)
         torch.cuda.synchronize()
         assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), (M, N, K, rep)
     fp8.check()
