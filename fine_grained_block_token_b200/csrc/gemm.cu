@@ -41,6 +41,13 @@
 // stalled the promotion ~110 cycles per chunk) and the bf16 stores to TMA
 // (the row-per-thread stores cost ~7,400 cycles per tile) took the chunk
 // from ~1,050-1,200 to ~940-1,010 cycles.
+// Tail wave: with T tiles on G CTAs, q = T / G full waves leave r = T % G
+// tiles; when 2 r <= G each of those is split into two 128 x 128 items
+// (MMA N = 128, a 128-row W box, promotion warps 64 columns each) run by
+// two CTAs, so the last wave takes about two thirds of a full tile's time
+// instead of a whole one.  Every output element is still accumulated in the
+// same K order with the same products, so results are bit for bit those of
+// the full tiles.  With T <= G / 2 every tile is split.
 // Every mbarrier wait is bounded in time; on expiry the kernel records an
 // error code in the error word, drains what it started and exits cleanly.
 #include <cstdint>
@@ -68,6 +75,7 @@ constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 384;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr uint32_t IDESC = ptx::idesc_e4m3_f32(BM, BN);
+constexpr uint32_t IDESC_HALF = ptx::idesc_e4m3_f32(BM, BN / 2);   // split tail items
 
 constexpr int STAGE_ROWS = 32;     // epilogue staging: 32 rows x 64 bytes per warp
 constexpr int STAGE_COLS = 32;     // bf16 columns per staging pass
@@ -101,6 +109,7 @@ __device__ __forceinline__ void record_error(int* err, int code) {
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
+                    const __grid_constant__ CUtensorMap tmap_b_half,
                     const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -124,6 +133,25 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
   const int num_n = (N + BN - 1) / BN;
   const int num_kb = K / BK;
   const int num_tiles = num_m * num_n;
+  // work items: full tiles, then (split tail) two 128-column halves per
+  // remaining tile
+  const int G = gridDim.x;
+  const int q_waves = num_tiles / G, r_tail = num_tiles % G;
+  const bool split = r_tail > 0 && 2 * r_tail <= G;
+  const int num_items = split ? q_waves * G + 2 * r_tail : num_tiles;
+  // item -> (M block, first column, full 256-column tile?)
+  auto map_item = [&](int item, int& m_blk, int& col0, bool& full) {
+    int tile = item, sub = 0;
+    full = true;
+    if (split && item >= q_waves * G) {
+      const int h = item - q_waves * G;
+      tile = q_waves * G + (h >> 1);
+      sub = h & 1;
+      full = false;
+    }
+    m_blk = tile % num_m;
+    col0 = (tile / num_m) * BN + sub * (BN / 2);
+  };
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -142,6 +170,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     ptx::fence_barrier_init();
     ptx::prefetch_tmap(&tmap_a);
     ptx::prefetch_tmap(&tmap_b);
+    ptx::prefetch_tmap(&tmap_b_half);
     ptx::prefetch_tmap(&tmap_y);
   }
   if (warp == 2) {
@@ -165,8 +194,10 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
       for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
       uint32_t c = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m_blk = tile % num_m, n_blk = tile / num_m;
+      for (int item = blockIdx.x; item < num_items && ok; item += gridDim.x) {
+        int m_blk, col0;
+        bool full;
+        map_item(item, m_blk, col0, full);
         for (int kb = 0; kb < num_kb; ++kb, ++c) {
           const int s = c % STAGES;
           const uint32_t ph = (c / STAGES) & 1u;
@@ -175,11 +206,11 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
+          ptx::mbar_arrive_expect_tx(full_bar(s), A_BYTES + (full ? B_BYTES : B_BYTES / 2));
           ptx::tma_load_2d(smem_base + SMEM_A_OFF + s * A_BYTES, &tmap_a, full_bar(s), kb * BK,
                            m_blk * BM);
-          ptx::tma_load_2d(smem_base + SMEM_B_OFF + s * B_BYTES, &tmap_b, full_bar(s), kb * BK,
-                           n_blk * BN);
+          ptx::tma_load_2d(smem_base + SMEM_B_OFF + s * B_BYTES, full ? &tmap_b : &tmap_b_half,
+                           full_bar(s), kb * BK, col0);
           last_phase[s] = static_cast<int>(ph);
         }
       }
@@ -195,7 +226,11 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
       const uint64_t desc_b = ptx::sdesc_kmajor_sw128(smem_base + SMEM_B_OFF);
       uint32_t c = 0;
       bool ok = true, issued = false;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int item = blockIdx.x; item < num_items && ok; item += gridDim.x) {
+        int m_blk, col0;
+        bool full;
+        map_item(item, m_blk, col0, full);
+        const uint32_t idesc = full ? IDESC : IDESC_HALF;
         for (int kb = 0; kb < num_kb; ++kb, ++c) {
           const int s = c % STAGES;
           const uint32_t sph = (c / STAGES) & 1u;
@@ -215,7 +250,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
 #pragma unroll
             for (int k = 0; k < BK / UMMA_K; ++k)
               ptx::mma_f8f6f4(d, ptx::sdesc_advance(da, k * UMMA_K), ptx::sdesc_advance(db, k * UMMA_K),
-                              IDESC, k > 0 ? 1u : 0u);
+                              idesc, k > 0 ? 1u : 0u);
             ptx::mma_commit(empty_bar(s));
             ptx::mma_commit(tfull_bar(buf));
           }
@@ -240,8 +275,10 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     constexpr int PF = 4;
     uint32_t c = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const int m_blk = tile % num_m, n_blk = tile / num_m;
+    for (int item = blockIdx.x; item < num_items && ok; item += gridDim.x) {
+      int m_blk, col0;
+      bool full;
+      map_item(item, m_blk, col0, full);
       const float* sa_r[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -251,7 +288,8 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
       const float* sw_r[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int nb = n_blk * 2 + h;
+        // a full tile's two weight blocks; a split item's one, for both halves
+        const int nb = col0 / 128 + (full ? h : 0);
         sw_r[h] = args.s_w + static_cast<int64_t>(nb < nblk_count ? nb : nblk_count - 1) * num_kb;
       }
       float pa[PF][4], pw[PF][2];
@@ -302,11 +340,16 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const uint32_t stage = smem_base + SMEM_Y_OFF + static_cast<uint32_t>(warp - 4) * STAGE_WARP_BYTES;
     uint32_t c = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const int m_blk = tile % num_m, n_blk = tile / num_m;
+    for (int item = blockIdx.x; item < num_items && ok; item += gridDim.x) {
+      int m_blk, col0;
+      bool full;
+      map_item(item, m_blk, col0, full);
       const int row0 = m_blk * BM + quarter * 32;   // this warp's first row
-      const int nb = n_blk * 2 + half;
-      const bool box_ok = nb < nblk_count && row0 < M;
+      // this warp's columns: 128 of a full tile, 64 of a split item
+      const int ncol = full ? 128 : 64;
+      const int wcol0 = col0 + half * ncol;
+      const int nj = ncol / 16;                     // 16-column TMEM loads per chunk
+      const bool box_ok = wcol0 < nblk_count * 128 && row0 < M;
       float2 acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
@@ -331,20 +374,22 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t tb = tmem_base + lane_off + static_cast<uint32_t>(buf * BN + half * 128);
+        const uint32_t tb = tmem_base + lane_off + static_cast<uint32_t>(buf * BN + half * ncol);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          uint32_t v[16];
-          ptx::tmem_ld_32x32b_x16(tb + j * 16, v);
-          ptx::tmem_ld_wait();
-          if (j == 7) {
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
-          }
+          if (j < nj) {
+            uint32_t v[16];
+            ptx::tmem_ld_32x32b_x16(tb + j * 16, v);
+            ptx::tmem_ld_wait();
+            if (j == nj - 1) {
+              ptx::tc_fence_before();
+              __syncwarp();
+              if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
+            }
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            acc[j * 8 + q] = __ffma2_rn(make_float2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1])), sc2, acc[j * 8 + q]);
+            for (int q = 0; q < 8; ++q)
+              acc[j * 8 + q] = __ffma2_rn(make_float2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1])), sc2, acc[j * 8 + q]);
+          }
         }
       }
       if (!ok) break;
@@ -354,6 +399,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
       // written).
 #pragma unroll
       for (int pass = 0; pass < 128 / STAGE_COLS; ++pass) {
+        if (pass * STAGE_COLS >= ncol) break;
         if (lane == 0) ptx::bulk_wait_group_read<0>();   // the staging box is free again
         __syncwarp();
 #pragma unroll
@@ -372,7 +418,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
         ptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && box_ok) {
-          ptx::tma_store_2d(&tmap_y, stage, (nb * 128 + pass * STAGE_COLS) * 2, row0);
+          ptx::tma_store_2d(&tmap_y, stage, (wcol0 + pass * STAGE_COLS) * 2, row0);
           ptx::bulk_commit_group();
         }
       }
@@ -472,8 +518,9 @@ cudaError_t launch_block_linear(const void* q_a, const float* s_a, const void* q
     return launch_block_linear_pairs(q_a, s_a, q_w, s_w, y, M, N, K, dev, st);
   cudaError_t e = ensure_smem_attr();
   if (e != cudaSuccess) return e;
-  CUtensorMap ta, tb, ty;
+  CUtensorMap ta, tb, tb2, ty;
   if (!make_tmap_u8(&ta, q_a, M, K, BM, BK) || !make_tmap_u8(&tb, q_w, N, K, BN, BK) ||
+      !make_tmap_u8(&tb2, q_w, N, K, BN / 2, BK) ||
       !make_tmap_u8(&ty, y, M, 2 * N, STAGE_ROWS, STAGE_COLS * 2, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   GemmArgs a;
@@ -485,7 +532,10 @@ cudaError_t launch_block_linear(const void* q_a, const float* s_a, const void* q
   a.K = static_cast<int>(K);
   a.err = dev.error_flag;
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  // one CTA per SM; with at most half as many tiles as SMs, two CTAs per
+  // tile (every tile split into two 128-column items)
+  int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  if (2 * tiles <= dev.sm_count) grid = static_cast<int>(2 * tiles);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -495,7 +545,7 @@ cudaError_t launch_block_linear(const void* q_a, const float* s_a, const void* q
   set_programmatic_serialization(at[0]);
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_prefill_kernel, ta, tb, ty, a);
+  return cudaLaunchKernelEx(&cfg, gemm_prefill_kernel, ta, tb, tb2, ty, a);
 }
 
 cudaError_t launch_block_linear_fused(const void* x, const void* q_w, const float* s_w, void* y,
