@@ -298,3 +298,21 @@ def test_decode_graph_replay_bit_identical(fp8):
             assert torch.equal(it["y"].view(torch.int16), it["ref"].view(torch.int16)), (it["M"], rep)
     del graph
     fp8.check()
+
+
+@pytest.mark.parametrize("M,N,K", [(7000, 640, 256), (4096, 4096, 512), (150, 2048, 384)])
+def test_split_tail_wave(fp8, M, N, K):
+    """Shapes whose last wave of 128x256 tiles is run as 128-column halves:
+    7000x640 has 55x3 = 165 tiles on 148 CTAs (17 split, some of them in the
+    partial last N tile), 4096x4096 has 512 (68 split), 150x2048 has 16 (all
+    split).  Sampled rows against the oracle, and the in-GEMM quantization
+    schedule (full tiles only) equal bit for bit: the split items must keep
+    every element's K order and products."""
+    xb = wl.sweep_x(M, K)
+    wb = wl.normal((N, K), 0.02, 1, M + N + K)
+    rows = _sample_rows(M, 24, seed=M + N)
+    y, R, (x, q_a, s_a, q_w, s_w, y_full) = _run(fp8, xb, wb, rows=rows)
+    check_gemm(y, R, f"split tail {M}x{N}x{K}")
+    y_fused = fp8.block_linear_fused(x, q_w, s_w, in_kernel=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y_full.view(torch.int16), y_fused.view(torch.int16))

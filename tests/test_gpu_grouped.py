@@ -112,6 +112,27 @@ def test_pairs_equal_single_cta(fp8, M, N, K, E, seed):
     check_gemm(Y[idx], R[idx], f"grouped pairs {M}x{N}x{K} E={E}")
 
 
+def test_pairs_many_experts(fp8):
+    """256 experts over 4100 rows, a third of them empty and many of a few
+    rows (so most 256-row pair tiles are mostly padding and the packed
+    activation factors need the bound of ceil(M / 256) + E groups): pairs
+    equal the single-CTA kernel bit for bit, sampled rows match the oracle."""
+    M, N, K, E = 4100, 256, 384, 256
+    g = np.random.default_rng(77)
+    q_a, s_a, q_w, s_w = _quantized(fp8, M, N, K, E, 31)
+    off = _segments(g, M, E, p_empty=0.33)
+    offd = torch.from_numpy(off).cuda()
+    ys = [torch.full((M, N), 3.0, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    fp8.grouped_linear_ue8m0(q_a, s_a, q_w, s_w, offd, ys[0])
+    fp8.grouped_linear_ue8m0(q_a, s_a, q_w, s_w, offd, ys[1], pairs=False)
+    fp8.check()
+    assert torch.equal(ys[0].view(torch.int16), ys[1].view(torch.int16))
+    rows = np.unique(np.concatenate([off[:-1], np.maximum(off[1:] - 1, 0), g.choice(M, 8, replace=False)]))
+    rows = rows[rows < M]
+    R = oracle.grouped_linear_ue8m0(u8(q_a), u8(s_a), u8(q_w), u8(s_w), off, rows=rows, nthreads=8)
+    check_gemm(f32(ys[0])[rows], R[rows], "grouped pairs 256 experts")
+
+
 def test_pairs_workspace_checks(fp8):
     """The workspace call refuses a short or missing workspace before any
     launch, and needs none at M <= 128."""
