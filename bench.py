@@ -428,6 +428,112 @@ def moe_oracle_rows(xb, q_w, s_w, off, rows):
     return t, 2.0 * len(rows) * q_w.shape[1] * q_w.shape[2], R[rows]
 
 
+def moe_items(fp8, dev):
+    """The DeepSeek-V3 expert linears (up, down): routed activations, the
+    experts' UE8M0-quantized weights, outputs and the CTA-pair workspace."""
+    import torch
+    items = []
+    for name in ("up", "down"):
+        xb, off = wl.deepseek_moe(name)
+        N, K = wl.MOE_LINEARS[name]
+        E = wl.MOE_EXPERTS
+        w = wl.deepseek_moe_weights(name, dev)
+        q_w, s_w = fp8.quant_weight_ue8m0(w)
+        del w
+        M = xb.shape[0]
+        items.append(dict(label=name, xb=xb, x=wl.to_torch_bf16(xb).to(dev), off_np=off,
+                          off=torch.from_numpy(off).to(dev), q_w=q_w.view(E, N, K),
+                          s_w=s_w.view(E, N // 128, K // 128),
+                          q_a=torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev),
+                          s_a=torch.empty((M, K // 128), dtype=torch.float8_e8m0fnu, device=dev),
+                          y=torch.empty((M, N), dtype=torch.bfloat16, device=dev), M=M, N=N, K=K))
+        # the CTA-pair schedule's packed scale factors (allocated once, reused)
+        items[-1]["ws"] = torch.empty(max(fp8.grouped_ue8m0_workspace_bytes(M, N, K, E), 16),
+                                      dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize(dev)
+    return items
+
+
+def moe_step_fn(fp8, items):
+    """One MoE step: per expert linear, the ue8m0 activation quantization of
+    the routed rows and the grouped GEMM (events around each GEMM if given)."""
+    def step(ev=None):
+        for i, it in enumerate(items):
+            fp8.quant_act_ue8m0(it["x"], it["q_a"], it["s_a"])
+            if ev is not None:
+                ev[2 * i].record()
+            fp8.grouped_linear_ue8m0(it["q_a"], it["s_a"], it["q_w"], it["s_w"], it["off"], it["y"],
+                                     workspace=it["ws"])
+            if ev is not None:
+                ev[2 * i + 1].record()
+    return step
+
+
+def moe_oracle_check(items, rows_per_linear, seed=0):
+    """The oracle on sampled routed rows of each expert linear (CPU baseline
+    and parity check)."""
+    import torch
+    t_tot, f_tot, worst = 0.0, 0.0, 0.0
+    g = np.random.default_rng(seed)
+    for it in items:
+        rows = np.sort(g.choice(it["M"], rows_per_linear, replace=False))
+        qw = it["q_w"].view(torch.uint8).cpu().numpy()
+        sw = it["s_w"].view(torch.uint8).cpu().numpy()
+        t, f, R = moe_oracle_rows(it["xb"], qw, sw, it["off_np"], rows)
+        t_tot += t
+        f_tot += f
+        Y = it["y"][torch.as_tensor(rows, device=it["y"].device)].float().cpu().numpy()
+        worst = max(worst, within_tolerance(Y, R))
+    cpu = {"value": f_tot / t_tot / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count() or 1,
+           "kind": "oracle", "seconds": t_tot,
+           "sample": f"{rows_per_linear} random routed rows per expert linear (up, down): "
+                     "ue8m0 activation quant + fp64 grouped GEMM of those rows, all N columns"}
+    parity = {"rows_per_linear": rows_per_linear, "within_tolerance": worst <= 1.0,
+              "worst_bound_ratio": worst}
+    return cpu, parity
+
+
+def leg_moe(fp8, dev, barrier, args):
+    """The grouped MoE step as a leg of the default run: graph-replayed
+    steps, then a pass with events around the grouped GEMMs."""
+    import torch
+    items = moe_items(fp8, dev)
+    step = moe_step_fn(fp8, items)
+    for _ in range(min(args.warmup, 3)):
+        step()
+    g = capture_graph(step, dev)
+    ms = timed_replays(g.replay, args.steps, barrier)
+    del g
+    n = len(items)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(args.steps)]
+    barrier()
+    for k in range(args.steps):
+        step(evs[k])
+    barrier()
+    gemm_ms = sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs for i in range(n))
+    fp8.check()
+    flops = sum(2 * it["M"] * it["N"] * it["K"] for it in items)
+    return items, dict(ms=ms, gemm_ms=gemm_ms, flops=flops)
+
+
+def moe_json(leg, world, args, cpu_ok, fp8_peak, peak_src):
+    items, d = leg
+    n = len(items)
+    gemm_tf = d["flops"] * args.steps / (d["gemm_ms"] * 1e-3) / 1e12
+    cpu, parity = moe_oracle_check(items, 4) if cpu_ok else (None, None)
+    return {"deepseek_moe": {
+        "value": whole_job_rate(world, d["flops"], args.steps, d["ms"]) / 1e12, "unit": "TFLOP/s",
+        "ms_per_step": d["ms"] / args.steps,
+        "config": {"workload": "deepseek_moe", "experts": wl.MOE_EXPERTS, "routed_rows": wl.MOE_ROWS,
+                   "linears": {it["label"]: [it["M"], it["N"], it["K"]] for it in items},
+                   "l2": "no flush: the step's expert weights (470 + 235 MB) exceed the 126 MB L2"},
+        "gemm": {"kernel": "gemm_ue8m0_pair_kernel (grouped; timed with its two scale-pack kernels)",
+                 "achieved": gemm_tf, "peak": fp8_peak, "unit": "TFLOP/s", "frac": gemm_tf / fp8_peak,
+                 "ms_per_launch": d["gemm_ms"] / (args.steps * n),
+                 "traffic": recorded_traffic("gemm_ue8m0_pair_kernel", "deepseek_moe")},
+        "cpu_baseline": cpu, "parity": parity}}
+
+
 def run_moe(args):
     """Grouped (MoE expert) UE8M0 linears: one step = per expert linear (up,
     down), ue8m0 activation quantization of the routed rows + the grouped
@@ -451,37 +557,10 @@ def run_moe(args):
 
     hbm_peak, bf16_peak, peak_src = peaks()
     fp8_peak = bf16_peak * FP8_OVER_BF16
-    items = []
-    for name in ("up", "down"):
-        xb, off = wl.deepseek_moe(name)
-        N, K = wl.MOE_LINEARS[name]
-        E = wl.MOE_EXPERTS
-        w = wl.deepseek_moe_weights(name, dev)
-        q_w, s_w = fp8.quant_weight_ue8m0(w)
-        del w
-        M = xb.shape[0]
-        items.append(dict(label=name, xb=xb, x=wl.to_torch_bf16(xb).to(dev), off_np=off,
-                          off=torch.from_numpy(off).to(dev), q_w=q_w.view(E, N, K),
-                          s_w=s_w.view(E, N // 128, K // 128),
-                          q_a=torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev),
-                          s_a=torch.empty((M, K // 128), dtype=torch.float8_e8m0fnu, device=dev),
-                          y=torch.empty((M, N), dtype=torch.bfloat16, device=dev), M=M, N=N, K=K))
-        # the CTA-pair schedule's packed scale factors (allocated once, reused)
-        items[-1]["ws"] = torch.empty(max(fp8.grouped_ue8m0_workspace_bytes(M, N, K, E), 16),
-                                      dtype=torch.uint8, device=dev)
-    torch.cuda.synchronize()
+    items = moe_items(fp8, dev)
     flops_step = sum(2 * it["M"] * it["N"] * it["K"] for it in items)
     n = len(items)
-
-    def step(ev=None):
-        for i, it in enumerate(items):
-            fp8.quant_act_ue8m0(it["x"], it["q_a"], it["s_a"])
-            if ev is not None:
-                ev[2 * i].record()
-            fp8.grouped_linear_ue8m0(it["q_a"], it["s_a"], it["q_w"], it["s_w"], it["off"], it["y"],
-                                     workspace=it["ws"])
-            if ev is not None:
-                ev[2 * i + 1].record()
+    step = moe_step_fn(fp8, items)
 
     for _ in range(args.warmup):
         step()
@@ -542,23 +621,7 @@ def run_moe(args):
     if rank == 0:
         cpu = parity = None
         if world == 1 and not args.no_cpu:
-            t_tot, f_tot, worst = 0.0, 0.0, 0.0
-            g = np.random.default_rng(0)
-            for it in items:
-                rows = np.sort(g.choice(it["M"], args.cpu_rows, replace=False))
-                qw = it["q_w"].view(torch.uint8).cpu().numpy()
-                sw = it["s_w"].view(torch.uint8).cpu().numpy()
-                t, f, R = moe_oracle_rows(it["xb"], qw, sw, it["off_np"], rows)
-                t_tot += t
-                f_tot += f
-                Y = it["y"][torch.as_tensor(rows, device=dev)].float().cpu().numpy()
-                worst = max(worst, within_tolerance(Y, R))
-            cpu = {"value": f_tot / t_tot / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count() or 1,
-                   "kind": "oracle", "seconds": t_tot,
-                   "sample": f"{args.cpu_rows} random routed rows per expert linear (up, down): "
-                             "ue8m0 activation quant + fp64 grouped GEMM of those rows, all N columns"}
-            parity = {"rows_per_linear": args.cpu_rows, "within_tolerance": worst <= 1.0,
-                      "worst_bound_ratio": worst}
+            cpu, parity = moe_oracle_check(items, args.cpu_rows)
         line = {
             "metric": METRIC, "value": whole_job_rate(world, flops_step, args.steps, elapsed_ms) / 1e12,
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -599,8 +662,8 @@ def run_moe(args):
 #
 # The default run reports every workload of the build on the same JSON line:
 # besides the headline prefill step, `decode` (the 16 Llama-3-8B decode
-# linears and a whole layer per token count), `deepseek_mlp`, `sweep` and
-# `tiny`.  Each leg times on the device (CUDA events around CUDA-graph
+# linears and a whole layer per token count), `deepseek_mlp`, `sweep`,
+# `tiny` and `deepseek_moe` (the grouped expert linears).  Each leg times on the device (CUDA events around CUDA-graph
 # replays, max over ranks) and carries its roofline fraction, an oracle check
 # of sampled outputs and an oracle CPU baseline.
 L2_BYTES = 126e6
@@ -978,6 +1041,8 @@ def legs_json(legs, world, args, hbm_peak, fp8_peak, peak_src):
         out.update(sweep_json(legs["sweep"], cpu_ok, hbm_peak, fp8_peak))
     if "tiny" in legs:
         out.update(tiny_json(legs["tiny"], cpu_ok))
+    if "deepseek_moe" in legs:
+        out.update(moe_json(legs["deepseek_moe"], world, args, cpu_ok, fp8_peak, peak_src))
     return out
 
 
@@ -1337,6 +1402,8 @@ def run_ours(args):
             legs["sweep"] = leg_sweep(fp8, dev, barrier, args)
         if "tiny" in want:
             legs["tiny"] = leg_tiny(fp8, dev, barrier, args)
+        if "deepseek_moe" in want:
+            legs["deepseek_moe"] = leg_moe(fp8, dev, barrier, args)
     sampler.stop()
     fp8.check()
 
@@ -1360,6 +1427,9 @@ def run_ours(args):
             leg_slots += [(sw[k], "quant_ms"), (sw[k], "gemm_ms"), (sw[k], "fused_ms"), (sw[k], "fused_ik_ms")]
     if "tiny" in legs:
         leg_slots.append((legs["tiny"], "ms"))
+    if "deepseek_moe" in legs:
+        _, dm = legs["deepseek_moe"]
+        leg_slots += [(dm, "ms"), (dm, "gemm_ms")]
     maxed = max_over_ranks(times + [d[k] for d, k in leg_slots], dev, world)
     elapsed_ms, e2e_ms, act_ms, gemm_ms, fused_ms, fused_ik_ms_max = maxed[:6]
     fused_ik_ms = fused_ik_ms_max if fused_ik_ms is not None else None
@@ -1490,8 +1560,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch every step's kernels one by one")
     ap.add_argument("--no-legs", action="store_true",
-                    help="headline prefill step only (skip the decode, deepseek_mlp, sweep, tiny keys)")
-    ap.add_argument("--legs", default="decode,deepseek_mlp,sweep,tiny",
+                    help="headline prefill step only (skip the decode, deepseek_mlp, sweep, tiny, deepseek_moe keys)")
+    ap.add_argument("--legs", default="decode,deepseek_mlp,sweep,tiny,deepseek_moe",
                     help="comma-separated per-config legs to run with the prefill workload")
     ap.add_argument("--decode-launches", type=int, default=96,
                     help="timed launches per decode linear (rounded up to whole weight rotations)")
