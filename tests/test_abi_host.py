@@ -182,6 +182,50 @@ def test_grouped_argument_errors(lib):
     assert f(a, sa, w, sw, off, off, 4, 128, 128, 2, None) == 8      # y over the offsets
 
 
+def test_ue8m0_pair_workspace_sizes(lib):
+    """Workspace of the CTA-pair schedules: none at M <= 128; otherwise, per
+    K block, 512 bytes per packed group of 128 activation rows -- 2 per
+    256-row block, and for E > 1 every expert's segment padded to 256 rows,
+    bounded by 2 (ceil(M/256) + E) -- plus 512 bytes per 128-row weight
+    block (2 per 256 output columns) of every expert."""
+    fd = lib.fp8_block_linear_ue8m0_workspace_bytes
+    fd.argtypes = [ctypes.c_int64] * 3
+    fd.restype = ctypes.c_size_t
+    fg = lib.fp8_grouped_linear_ue8m0_workspace_bytes
+    fg.argtypes = [ctypes.c_int64] * 4
+    fg.restype = ctypes.c_size_t
+    cdiv = lambda a, b: -(-a // b)
+    for M, N, K in [(129, 128, 128), (4096, 28672, 4096), (4096, 4096, 14336), (300, 384, 512)]:
+        KB = K // 128
+        assert fd(M, N, K) == KB * 2 * cdiv(M, 256) * 512 + KB * 2 * cdiv(N, 256) * 512, (M, N, K)
+        assert fg(M, N, K, 1) == fd(M, N, K)
+    for M, N, K, E in [(8192, 4096, 7168, 16), (8192, 7168, 2048, 16), (300, 256, 256, 3),
+                       (4100, 256, 384, 256)]:
+        KB = K // 128
+        assert fg(M, N, K, E) == KB * 2 * (cdiv(M, 256) + E) * 512 + E * KB * 2 * cdiv(N, 256) * 512
+    assert fd(128, 4096, 4096) == 0 and fg(128, 4096, 4096, 8) == 0
+    assert fg(300, 256, 256, 0) == 0 and fg(300, 256, 256, 1025) == 0 and fg(300, 100, 256, 2) == 0
+
+
+def test_grouped_workspace_argument_errors(lib):
+    """fp8_grouped_linear_ue8m0_ws refuses a missing, short, misaligned or
+    overlapping workspace before touching the device (M > 128 needs one)."""
+    f = lib.fp8_grouped_linear_ue8m0_ws
+    f.argtypes = [V, V, V, V, V, V] + [ctypes.c_int64] * 4 + [V, ctypes.c_size_t, V]
+    fg = lib.fp8_grouped_linear_ue8m0_workspace_bytes
+    fg.argtypes = [ctypes.c_int64] * 4
+    fg.restype = ctypes.c_size_t
+    M, N, K, E = 300, 256, 256, 3
+    need = fg(M, N, K, E)
+    a, sa, w, sw, off, y, ws = (_p(0x10000000 * (i + 1)) for i in range(7))
+    assert f(a, sa, w, sw, off, y, M, N, K, E, None, 0, None) == 1            # no workspace
+    assert f(a, sa, w, sw, off, y, M, N, K, E, ws, need - 16, None) == 7      # too small
+    assert f(a, sa, w, sw, off, y, M, N, K, E, _p(0x70000008), need, None) == 3
+    assert f(a, sa, w, sw, off, y, M, N, K, E, y, need, None) == 8            # workspace over y
+    assert f(a, sa, w, sw, off, y, M, N, K, 0, ws, need, None) == 2           # E < 1
+    assert f(a, sa, w, sw, off, y, 0, N, K, E, None, 0, None) == 0           # empty
+
+
 def test_valid_call_without_gpu_reports_cuda_error(lib):
     """With no usable device the library answers FP8BL_ERR_CUDA (or ARCH on
     a non-B200 device) instead of crashing or falling back to the CPU."""
